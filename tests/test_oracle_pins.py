@@ -1,0 +1,350 @@
+"""Pins for the CPU oracle: checks against facts the pages and the mathematics fix.
+
+None of these re-types the oracle's own formula.  Each pins the oracle against
+something independent of it:
+
+* hand-derived worked examples of the page's packing formula (tests/golden),
+* the bitstream definition checked bit position by bit position with Python
+  integers,
+* exact-grid weights whose quantization is known in closed form,
+* the closed-form dequantization error bound,
+* exact rational arithmetic (fractions.Fraction) on tiny cases,
+* numpy's matmul on a dequantized weight decoded with library conversions,
+* the running-sum stress case whose result is known exactly,
+* the batch/stride invariants the pages' bug reports are about,
+* the probe error magnitude the issue reports.
+"""
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from group_wise_affine_qmv_b200 import inputs
+
+pytestmark = pytest.mark.filterwarnings("ignore::DeprecationWarning")
+
+
+# ---------------------------------------------------------------------------
+# library-side decoders (independent of the oracle's own converters)
+# ---------------------------------------------------------------------------
+
+def lib_half_to_f64(bits: np.ndarray, dtype: str) -> np.ndarray:
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    if dtype == "bf16":
+        return torch.from_numpy(b.view(np.int16).copy()).view(torch.bfloat16).to(torch.float64).numpy()
+    return b.view(np.float16).astype(np.float64)
+
+
+def lib_half_bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def parse_golden(path):
+    cases = []
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        head, words, codes = [p.strip() for p in line.split("|")]
+        bits, group = map(int, head.split())
+        cases.append((bits, group, np.array([int(w, 16) for w in words.split()], np.uint32),
+                      np.array([int(c) for c in codes.split()], np.uint8)))
+    return cases
+
+
+# ---------------------------------------------------------------------------
+# half-precision rounding helpers vs library conversions
+# ---------------------------------------------------------------------------
+
+def test_half_rounding_matches_library(orc):
+    rng = np.random.default_rng(0)
+    vals = np.concatenate([
+        rng.standard_normal(2000).astype(np.float32) * np.float32(3.0),
+        (rng.standard_normal(500) * 1e-6).astype(np.float32),   # fp16 subnormals
+        (rng.standard_normal(500) * 3e4).astype(np.float32),    # near fp16 max
+        np.array([0.0, -0.0, 1.0, 65504.0, 65519.0, 65520.0, 2.0 ** -24, 2.0 ** -25,
+                  3 * 2.0 ** -26, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8], np.float32),
+    ])
+    got_bf = orc.float_to_half_bits(vals, "bf16")
+    ref_bf = lib_half_bits(torch.from_numpy(vals).to(torch.bfloat16))
+    assert np.array_equal(got_bf, ref_bf)
+    got_h = orc.float_to_half_bits(vals, "f16")
+    ref_h = vals.astype(np.float16).view(np.uint16)
+    assert np.array_equal(got_h, ref_h)
+    # and decoding
+    assert np.array_equal(orc.half_to_double(ref_bf, "bf16"), lib_half_to_f64(ref_bf, "bf16"))
+    finite = np.isfinite(vals.astype(np.float16))
+    assert np.array_equal(orc.half_to_double(ref_h[finite], "f16"), lib_half_to_f64(ref_h[finite], "f16"))
+
+
+# ---------------------------------------------------------------------------
+# packing: page formula worked examples and the bitstream definition
+# ---------------------------------------------------------------------------
+
+def test_golden_pack_examples(orc, golden_dir):
+    cases = parse_golden(os.path.join(golden_dir, "pack_formula_examples.txt"))
+    assert len(cases) >= 10
+    for bits, group, words, codes in cases:
+        K = codes.size
+        assert np.array_equal(orc.pack(codes[None, :], bits)[0], words), (bits, group)
+        assert np.array_equal(orc.unpack(words[None, :], K, bits)[0], codes), (bits, group)
+        if bits in (2, 4, 8):
+            assert np.array_equal(orc.unpack_formula(words[None, :], K, group, bits)[0], codes)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+def test_bitstream_every_position_every_value(orc, bits):
+    """Code v at position i sets exactly stream bits [i*bits, (i+1)*bits) to v."""
+    K = 128
+    maxq = (1 << bits) - 1
+    values = np.arange(1, maxq + 1, dtype=np.uint8)
+    rows = []
+    expect = []
+    for i in range(K):
+        for v in values:
+            c = np.zeros(K, np.uint8)
+            c[i] = v
+            rows.append(c)
+            expect.append(int(v) << (i * bits))
+    codes = np.stack(rows)
+    packed = orc.pack(codes, bits)
+    for r in range(codes.shape[0]):
+        stream = sum(int(w) << (32 * j) for j, w in enumerate(packed[r]))
+        assert stream == expect[r]
+    assert np.array_equal(orc.unpack(packed, K, bits), codes)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("group", [32, 64, 128])
+def test_formula_equals_bitstream_random(orc, bits, group):
+    rng = np.random.default_rng(bits * 1000 + group)
+    K = 512
+    codes = rng.integers(0, 1 << bits, size=(7, K), dtype=np.uint8)
+    packed = orc.pack(codes, bits)
+    assert np.array_equal(orc.unpack_formula(packed, K, group, bits), codes)
+    assert np.array_equal(orc.unpack(packed, K, bits), codes)
+
+
+# ---------------------------------------------------------------------------
+# quantizer
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("group", [32, 64, 128])
+@pytest.mark.parametrize("sdtype", ["bf16", "f16"])
+def test_quantize_exact_grid(orc, bits, group, sdtype):
+    """W = s*q + b exactly, q spanning 0..2^bits-1 in every group: codes, s, b recovered."""
+    rng = np.random.default_rng(bits + 7 * group)
+    N, K = 5, 4 * group
+    maxq = (1 << bits) - 1
+    ng = K // group
+    s = (2.0 ** rng.integers(-6, 0, size=(N, ng))).astype(np.float32)   # powers of two
+    b = (rng.integers(-64, 64, size=(N, ng)) / 16.0).astype(np.float32)  # exact in bf16/f16
+    q = rng.integers(0, maxq + 1, size=(N, K)).astype(np.uint8)
+    q.reshape(N, ng, group)[:, :, 0] = 0
+    q.reshape(N, ng, group)[:, :, 1] = maxq
+    w = (np.repeat(s, group, axis=1) * q.astype(np.float32) + np.repeat(b, group, axis=1)).astype(np.float32)
+    # w is exact in fp32: |q| < 2^8, s a power of two, b on a 1/16 grid
+    Q = orc.quantize(w, group, bits, sdtype)
+    assert np.array_equal(Q.codes, q)
+    assert np.array_equal(Q.scale32, s)
+    assert np.array_equal(Q.bias32, b)
+    assert np.array_equal(lib_half_to_f64(Q.scale_bits, sdtype), s.astype(np.float64))
+    assert np.array_equal(lib_half_to_f64(Q.bias_bits, sdtype), b.astype(np.float64))
+    assert np.array_equal(Q.dequant(), w.astype(np.float64))
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("group", [32, 128])
+def test_quantize_error_bound(orc, bits, group):
+    """|w - w'| <= scale/2 + q*|scale - s_stored| + |bias - b_stored| (+ fp32 slack)."""
+    w = inputs.normal((33, 512), 1.0, seed=bits * 31 + group).numpy()
+    Q = orc.quantize(w, group, bits, "bf16")
+    maxq = (1 << bits) - 1
+    assert Q.codes.max() <= maxq
+    s32 = np.repeat(Q.scale32.astype(np.float64), group, axis=1)
+    b32 = np.repeat(Q.bias32.astype(np.float64), group, axis=1)
+    ss = np.repeat(lib_half_to_f64(Q.scale_bits, "bf16"), group, axis=1)
+    bs = np.repeat(lib_half_to_f64(Q.bias_bits, "bf16"), group, axis=1)
+    wd = Q.dequant()
+    bound = s32 / 2 + Q.codes * np.abs(s32 - ss) + np.abs(b32 - bs)
+    slack = 1e-6 * (np.abs(w) + s32 * maxq + np.abs(b32))
+    assert np.all(np.abs(w - wd) <= bound + slack)
+    # every group hits both ends of the code range (min -> 0, max -> maxq)
+    codes = Q.codes.reshape(33, -1, group)
+    assert np.all(codes.min(axis=2) == 0)
+    assert np.all(codes.max(axis=2) == maxq)
+    # bias is the group minimum exactly
+    assert np.array_equal(Q.bias32, w.reshape(33, -1, group).min(axis=2))
+
+
+def test_quantize_constant_group(orc):
+    w = np.full((3, 64), 0.75, np.float32)
+    w[1, 32:] = -2.5
+    Q = orc.quantize(w, 32, 4, "bf16")
+    assert np.all(Q.codes == 0)
+    assert np.all(Q.scale32 == 0)
+    assert np.array_equal(Q.bias32, np.array([[0.75, 0.75], [0.75, -2.5], [0.75, 0.75]], np.float32))
+    assert np.array_equal(Q.dequant(), w.astype(np.float64))
+
+
+# ---------------------------------------------------------------------------
+# contraction
+# ---------------------------------------------------------------------------
+
+def _exact_linear(x_bits, x_dtype, codes, sbits, bbits, group, sdtype):
+    xv = lib_half_to_f64(x_bits, x_dtype)
+    sv = lib_half_to_f64(sbits, sdtype)
+    bv = lib_half_to_f64(bbits, sdtype)
+    M, K = xv.shape
+    N = codes.shape[0]
+    out = np.empty((M, N), dtype=object)
+    for m in range(M):
+        for n in range(N):
+            acc = Fraction(0)
+            for k in range(K):
+                w = Fraction(float(sv[n, k // group])) * int(codes[n, k]) + Fraction(float(bv[n, k // group]))
+                acc += Fraction(float(xv[m, k])) * w
+            out[m, n] = acc
+    return out
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("x_dtype", ["bf16", "f16"])
+def test_linear_brute_force_exact(orc, bits, x_dtype):
+    """Tiny cases: oracle fp64 vs exact rational arithmetic."""
+    group, K, N, M = 32, 64, 3, 2
+    tdt = torch.bfloat16 if x_dtype == "bf16" else torch.float16
+    w = inputs.normal((N, K), 1.0, seed=bits).numpy()
+    x = inputs.normal((M, K), 1.0, tdt, seed=bits + 100)
+    xb = lib_half_bits(x)
+    Q = orc.quantize(w, group, bits, x_dtype)
+    y = orc.linear_contig(xb, x_dtype, Q.dequant())
+    ex = _exact_linear(xb, x_dtype, Q.codes, Q.scale_bits, Q.bias_bits, group, x_dtype)
+    mag = np.abs(lib_half_to_f64(xb, x_dtype)) @ np.abs(Q.dequant()).T
+    for m in range(M):
+        for n in range(N):
+            assert abs(Fraction(float(y[m, n])) - ex[m, n]) <= Fraction(1e-13) * Fraction(float(mag[m, n]) + 1e-300)
+    # the factored form s*sum(qx) + b*sum(x) is the same number
+    for m in range(M):
+        for n in range(N):
+            f = orc.factored_dot(xb[m], x_dtype, Q.codes[n], Q.scale_bits[n], Q.bias_bits[n], group, x_dtype)
+            assert abs(f - y[m, n]) <= 1e-12 * (mag[m, n] + 1e-300)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_linear_matches_numpy_matmul(orc, bits):
+    """Decode W with the page's word/shift formula in numpy and library half decoding,
+    multiply with numpy's matmul, compare to the oracle."""
+    group, K, N, M = 64, 512, 37, 5
+    w = inputs.normal((N, K), 0.02, seed=11).numpy()
+    x = inputs.normal((M, K), 1.0, torch.bfloat16, seed=12)
+    Q = orc.quantize(w, group, bits, "bf16")
+    per = 32 // bits
+    k = np.arange(K)
+    g, inG = k // group, k % group
+    idx = g * (group // per) + inG // per
+    shift = (inG % per) * bits
+    q = (Q.packed[:, idx] >> shift.astype(np.uint32)) & np.uint32((1 << bits) - 1)
+    s = lib_half_to_f64(Q.scale_bits, "bf16")[:, g]
+    b = lib_half_to_f64(Q.bias_bits, "bf16")[:, g]
+    wd = s * q.astype(np.float64) + b
+    ref = lib_half_to_f64(lib_half_bits(x), "bf16") @ wd.T
+    got = orc.linear_contig(lib_half_bits(x), "bf16", Q.dequant())
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_batch_invariants_probe(orc):
+    """[B,K], [1,S,K], [B,1,K] and [2,4,K] all equal the row-wise 2D result
+    (the shape table of transformers issue #47331)."""
+    w, _ = inputs.probe_case()
+    Q = orc.quantize(w.numpy(), 64, 4, "bf16")
+    wd = Q.dequant()
+    x = inputs.normal((8, 2048), 1.0, torch.bfloat16, seed=5)
+    xb = lib_half_bits(x)
+    flat = orc.linear_contig(xb, "bf16", wd)
+    for shape in [(8, 2048), (1, 8, 2048), (8, 1, 2048), (2, 4, 2048)]:
+        y = orc.linear_contig(xb.reshape(shape), "bf16", wd)
+        assert np.array_equal(y.reshape(8, -1), flat), shape
+
+
+def test_strided_views_equal_contiguous(orc):
+    """candle pitfall page: narrowed Q/K heads and the narrowed Linear4D input
+    must give what their contiguous() copies give, for every batch element."""
+    qkv, q, k = inputs.qkv_case()
+    assert q.stride() == (3840, 320, 64, 1) and k.stride() == (3840, 320, 64, 1)
+    base = lib_half_bits(qkv).ravel()
+    kq = orc.quantize(k.float().numpy(), 64, 8, "bf16")  # per-(b,h) weight bank [2,4,5,64]
+    wd = kq.dequant()
+    y_view = orc.linear(base, "bf16", q.shape, q.stride(), wd)
+    y_copy = orc.linear_contig(lib_half_bits(q.contiguous()), "bf16", wd)
+    assert np.array_equal(y_view, y_copy)
+    # the view must not behave like the single-stride batch of the buggy hosts
+    wrong = orc.linear(base, "bf16", (8, 5, 64), (320, 64, 1), wd.reshape(8, 5, 64))
+    assert not np.array_equal(wrong.reshape(2, 4, 5, 5)[1], y_copy[1])
+
+    xbase, x, w = inputs.linear4d_case()
+    assert x.stride() == (16896, 4224, 1408, 1)
+    Q = orc.quantize(w.numpy(), 32, 8, "bf16")
+    wd = Q.dequant()
+    y_view = orc.linear(lib_half_bits(xbase).ravel(), "bf16", x.shape, x.stride(), wd)
+    y_copy = orc.linear_contig(lib_half_bits(x.contiguous()), "bf16", wd)
+    assert np.array_equal(y_view, y_copy)
+
+
+@pytest.mark.parametrize("x_dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+def test_stress_running_sum_closed_form(orc, x_dtype, bits):
+    """mlx PR #4516: constant groups (scale 0, q 0, bias 1) make y = sum(x) exactly."""
+    K, N = 4096, 7
+    tdt = torch.bfloat16 if x_dtype == "bf16" else torch.float16
+    x = inputs.stress_x(K, 2, tdt)
+    Q = orc.quantize(inputs.stress_w(N, K).numpy(), 128, bits, x_dtype)
+    assert np.all(Q.codes == 0) and np.all(Q.scale32 == 0)
+    y = orc.linear_contig(lib_half_bits(x), x_dtype, Q.dequant())
+    small = 2.0 ** -9 if x_dtype == "bf16" else 2.0 ** -12
+    assert np.all(y == (K // 2) * (1.0 + small))
+
+
+def test_grouped_equals_per_expert(orc):
+    E, N, K = 4, 6, 64
+    w = inputs.normal((E, N, K), 0.02, seed=21).numpy()
+    Q = orc.quantize(w, 32, 8, "bf16")
+    wd = Q.dequant()
+    offsets = np.array([0, 3, 3, 7, 9], np.int64)
+    x = lib_half_bits(inputs.normal((9, K), 1.0, torch.bfloat16, seed=22))
+    y = orc.linear_grouped(x, "bf16", offsets, wd)
+    for e in range(E):
+        seg = slice(offsets[e], offsets[e + 1])
+        if offsets[e + 1] > offsets[e]:
+            assert np.array_equal(y[seg], orc.linear_contig(x[seg], "bf16", wd[e]))
+
+
+def test_sampled_equals_full(orc):
+    w = inputs.normal((40, 128), 0.02, seed=31).numpy()
+    Q = orc.quantize(w, 64, 4, "bf16")
+    wd = Q.dequant()
+    x = lib_half_bits(inputs.normal((6, 128), 1.0, torch.bfloat16, seed=32))
+    full = orc.linear_contig(x, "bf16", wd)
+    rows = np.array([0, 5, 3, 2], np.int64)
+    cols = np.array([39, 0, 17, 17], np.int64)
+    assert np.array_equal(orc.linear_sampled(x, "bf16", wd, rows, cols), full[rows, cols])
+
+
+def test_probe_error_magnitude_matches_issue(orc):
+    """transformers issue #47331 reports, for the 2D probe, a per-row error of
+    0.005-0.006 between a bf16 kernel (bf16 scales) and x @ dequant(W)^T built
+    with the fp32 scales.  The oracle with bf16 scales, rounded to bf16, must
+    show the same magnitude against that fp32-scale reference."""
+    w, xs = inputs.probe_case()
+    Q = orc.quantize(w.numpy(), 64, 4, "bf16")
+    ref_w = (np.repeat(Q.scale32.astype(np.float64), 64, axis=1) * Q.codes
+             + np.repeat(Q.bias32.astype(np.float64), 64, axis=1))
+    x = xs[0]
+    y = orc.linear_contig(lib_half_bits(x), "bf16", Q.dequant())
+    y_bf16 = torch.from_numpy(y).to(torch.bfloat16).double().numpy()
+    ref = orc.linear_contig(lib_half_bits(x), "bf16", ref_w)
+    err = np.abs(y_bf16 - ref).max(-1) / np.abs(ref).max(-1)
+    assert np.all((err > 0.002) & (err < 0.012)), err
