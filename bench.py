@@ -1,0 +1,478 @@
+#!/usr/bin/env python3
+"""Benchmark: decode sweep of a 28-layer 0.6B-class decoder through aq_qmm_t.
+
+One step = every projection of every layer (q, k, v, o, gate, up, down) plus
+lm_head, at a decode batch of 32 tokens (x [32, 1, K] bf16), for 4-bit AND
+8-bit weights (G = 64), all weights distinct and resident in HBM (1.07 GB per
+step, larger than L2, so every step streams its weights from HBM).  The step
+is captured once in a CUDA graph and replayed.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0.  `value` is whole-job HBM throughput in GB/s
+(algorithmic bytes: packed W + scales + biases + x + y of every call, each
+counted once) with inputs resident on the device; `e2e` is the same metric
+with the step's activations copied host->device and the logits copied back
+inside the timed region.  Multi-GPU runs are independent replicas (the
+operation has no exchange step on one layer): per-GPU work is fixed.
+The reference arm (--impl reference) times the CPU oracle on a bounded row
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from group_wise_affine_qmv_b200 import inputs  # noqa: E402
+
+METRIC = "W4/W8 qmm_t µs and HBM GB/s (% of peak) decode; prefill TFLOP/s (% bf16 peak)"
+GROUP = inputs.DECODE_GROUP
+BITS_LIST = (4, 8)
+FALLBACK_HBM_GBS = 6650.0
+
+
+def matrix_bytes(K, N, bits, M=inputs.DECODE_BATCH):
+    """Algorithmic bytes of one call: packed W + bf16 scales + bf16 biases + x + y (bf16)."""
+    return N * K * bits // 8 + 2 * 2 * N * (K // GROUP) + 2 * M * K + 2 * M * N
+
+
+def sweep_shapes(layers):
+    return inputs.decode_sweep_shapes(layers)
+
+
+def sweep_bytes(layers):
+    tot = 0
+    for bits in BITS_LIST:
+        for _, K, N in sweep_shapes(layers):
+            tot += matrix_bytes(K, N, bits)
+    return tot
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, else nvidia-smi)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.max_mhz = None
+        self.reasons = set()
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                if self._nvml is not None:
+                    p = self._nvml
+                    self.samples.append(p.nvmlDeviceGetClockInfo(self._h, p.NVML_CLOCK_SM))
+                    try:
+                        mask = p.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                    except Exception:
+                        mask = p.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                    for bit, name in self.REASONS.items():
+                        if mask & bit:
+                            self.reasons.add(name)
+                else:
+                    out = subprocess.run(
+                        ["nvidia-smi", f"--id={self.index}", "--query-gpu=clocks.sm,clocks.max.sm,"
+                         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                         "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5).stdout
+                    f = [v.strip() for v in out.strip().split(",")]
+                    self.samples.append(float(f[0]))
+                    self.max_mhz = float(f[1])
+                    for name, val in zip(["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                          "sw_power_cap"], f[2:]):
+                        if val.lower() == "active":
+                            self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.02)
+
+    def __enter__(self):
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self._thread.join(timeout=10)
+
+    def summary(self):
+        s = sorted(self.samples)
+        med = s[len(s) // 2] if s else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(s)}
+
+
+# ---------------------------------------------------------------------------
+# peaks and committed ncu traffic
+# ---------------------------------------------------------------------------
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def committed_traffic(kernel_tag: str):
+    """Per-launch DRAM bytes of `kernel_tag` from the committed ncu summary, if the
+    kernel source has not changed since the capture (source hash recorded there)."""
+    import hashlib
+    summ = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(summ):
+        return None
+    src_hash = hashlib.sha256()
+    for name in sorted(os.listdir(os.path.join(ROOT, "group_wise_affine_qmv_b200", "csrc"))):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(ROOT, "group_wise_affine_qmv_b200", "csrc", name), "rb") as f:
+                src_hash.update(f.read())
+    cur = src_hash.hexdigest()[:16]
+    for line in open(summ):
+        parts = line.split()
+        if len(parts) >= 3 and parts[0] == kernel_tag and parts[1] == cur:
+            try:
+                return float(parts[2])
+            except ValueError:
+                return None
+    return None
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def build_workload(device, layers):
+    from group_wise_affine_qmv_b200 import aq
+    mats = {}
+    seed = 1000
+    for bits in BITS_LIST:
+        lst = []
+        for name, K, N in sweep_shapes(layers):
+            seed += 1
+            w = inputs.decode_w(K, N, seed, device=device)
+            wq, sc, bi = aq.aq_quantize(w, GROUP, bits, scale_dtype=torch.bfloat16)
+            del w
+            lst.append((name, K, N, wq, sc, bi))
+        mats[bits] = lst
+    xs = {K: inputs.decode_x(K, seed=7 + K, device=device) for K in (1024, 3072)}
+    ys = {}
+    for bits in BITS_LIST:
+        ys[bits] = [torch.empty(inputs.DECODE_BATCH, 1, N, dtype=torch.bfloat16, device=device)
+                    for (_, _, N, _, _, _) in mats[bits]]
+    return mats, xs, ys
+
+
+def run_step(mats, xs, ys):
+    from group_wise_affine_qmv_b200 import aq
+    n = 0
+    for bits in BITS_LIST:
+        for (name, K, N, wq, sc, bi), y in zip(mats[bits], ys[bits]):
+            aq.aq_qmm_t(xs[K], wq, sc, bi, GROUP, bits, out=y)
+            n += 1
+    return n
+
+
+def cpu_baseline(layers, budget_s=12.0):
+    """The oracle as it stands, on a bounded row sample of the lm_head matrix (4-bit),
+    scaled to GB/s of algorithmic bytes."""
+    import numpy as np
+    import oracle
+    K, N = inputs.LM_HEAD[1], inputs.LM_HEAD[2]
+    rows = 4096
+    w = inputs.decode_w(K, rows, seed=424242)
+    x = inputs.decode_x(K, seed=7 + K).reshape(inputs.DECODE_BATCH, K)
+    Q = oracle.quantize(w.numpy(), GROUP, 4, "bf16")
+    xb = x.contiguous().view(torch.int16).numpy().view(np.uint16)
+    done_rows = 0
+    t0 = time.perf_counter()
+    chunk = 256
+    while time.perf_counter() - t0 < budget_s:
+        lo = done_rows % rows
+        codes = oracle.unpack(Q.packed[lo:lo + chunk], K, 4)
+        wd = oracle.dequant(codes, Q.scale_bits[lo:lo + chunk], Q.bias_bits[lo:lo + chunk], GROUP, "bf16")
+        oracle.linear_contig(xb, "bf16", wd)
+        done_rows += chunk
+    dt = time.perf_counter() - t0
+    bytes_done = done_rows * (K * 4 // 8 + 2 * 2 * (K // GROUP)) + 2 * inputs.DECODE_BATCH * (K + done_rows)
+    cores = len(os.sched_getaffinity(0))
+    return {"value": bytes_done / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done_rows} lm_head rows (K={K}, 4-bit, G={GROUP}) x 32 tokens: unpack + fp64 dequant "
+                      f"+ fp64 contraction, {dt:.1f} s"}
+
+
+def dist_setup(n_gpus):
+    if n_gpus > 1 or "RANK" in os.environ:
+        import datetime
+        import torch.distributed as dist
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, rank, world, local
+    torch.cuda.set_device(0)
+    return None, 0, 1, 0
+
+
+def max_over_ranks(dist, value, device):
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is not None:
+        dist.barrier(device_ids=[device.index])
+    torch.cuda.synchronize(device)
+
+
+def ours(args):
+    dist, rank, world, local = dist_setup(args.gpus)
+    device = torch.device("cuda", local)
+    layers = args.layers
+    mats, xs, ys = build_workload(device, layers)
+    launches_per_step = sum(len(v) for v in mats.values())
+    step_bytes = sweep_bytes(layers)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize(device)
+
+    # eager warm-up (also checks that every call succeeds), then capture one step
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            run_step(mats, xs, ys)
+    torch.cuda.synchronize(device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        run_step(mats, xs, ys)
+    torch.cuda.synchronize(device)
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            graph.replay()
+    torch.cuda.synchronize(device)
+
+    # ---- device-resident timing ----
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist, device)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            ev1.record(stream)
+        ev1.synchronize()
+    barrier(dist, device)
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(dist, ms, device)
+    ms_per_step = ms_max / args.steps
+    value = world * step_bytes * args.steps / (ms_max / 1e3) / 1e9
+
+    # ---- per-bits breakdown: the 28 layers, then lm_head alone after them ----
+    # (each lm_head call follows the layers' 288-683 MB of weights, so none of its
+    #  weights are left in L2 from the previous call)
+    from group_wise_affine_qmv_b200 import aq
+    detail = {}
+    reps = max(20, args.steps // 10)
+    for bits in BITS_LIST:
+        g_layers = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_layers, stream=stream):
+            for (name, K, N, wq, sc, bi), y in zip(mats[bits][:-1], ys[bits][:-1]):
+                aq.aq_qmm_t(xs[K], wq, sc, bi, GROUP, bits, out=y)
+        lm = mats[bits][-1]
+        glm = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(glm, stream=stream):
+            aq.aq_qmm_t(xs[lm[1]], lm[3], lm[4], lm[5], GROUP, bits, out=ys[bits][-1])
+        with torch.cuda.stream(stream):
+            g_layers.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                g_layers.replay()
+            e1.record(stream)
+            e1.synchronize()
+            layers_ms = e0.elapsed_time(e1) / reps
+            tl = 0.0
+            for _ in range(reps):
+                g_layers.replay()
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record(stream)
+                glm.replay()
+                a1.record(stream)
+                a1.synchronize()
+                tl += a0.elapsed_time(a1)
+        lm_us = tl / reps * 1e3
+        lm_bytes = matrix_bytes(lm[1], lm[2], bits)
+        lb = sum(matrix_bytes(K, N, bits) for (_, K, N, *_r) in mats[bits][:-1])
+        detail[f"w{bits}"] = {"layers_us": round(layers_ms * 1e3, 2), "layers_GBps": round(lb / layers_ms / 1e6, 1),
+                              "lm_head_us": round(lm_us, 2), "lm_head_GBps": round(lm_bytes / lm_us / 1e3, 1),
+                              "lm_head_frac_of_peak": None}
+        del g_layers, glm
+
+    # ---- end-to-end: activations H2D, graph, logits D2H, per step ----
+    x_host = {K: xs[K].cpu().pin_memory() for K in xs}
+    logits_host = {bits: torch.empty(ys[bits][-1].shape, dtype=torch.bfloat16).pin_memory() for bits in BITS_LIST}
+    h2d = sum(t.numel() * t.element_size() for t in x_host.values())
+    d2h = sum(t.numel() * t.element_size() for t in logits_host.values())
+    e2e_steps = max(3, args.steps // 4)
+    barrier(dist, device)
+    with torch.cuda.stream(stream):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            for K in xs:
+                xs[K].copy_(x_host[K], non_blocking=True)
+            graph.replay()
+            for bits in BITS_LIST:
+                logits_host[bits].copy_(ys[bits][-1], non_blocking=True)
+        f1.record(stream)
+    f1.synchronize()
+    barrier(dist, device)
+    e2e_ms = max_over_ranks(dist, f0.elapsed_time(f1), device)
+    e2e_value = world * step_bytes * e2e_steps / (e2e_ms / 1e3) / 1e9
+
+    peak, peak_kind = hbm_peak()
+    for bits in BITS_LIST:
+        detail[f"w{bits}"]["lm_head_frac_of_peak"] = round(detail[f"w{bits}"]["lm_head_GBps"] / peak, 4)
+    per_launch_bytes = step_bytes / launches_per_step
+    per_launch_s = (ms / 1e3) / args.steps / launches_per_step
+    achieved = per_launch_bytes / per_launch_s / 1e9
+    traffic = committed_traffic("qmm_t_decode_sweep")
+
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) weights quantized on the device, N(0,1) activations)",
+        "config": {"workload": "decode sweep: 28 layers x (q,k,v,o,gate,up,down) + lm_head, x [32,1,K] bf16, "
+                               "bits 4 and 8, G=64",
+                   "tokens": inputs.DECODE_BATCH, "layers": layers, "bits": list(BITS_LIST), "group": GROUP,
+                   "bytes_per_step": step_bytes, "l2": "inputs larger than L2 (weights streamed from HBM each step)",
+                   "graph": "one CUDA graph per step", "parallelism": f"replicas x{world}"},
+        "detail": detail,
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "kernel": "aq_qmm_t (all launches of the step)", "peak_source": peak_kind},
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(layers)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    del graph
+    if dist is not None:
+        dist.barrier(device_ids=[device.index])
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle, as it stands, on a bounded sample per step
+# ---------------------------------------------------------------------------
+
+def reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    layers = args.layers
+    # per step: a bounded row sample of every matrix shape of the sweep, 4- and 8-bit
+    shapes = sorted({(K, N) for _, K, N in sweep_shapes(layers)})
+    rows_per_matrix = 8
+    prepared = []
+    for bits in BITS_LIST:
+        for (K, N) in shapes:
+            w = inputs.decode_w(K, rows_per_matrix, seed=K * 7 + N + bits)
+            Q = oracle.quantize(w.numpy(), GROUP, bits, "bf16")
+            x = inputs.decode_x(K, seed=7 + K).reshape(inputs.DECODE_BATCH, K)
+            prepared.append((bits, K, Q, x.contiguous().view(torch.int16).numpy().view(np.uint16)))
+
+    def step():
+        b = 0
+        for bits, K, Q, xb in prepared:
+            codes = oracle.unpack(Q.packed, K, bits)
+            wd = oracle.dequant(codes, Q.scale_bits, Q.bias_bits, GROUP, "bf16")
+            oracle.linear_contig(xb, "bf16", wd)
+            b += rows_per_matrix * (K * bits // 8 + 4 * (K // GROUP)) + 2 * inputs.DECODE_BATCH * (K + rows_per_matrix)
+        return b
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    t0 = time.perf_counter()
+    tot = 0
+    for _ in range(args.steps):
+        tot += step()
+    dt = time.perf_counter() - t0
+    value = tot / dt / 1e9
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"{rows_per_matrix} rows of each of the {len(shapes)} matrix shapes of the sweep, bits 4 and 8, "
+              f"x 32 tokens per step")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": "decode sweep row sample (CPU oracle)", "layers": layers},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=inputs.DECODE_LAYERS)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        reference(args)
+    else:
+        ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,81 @@
+// aq_internal.h -- shared declarations between the host dispatcher and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "aq.h"
+
+namespace aq {
+
+// Element types of x / scales / biases (16-bit) and of y.
+enum class DT : int { F32 = AQ_F32, BF16 = AQ_BF16, F16 = AQ_F16 };
+
+// ---------------------------------------------------------------------------
+// CUDA-core GEMV (qmv) arguments.  One launch batch per blockIdx.y; inside a
+// launch batch, M rows of x (row stride x_row) against N rows of W.
+// ---------------------------------------------------------------------------
+struct QmvArgs {
+    const void* x;
+    const uint32_t* wq;
+    const void* scales;
+    const void* biases;
+    void* y;
+    int64_t x_row, y_row;          // elements between consecutive rows of x / y
+    int64_t w_row, s_row, b_row;   // row strides of W (words), scales, biases (elements)
+    int64_t M, N, K;
+    int log2g;                     // log2(group)
+    int xvec;                      // 1: x rows 16-byte aligned (vector loads allowed)
+    int64_t bshape1;               // size of the inner launch-batch dim (1 if none)
+    int64_t xb[2], yb[2], wb[2], sb[2], bb[2];  // launch-batch strides (outer, inner)
+};
+
+// Launches the GEMV kernel for `nbatch` launch batches.  Returns cudaSuccess or the launch error.
+cudaError_t launch_qmv(const QmvArgs& a, int bits, DT xdt, DT ydt, int64_t nbatch, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// Quantize / dequantize.
+// ---------------------------------------------------------------------------
+struct QuantArgs {
+    const void* w;        // [N, K] (quantize input / dequantize output)
+    uint32_t* wq;         // [N, K*bits/32]
+    void* scales;         // [N, K/G]
+    void* biases;
+    int64_t w_row, wq_row, s_row, b_row;
+    int64_t N, K;
+    int group, bits;
+};
+cudaError_t launch_quantize(const QuantArgs& a, DT wdt, DT sdt, cudaStream_t s);
+cudaError_t launch_dequantize(const QuantArgs& a, DT wdt, DT sdt, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// tcgen05 tensor-core kernel (A = dequantized W in TMEM, B = x tile in SMEM).
+// ---------------------------------------------------------------------------
+struct MmaProblem {
+    // x viewed as [nb0, nb1, M, K] (strides in elements); y likewise with N.
+    const void* x;
+    void* y;
+    const uint32_t* wq;
+    const void* scales;
+    const void* biases;
+    int64_t M, N, K;
+    int64_t x_row, y_row;
+    int64_t nb[2];              // launch batch dims (outer, inner), 1 if absent
+    int64_t xb[2], yb[2];
+    int64_t w_row;              // words
+    int group, bits;
+    DT xdt, ydt;
+    // grouped (mixture-of-experts) mode: offsets != nullptr
+    const int64_t* offsets;     // device, n_experts + 1
+    int n_experts;
+    int64_t w_expert, s_expert, b_expert;  // per-expert strides (words / elements)
+};
+
+// Whether the tensor-core kernel can run this problem (alignment, bits, K), and why not.
+bool mma_supported(const MmaProblem& p, const char** why);
+cudaError_t launch_mma(const MmaProblem& p, cudaStream_t s);
+
+// Device-side error word (set by kernels whose bounded waits expire).
+cudaError_t read_and_clear_device_error(int* value, cudaStream_t s);
+
+}  // namespace aq

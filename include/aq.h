@@ -1,0 +1,211 @@
+/*
+ * aq.h -- C ABI of libaq: affine group-quantized linear layers on B200 (sm_100a).
+ *
+ *     y = x . dequant(W)^T,   dequant(W)[n, k] = scale[n, k/G] * q[n, k] + bias[n, k/G]
+ *
+ * The operation, as the pages define it:
+ *  - "MetalConfig quantization: batched generate silently corrupts all rows
+ *    after the first" (transformers issue #47331), probe script and shape
+ *    table: affine_qmm_t(x, w_packed, scales, biases, group, bits) must equal
+ *    x @ dequant(W)^T row by row for every input shape -- [B, K], [1, S, K],
+ *    [B, 1, K], [2, 4, K] -- i.e. leading batch dims are real batch dims.
+ *  - "Metal Kernel Bits=8 Final Report", section 3.1: W [outDim, inDim*bits/32]
+ *    uint32 with 32/bits codes per word, code inG of group g at word
+ *    g*(G/(32/bits)) + inG/(32/bits), shift (inG % (32/bits))*bits; scales
+ *    [outDim, inDim/G] (and G is inDim / scales.shape[-1]).
+ *  - 3/5/6-bit codes: a dense little-endian bitstream per row, code i at bit
+ *    i*bits of the row's uint32 words (the same rule the power-of-two formula
+ *    is a special case of).
+ *  - "mlx PR #4516": the bias term bias * sum(x) is formed from inputs widened
+ *    to fp32 before they are added; rows past the end of the last row tile
+ *    cost no per-row check inside the reduction loop.
+ *  - candle "Metal batched matmul" pitfall page: strided batch views (narrowed
+ *    Q/K heads, narrowed Linear inputs) are handled from EVERY batch stride,
+ *    never from stride[-3] alone; uniform batch strides fold into rows.
+ *
+ * Conventions for every entry point:
+ *  - All tensor arguments are aq_view descriptors of DEVICE memory owned by
+ *    the caller.  The library allocates no memory, never synchronizes the
+ *    stream, and keeps no pointer after the call returns.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream) of the current
+ *    device; work is enqueued on it and runs asynchronously.
+ *  - Strides are in ELEMENTS, may be any non-negative value, and the innermost
+ *    stride of every view must be 1.
+ *  - Arguments are validated on the host before any launch; on error nothing
+ *    is launched and a status != AQ_OK is returned (never an abort).
+ *    aq_status_string() names the status; aq_last_error_message() gives a
+ *    one-line detail of the most recent failure on the calling thread.
+ *  - Kernels never trap.  A kernel whose internal pipeline wait exceeds its
+ *    bound records a device-side error instead; aq_device_error() reads and
+ *    clears it (this one call synchronizes the stream).
+ */
+#ifndef AQ_H
+#define AQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum aq_status {
+    AQ_OK = 0,
+    AQ_ERR_NULL = 1,         /* a required pointer (view or data) is NULL            */
+    AQ_ERR_DTYPE = 2,        /* dtype not allowed or dtypes disagree                 */
+    AQ_ERR_RANK = 3,         /* view rank outside the allowed range                  */
+    AQ_ERR_SHAPE = 4,        /* shapes inconsistent with each other / K, N, G, bits  */
+    AQ_ERR_STRIDE = 5,       /* innermost stride != 1, or a negative stride          */
+    AQ_ERR_BITS = 6,         /* bits not in {2, 3, 4, 5, 6, 8}                       */
+    AQ_ERR_GROUP = 7,        /* group not in {32, 64, 128}, or K % group != 0        */
+    AQ_ERR_ALIGN = 8,        /* a data pointer is not 16-byte aligned                */
+    AQ_ERR_UNSUPPORTED = 9,  /* valid request the library does not implement         */
+    AQ_ERR_OVERLAP = 10,     /* the output overlaps an input                         */
+    AQ_ERR_CUDA = 11,        /* a CUDA runtime/driver call or a launch failed        */
+    AQ_ERR_DEVICE = 12,      /* current device is not an sm_100 (B200-class) GPU     */
+    AQ_ERR_TIMEOUT = 13      /* a kernel's bounded pipeline wait expired (device)    */
+} aq_status;
+
+typedef enum aq_dtype {
+    AQ_F32 = 0,
+    AQ_BF16 = 1,
+    AQ_F16 = 2,
+    AQ_U32 = 3
+} aq_dtype;
+
+/* A strided view of device memory: element (i0, .., i{rank-1}) lives at
+ * data + sum_j i_j * stride[j] elements.  Entries past `rank` are ignored. */
+typedef struct aq_view {
+    void* data;
+    int32_t dtype;      /* aq_dtype */
+    int32_t rank;
+    int64_t shape[4];
+    int64_t stride[4];  /* in elements */
+} aq_view;
+
+/*
+ * aq_quantize -- group-wise affine quantization of W.
+ *   For each row n and group g of `group` consecutive K elements, in IEEE
+ *   fp32: scale = (max - min) / (2^bits - 1), bias = min,
+ *   q = clamp(rint((w - bias) / scale), 0, 2^bits - 1) (ties to even; a
+ *   constant group has scale 0 and every q = 0); the stored scale and bias are
+ *   then rounded to nearest-even in the dtype of `scales`/`biases`.
+ *   (transformers issue #47331 probe script: quantize the fp32 W, then convert
+ *   scales/biases to bf16.)
+ * w:      [N, K] AQ_F32, AQ_BF16 or AQ_F16 (rank 2; rows may be strided).
+ * wq:     [N, K*bits/32] AQ_U32 out, packed as described at the top.
+ * scales: [N, K/group] AQ_BF16 or AQ_F16 out; biases: same shape and dtype.
+ * W must be finite; NaN/Inf inputs give unspecified codes.
+ */
+aq_status aq_quantize(const aq_view* w, int group, int bits, const aq_view* wq,
+                      const aq_view* scales, const aq_view* biases, void* stream);
+
+/*
+ * aq_dequantize -- w_out[n, k] = scale[n, k/G] * q[n, k] + bias[n, k/G],
+ *   evaluated in fp32 and rounded once to the dtype of w_out.
+ * wq [N, K*bits/32] AQ_U32; scales/biases [N, K/group] AQ_BF16|AQ_F16;
+ * w_out [N, K] AQ_F32, AQ_BF16 or AQ_F16.  All rank 2.
+ */
+aq_status aq_dequantize(const aq_view* wq, const aq_view* scales, const aq_view* biases,
+                        int group, int bits, const aq_view* w_out, void* stream);
+
+/*
+ * aq_qmm_t -- y = x . dequant(W)^T for any number of rows.
+ * x:      rank 1..4, [..., M, K], AQ_BF16 or AQ_F16, any batch/row strides.
+ *         Batch dims whose strides are uniform (stride[i] == stride[i+1] *
+ *         shape[i+1] for x and y) fold into rows; the others are real batch
+ *         dims whose offsets come from every one of their strides.
+ * wq:     [..., N, K*bits/32] AQ_U32 with 0..2 batch dims that are 1
+ *         (shared weight) or equal to x's corresponding batch dims
+ *         (right-aligned, as in broadcasting).
+ * scales, biases: [..., N, K/group], same dtype as x, same batch dims as wq.
+ * y:      x.shape[:-1] + [N], dtype of x or AQ_F32, must not overlap inputs.
+ * bits in {2,3,4,5,6,8}; group in {32,64,128}; K % group == 0.
+ * Rows per launch decide the kernel: a CUDA-core GEMV for a handful of rows,
+ * a tcgen05/TMEM tensor-core kernel above that.  Data pointers must be
+ * 16-byte aligned.
+ */
+aq_status aq_qmm_t(const aq_view* x, const aq_view* wq, const aq_view* scales,
+                   const aq_view* biases, int group, int bits, const aq_view* y, void* stream);
+
+/*
+ * aq_qmv -- same contract as aq_qmm_t, but always runs the CUDA-core GEMV
+ * kernel (128-bit weight loads, in-register unpack, fp32 s*sum(q*x) +
+ * b*sum(x) with inputs widened before every sum, warp-shuffle reduction,
+ * partial-rows tail without per-row checks in the loop).  Rows are processed
+ * a few at a time, so large M re-reads W.
+ */
+aq_status aq_qmv(const aq_view* x, const aq_view* wq, const aq_view* scales,
+                 const aq_view* biases, int group, int bits, const aq_view* y, void* stream);
+
+/*
+ * aq_qmm_t_grouped -- mixture-of-experts bank:
+ *   y_sorted[t] = x_sorted[t] . dequant(W_e)^T  for offsets[e] <= t < offsets[e+1].
+ * x_sorted: [T, K] AQ_BF16|AQ_F16 (rows grouped by expert, row stride free).
+ * offsets:  DEVICE pointer to n_experts+1 int64, non-decreasing, offsets[0] = 0,
+ *           offsets[n_experts] = T (not checked on the host: it lives on the device).
+ * wq_bank [E, N, K*bits/32] AQ_U32; s_bank, b_bank [E, N, K/group].
+ * y_sorted: [T, N], dtype of x or AQ_F32.
+ * (Prior art: the gathered QMV of "mlx PR #4516"; expert shapes from "Metal
+ * Kernel Bits=8 Final Report", section 4.3.)
+ */
+aq_status aq_qmm_t_grouped(const aq_view* x_sorted, const int64_t* offsets, int n_experts,
+                           const aq_view* wq_bank, const aq_view* s_bank, const aq_view* b_bank,
+                           int group, int bits, const aq_view* y_sorted, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Introspection (host only, no GPU work).                                 */
+/* ---------------------------------------------------------------------- */
+
+typedef enum aq_regime {
+    AQ_REGIME_QMV = 0,   /* CUDA-core GEMV                      */
+    AQ_REGIME_MMA = 1    /* tcgen05 tensor-core kernel (TMEM)   */
+} aq_regime;
+
+/* How a call will be executed: the result of view resolution and batch folding. */
+typedef struct aq_plan {
+    int32_t regime;            /* aq_regime                                            */
+    int32_t w_batched;         /* 1 if W has a non-broadcast batch dim                 */
+    int64_t M;                 /* rows per launch batch after folding                  */
+    int64_t N, K;
+    int32_t nbatch_dims;       /* launch batch dims left after folding (0..2)         */
+    int32_t pad_;
+    int64_t batch_shape[2];    /* outer first                                          */
+    int64_t x_batch_stride[2];
+    int64_t y_batch_stride[2];
+    int64_t w_batch_stride[2]; /* 0 where W broadcasts                                 */
+    int64_t s_batch_stride[2];
+    int64_t b_batch_stride[2];
+    int64_t x_row_stride;      /* elements between folded rows                         */
+    int64_t y_row_stride;
+    int64_t total_rows;        /* product of batch_shape * M                           */
+} aq_plan;
+
+/*
+ * Resolve views, fold batch dims and pick the kernel exactly as aq_qmm_t
+ * (force_qmv = 0) or aq_qmv (force_qmv = 1) would, without launching
+ * anything.  Data pointers are checked for NULL and alignment only.
+ */
+aq_status aq_plan_linear(const aq_view* x, const aq_view* wq, const aq_view* scales,
+                         const aq_view* biases, int group, int bits, const aq_view* y,
+                         int force_qmv, aq_plan* out);
+
+const char* aq_status_string(aq_status status);
+
+/* One-line description of the last error returned on the calling thread ("" if none). */
+const char* aq_last_error_message(void);
+
+/*
+ * Reads and clears the device-side error word of the current device after
+ * synchronizing `stream`.  Returns AQ_OK if no kernel recorded an error,
+ * AQ_ERR_TIMEOUT if a bounded wait expired, AQ_ERR_CUDA if the read failed.
+ */
+aq_status aq_device_error(void* stream);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int aq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AQ_H */

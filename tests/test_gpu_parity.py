@@ -1,0 +1,223 @@
+"""GPU parity: libaq (through the C ABI) against the CPU oracle, element by element.
+
+Inputs are seeded synthetic draws from group_wise_affine_qmv_b200.inputs; every
+quantized weight fed to a contraction is produced by the ORACLE quantizer, so
+no oracle input comes from the CUDA path.  Bars:
+* packing and codes: bit-exact; stored scales/biases: equal values;
+* contractions: per-row max|y-ref|/max|ref| <= 4e-3 for half outputs, every
+  row of every batch element (transformers issue #47331 probe metric);
+* running-sum stress: the exact bias*sum(x) value within 1e-6 relative in fp32
+  (mlx PR #4516).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from group_wise_affine_qmv_b200 import aq, inputs
+from tests.parity import (assert_rows_close, dtype_name, half_bits, oracle_linear_view, row_errors,
+                          to_device_quant)
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+DEV = "cuda"
+
+
+def _q(w: torch.Tensor, group: int, bits: int, sdtype: str = "bf16"):
+    Q = oracle.quantize(w.float().numpy(), group, bits, sdtype)
+    tdt = torch.bfloat16 if sdtype == "bf16" else torch.float16
+    return Q, to_device_quant(Q, DEV, tdt)
+
+
+# ---------------------------------------------------------------------------
+# quantize / dequantize
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("group", [32, 64, 128])
+@pytest.mark.parametrize("sdtype", ["bf16", "f16"])
+def test_quantize_bit_exact(bits, group, sdtype):
+    w = inputs.normal((67, 512), 1.0, seed=bits * 100 + group)
+    w[3, :group] = 0.25  # one constant group
+    Q = oracle.quantize(w.numpy(), group, bits, sdtype)
+    tdt = torch.bfloat16 if sdtype == "bf16" else torch.float16
+    wq, sc, bi = aq.aq_quantize(w.to(DEV), group, bits, scale_dtype=tdt)
+    torch.cuda.synchronize()
+    assert np.array_equal(wq.cpu().numpy().view(np.uint32), Q.packed)
+    assert np.array_equal(sc.float().cpu().numpy(), oracle.half_to_double(Q.scale_bits, sdtype).astype(np.float32))
+    assert np.array_equal(bi.float().cpu().numpy(), oracle.half_to_double(Q.bias_bits, sdtype).astype(np.float32))
+
+
+@pytest.mark.parametrize("wdtype", [torch.bfloat16, torch.float16])
+def test_quantize_half_input(wdtype):
+    w = inputs.normal((40, 256), 0.02, dtype=wdtype, seed=9)
+    Q = oracle.quantize(w.float().numpy(), 64, 4, "bf16")
+    wq, sc, bi = aq.aq_quantize(w.to(DEV), 64, 4, scale_dtype=torch.bfloat16)
+    assert np.array_equal(wq.cpu().numpy().view(np.uint32), Q.packed)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+def test_dequantize_matches_oracle(bits):
+    w = inputs.normal((33, 384), 1.0, seed=bits)
+    Q, (wq, sc, bi) = _q(w, 32, bits)
+    out = aq.aq_dequantize(wq, sc, bi, 32, bits, torch.float32).cpu().double().numpy()
+    ref = Q.dequant()
+    # one fp32 fma rounding
+    assert np.all(np.abs(out - ref) <= 2.0 ** -23 * np.abs(ref) + 1e-30)
+
+
+# ---------------------------------------------------------------------------
+# probe (issue #47331): [2,K], [2,1,K], [2,4,K] -- every row of every batch element
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("entry", ["aq_qmm_t", "aq_qmv"])
+def test_probe_every_row(entry):
+    w, xs = inputs.probe_case()
+    Q, (wq, sc, bi) = _q(w, 64, 4)
+    wd = Q.dequant()
+    fn = getattr(aq, entry)
+    for x in xs:
+        y = fn(x.to(DEV), wq, sc, bi, 64, 4)
+        ref = oracle_linear_view(x, wd)
+        err = row_errors(y, ref)
+        assert err.size == x.numel() // x.shape[-1]
+        assert np.all(err <= 4e-3), (tuple(x.shape), err)
+
+
+def test_probe_batched_equals_flat_bitwise():
+    """[B,1,K] and [2,4,K] give exactly the bits of the flattened 2D call."""
+    w, _ = inputs.probe_case()
+    _, (wq, sc, bi) = _q(w, 64, 4)
+    x = inputs.normal((8, 2048), 1.0, torch.bfloat16, seed=17).to(DEV)
+    flat = aq.aq_qmm_t(x, wq, sc, bi, 64, 4)
+    for shape in [(8, 1, 2048), (2, 4, 2048), (1, 8, 2048)]:
+        y = aq.aq_qmm_t(x.view(shape), wq, sc, bi, 64, 4)
+        assert torch.equal(y.reshape(8, -1), flat), shape
+
+
+# ---------------------------------------------------------------------------
+# ragged-output qmv and the stress case (config: bits 2/3/5/6, G 32/128, K 4096)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", inputs.RAGGED_BITS)
+@pytest.mark.parametrize("group", inputs.RAGGED_GROUPS)
+@pytest.mark.parametrize("N", inputs.RAGGED_N)
+def test_ragged_qmv(bits, group, N):
+    for xi, x_shape in enumerate(inputs.RAGGED_X_SHAPES):
+        w, x = inputs.ragged_case(bits, group, N, x_shape, seed=bits * 7 + group + N + 1000 * xi)
+        Q, (wq, sc, bi) = _q(w, group, bits)
+        wd = Q.dequant()
+        y = aq.aq_qmm_t(x.to(DEV), wq, sc, bi, group, bits)
+        ref = oracle_linear_view(x, wd)
+        assert_rows_close(y, ref, x, wd)
+
+
+@pytest.mark.parametrize("xdtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("group", [32, 128])
+@pytest.mark.parametrize("rows", [1, 4])
+def test_running_sum_stress_exact(xdtype, bits, group, rows):
+    """Constant groups (scale 0, q 0, bias 1): y = sum(x) exactly, in fp32 output."""
+    K = 4096
+    sd = dtype_name(torch.empty(0, dtype=xdtype))
+    for N in inputs.RAGGED_N:
+        Q, (wq, sc, bi) = _q(inputs.stress_w(N, K), group, bits, sd)
+        assert np.all(Q.codes == 0)
+        x = inputs.stress_x(K, rows, xdtype).to(DEV)
+        y = aq.aq_qmm_t(x.view(rows, 1, K) if rows > 1 else x, wq, sc, bi, group, bits, out_dtype=torch.float32)
+        small = 2.0 ** -9 if xdtype == torch.bfloat16 else 2.0 ** -12
+        exact = (K // 2) * (1.0 + small)
+        got = y.double().cpu().numpy()
+        assert np.all(np.abs(got - exact) <= 1e-6 * exact), (N, got.ravel()[:4], exact)
+
+
+# ---------------------------------------------------------------------------
+# strided batched views (candle pitfall page)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_qk_scores_strided(bits):
+    """scores = Q . K^T per (b, h) with K quantized (G = head_dim = 64) as a batched bank."""
+    qkv, q, k = inputs.qkv_case()
+    Q, (wq, sc, bi) = _q(k.float().contiguous().reshape(-1, 64), 64, bits)
+    wq = wq.view(2, 4, 5, -1)
+    sc = sc.view(2, 4, 5, 1)
+    bi = bi.view(2, 4, 5, 1)
+    wd = Q.dequant().reshape(2, 4, 5, 64)
+    qkv_d = qkv.to(DEV)
+    q_d = qkv_d.narrow(1, 0, 4)
+    assert q_d.stride() == (3840, 320, 64, 1)
+    y = aq.aq_qmm_t(q_d, wq, sc, bi, 64, bits)
+    ref = oracle_linear_view(q, wd)
+    err = row_errors(y, ref)
+    assert np.all(err <= 4e-3), err
+    # the contiguous copy gives the same bits, batch by batch, head by head
+    y_c = aq.aq_qmm_t(q_d.contiguous(), wq, sc, bi, 64, bits)
+    for b in range(2):
+        for h in range(4):
+            assert torch.equal(y[b, h], y_c[b, h]), (b, h)
+
+
+@pytest.mark.parametrize("entry", ["aq_qmm_t", "aq_qmv"])
+def test_linear4d_narrowed(entry):
+    base, x, w = inputs.linear4d_case()
+    Q, (wq, sc, bi) = _q(w, 32, 8)
+    wd = Q.dequant()
+    base_d = base.to(DEV)
+    x_d = base_d.narrow(1, 0, 2)
+    fn = getattr(aq, entry)
+    y = fn(x_d, wq, sc, bi, 32, 8)
+    ref = oracle_linear_view(x, wd)
+    assert np.all(row_errors(y, ref) <= 4e-3)
+    y_c = fn(x_d.contiguous(), wq, sc, bi, 32, 8)
+    for b0 in range(2):
+        for b1 in range(2):
+            assert torch.equal(y[b0, b1], y_c[b0, b1])
+
+
+# ---------------------------------------------------------------------------
+# edge cases
+# ---------------------------------------------------------------------------
+
+def test_empty_rows_launch_nothing():
+    w = inputs.normal((64, 256), 1.0, seed=1)
+    _, (wq, sc, bi) = _q(w, 64, 4)
+    x = torch.empty(0, 256, dtype=torch.bfloat16, device=DEV)
+    y = aq.aq_qmm_t(x, wq, sc, bi, 64, 4)
+    assert y.shape == (0, 64)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+def test_output_canaries_untouched(bits):
+    """Writes stay inside y: guard regions before/after and between strided rows keep their value."""
+    N, K, M = 37, 256, 3
+    w = inputs.normal((N, K), 1.0, seed=bits + 50)
+    Q, (wq, sc, bi) = _q(w, 64, bits)
+    x = inputs.normal((M, K), 1.0, torch.bfloat16, seed=51).to(DEV)
+    buf = torch.full((M + 2, N + 8), 12345.0, dtype=torch.bfloat16, device=DEV)
+    y = buf[1:M + 1, 4:4 + N]
+    aq.aq_qmm_t(x, wq, sc, bi, 64, bits, out=y)
+    b = buf.float().cpu()
+    assert torch.all(b[0] == 12345.0) and torch.all(b[-1] == 12345.0)
+    assert torch.all(b[:, :4] == 12345.0) and torch.all(b[:, 4 + N:] == 12345.0)
+    ref = oracle_linear_view(x.cpu(), Q.dequant())
+    assert np.all(row_errors(y, ref) <= 4e-3)
+
+
+def test_minimal_k_and_single_row():
+    w = inputs.normal((1, 32), 1.0, seed=77)
+    Q, (wq, sc, bi) = _q(w, 32, 4)
+    x = inputs.normal((1, 32), 1.0, torch.bfloat16, seed=78)
+    y = aq.aq_qmm_t(x.to(DEV), wq, sc, bi, 32, 4, out_dtype=torch.float32)
+    ref = oracle_linear_view(x, Q.dequant())
+    assert abs(float(y.item()) - ref.item()) <= 1e-5 * max(1.0, abs(ref.item()))
+
+
+def test_f16_activations():
+    w = inputs.normal((300, 1024), 0.02, seed=5)
+    Q, (wq, sc, bi) = _q(w, 64, 4, "f16")
+    x = inputs.normal((3, 1024), 1.0, torch.float16, seed=6)
+    y = aq.aq_qmm_t(x.to(DEV), wq, sc, bi, 64, 4)
+    ref = oracle_linear_view(x, Q.dequant())
+    assert np.all(row_errors(y, ref) <= 4e-3)
