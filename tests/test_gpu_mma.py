@@ -1,0 +1,151 @@
+"""GPU parity of the tcgen05 tensor-core regime (rows per launch > 4) against the oracle.
+
+Covers several tiles and ragged tails in every dimension: tokens (M not a
+multiple of 16), W rows (N not a multiple of 128), K from one stage (64) to
+many, every supported bit width, group size and activation dtype, strided and
+batched x views, fp32 outputs, and the grouped (mixture-of-experts) entry point
+with empty and uneven experts.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from group_wise_affine_qmv_b200 import aq, inputs
+from tests.parity import dtype_name, oracle_linear_view, row_errors, to_device_quant
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+DEV = "cuda"
+
+
+def _q(w, group, bits, sdtype="bf16"):
+    Q = oracle.quantize(w.float().numpy(), group, bits, sdtype)
+    tdt = torch.bfloat16 if sdtype == "bf16" else torch.float16
+    return Q, to_device_quant(Q, DEV, tdt)
+
+
+def _regime(x, wq, sc, bi, group, bits):
+    y = torch.empty(tuple(x.shape[:-1]) + (wq.shape[-2],), dtype=x.dtype, device=x.device)
+    return aq.aq_plan_linear(x, wq, sc, bi, group, bits, y)["regime"]
+
+
+@pytest.mark.parametrize("bits", [2, 4, 6, 8])
+@pytest.mark.parametrize("M,N,K", [(5, 129, 64), (16, 128, 128), (17, 300, 256), (32, 1000, 1024),
+                                   (33, 257, 512), (64, 640, 1024), (100, 200, 192), (256, 384, 640),
+                                   (300, 131, 320)])
+def test_mma_shapes(bits, M, N, K):
+    group = 64
+    w = inputs.normal((N, K), 0.02, seed=M * 7 + N + K + bits)
+    Q, (wq, sc, bi) = _q(w, group, bits)
+    x = inputs.normal((M, K), 1.0, torch.bfloat16, seed=M + K)
+    xd = x.to(DEV)
+    assert _regime(xd, wq, sc, bi, group, bits) == "mma"
+    y = aq.aq_qmm_t(xd, wq, sc, bi, group, bits)
+    ref = oracle_linear_view(x, Q.dequant())
+    err = row_errors(y, ref)
+    assert np.all(err <= 4e-3), (err.max(), int(err.argmax()))
+
+
+@pytest.mark.parametrize("group", [32, 64, 128])
+@pytest.mark.parametrize("xdtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("bits", [4, 8])
+def test_mma_groups_dtypes(group, xdtype, bits):
+    M, N, K = 24, 260, 4096   # K spans several scale/bias chunks for every group size
+    sd = dtype_name(torch.empty(0, dtype=xdtype))
+    w = inputs.normal((N, K), 0.02, seed=group + bits)
+    Q, (wq, sc, bi) = _q(w, group, bits, sd)
+    x = inputs.normal((M, K), 1.0, xdtype, seed=group * 3 + bits)
+    xd = x.to(DEV)
+    assert _regime(xd, wq, sc, bi, group, bits) == "mma"
+    y = aq.aq_qmm_t(xd, wq, sc, bi, group, bits)
+    ref = oracle_linear_view(x, Q.dequant())
+    assert np.all(row_errors(y, ref) <= 4e-3)
+    # fp32 output: only the weight rounding remains
+    y32 = aq.aq_qmm_t(xd, wq, sc, bi, group, bits, out_dtype=torch.float32)
+    assert np.all(row_errors(y32, ref) <= 3e-3)
+
+
+def test_mma_batched_and_strided_views():
+    """Non-foldable batch dims (launch batches), a row-strided x and a strided y."""
+    K, N, bits, group = 512, 200, 4, 64
+    w = inputs.normal((N, K), 0.02, seed=5)
+    Q, (wq, sc, bi) = _q(w, group, bits)
+    wd = Q.dequant()
+    base = inputs.normal((3, 4, 9, K), 1.0, torch.bfloat16, seed=6)
+    x = base.narrow(1, 1, 2)                      # [3, 2, 9, K], batch dim 0 does not fold
+    xd = base.to(DEV).narrow(1, 1, 2)
+    y = aq.aq_qmm_t(xd, wq, sc, bi, group, bits)
+    ref = oracle_linear_view(x, wd)
+    assert np.all(row_errors(y, ref) <= 4e-3)
+    # same bits as the contiguous copy, every batch element
+    yc = aq.aq_qmm_t(xd.contiguous(), wq, sc, bi, group, bits)
+    for b0 in range(3):
+        for b1 in range(2):
+            assert torch.equal(y[b0, b1], yc[b0, b1])
+    # every other row of a 2D x, written into every other row of a wider y
+    base2 = inputs.normal((40, K), 1.0, torch.bfloat16, seed=7)
+    x2 = base2[::2]
+    ybuf = torch.zeros(20, 2 * N, dtype=torch.bfloat16, device=DEV)
+    y2 = ybuf[:, :N]
+    aq.aq_qmm_t(base2.to(DEV)[::2], wq, sc, bi, group, bits, out=y2)
+    assert torch.all(ybuf[:, N:] == 0)
+    assert np.all(row_errors(y2, oracle_linear_view(x2, wd)) <= 4e-3)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_mma_matches_gemv_numerics(bits):
+    """The two regimes agree with each other to the same bar (different kernels)."""
+    M, N, K, group = 8, 512, 1024, 64
+    w = inputs.normal((N, K), 0.02, seed=11)
+    _, (wq, sc, bi) = _q(w, group, bits)
+    x = inputs.normal((M, K), 1.0, torch.bfloat16, seed=12).to(DEV)
+    a = aq.aq_qmm_t(x, wq, sc, bi, group, bits, out_dtype=torch.float32)
+    b = aq.aq_qmv(x, wq, sc, bi, group, bits, out_dtype=torch.float32)
+    rel = ((a - b).abs().amax(-1) / b.abs().amax(-1)).max().item()
+    assert rel <= 4e-3
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_grouped_experts(bits):
+    E, N, K, group = 6, 200, 256, 32
+    counts = [5, 0, 17, 1, 40, 9]
+    T = sum(counts)
+    offsets = np.zeros(E + 1, np.int64)
+    offsets[1:] = np.cumsum(counts)
+    w = inputs.normal((E, N, K), 0.02, seed=21)
+    Q = oracle.quantize(w.numpy(), group, bits, "bf16")
+    wq, sc, bi = to_device_quant(Q, DEV, torch.bfloat16)
+    x = inputs.normal((T, K), 1.0, torch.bfloat16, seed=22)
+    off_d = torch.from_numpy(offsets).to(DEV)
+    y = aq.aq_qmm_t_grouped(x.to(DEV), off_d, wq, sc, bi, group, bits)
+    xb = x.contiguous().view(torch.int16).numpy().view(np.uint16)
+    ref = oracle.linear_grouped(xb, "bf16", offsets, Q.dequant())
+    assert np.all(row_errors(y, ref) <= 4e-3)
+
+
+def test_grouped_moe_bank_shape():
+    """Expert bank of the "Metal Kernel Bits=8 Final Report" shapes (8-bit, G=32,
+    [2816 out, 1408 in]) on a reduced number of experts, routed top-8 at random."""
+    E, N, K, group, bits = 16, inputs.MOE_N, inputs.MOE_K, inputs.MOE_GROUP, inputs.MOE_BITS
+    routing = inputs.moe_routing(tokens=24, experts=E, topk=4, seed=3)
+    tok, offsets = inputs.moe_sort(routing, E)
+    w = inputs.normal((E, N, K), 0.02, seed=31)
+    Q = oracle.quantize(w.numpy(), group, bits, "bf16")
+    wq, sc, bi = to_device_quant(Q, DEV, torch.bfloat16)
+    x_tok = inputs.normal((24, K), 1.0, torch.bfloat16, seed=32)
+    x_sorted = x_tok[tok].contiguous()
+    y = aq.aq_qmm_t_grouped(x_sorted.to(DEV), offsets.to(DEV), wq, sc, bi, group, bits)
+    # oracle on a sample of 3 rows per expert segment, all columns
+    wd = Q.dequant()
+    xb = x_sorted.view(torch.int16).numpy().view(np.uint16)
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        for r in list(range(lo, min(hi, lo + 3))):
+            ref = oracle.linear_contig(xb[r:r + 1], "bf16", wd[e])
+            assert np.all(row_errors(y[r:r + 1], ref) <= 4e-3), (e, r)
+
+
+def test_device_error_word_clear():
+    aq.aq_device_error()

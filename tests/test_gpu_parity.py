@@ -195,12 +195,12 @@ def test_output_canaries_untouched(bits):
     w = inputs.normal((N, K), 1.0, seed=bits + 50)
     Q, (wq, sc, bi) = _q(w, 64, bits)
     x = inputs.normal((M, K), 1.0, torch.bfloat16, seed=51).to(DEV)
-    buf = torch.full((M + 2, N + 8), 12345.0, dtype=torch.bfloat16, device=DEV)
+    buf = torch.full((M + 2, N + 8), 3072.0, dtype=torch.bfloat16, device=DEV)
     y = buf[1:M + 1, 4:4 + N]
     aq.aq_qmm_t(x, wq, sc, bi, 64, bits, out=y)
     b = buf.float().cpu()
-    assert torch.all(b[0] == 12345.0) and torch.all(b[-1] == 12345.0)
-    assert torch.all(b[:, :4] == 12345.0) and torch.all(b[:, 4 + N:] == 12345.0)
+    assert torch.all(b[0] == 3072.0) and torch.all(b[-1] == 3072.0)
+    assert torch.all(b[:, :4] == 3072.0) and torch.all(b[:, 4 + N:] == 3072.0)
     ref = oracle_linear_view(x.cpu(), Q.dequant())
     assert np.all(row_errors(y, ref) <= 4e-3)
 
