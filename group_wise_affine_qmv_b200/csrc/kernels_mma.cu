@@ -1,36 +1,46 @@
 // kernels_mma.cu -- tensor-core kernel for y = x . dequant(W)^T on sm_100a (tcgen05 / TMEM).
 //
-// The contraction is done "weights-stationary": a tile of 128 rows of W is
-// the MMA's M side, the tokens of x (16..256 per tile) are its N side, so the
-// same kernel serves decode batches (tens of tokens) and prefill (hundreds).
+// Arithmetic (exact up to fp32 summation order).  With codes q, per-group
+// scale s and bias b (w = s*q + b), each output is
+//     y[n, t] = sum_g  s[n,g] * D_g[n, t]  +  b[n,g] * X_g[t],
+//     D_g[n, t] = sum_{k in g} q[n, k] * x[t, k],    X_g[t] = sum_{k in g} x[t, k].
+// The tensor core computes D_g with the INTEGER codes as its A operand (exact
+// in bf16/f16) and x as B, one fresh fp32 accumulator per group; the epilogue
+// warps fold s and b in with fp32 FMAs.  X_g is summed from x widened to fp32
+// before any addition ("mlx PR #4516", load_vector fix).  Rounding w to
+// bf16 before the MMA would cost ~2e-3 of max|y| on its own, while the output
+// rounding to bf16 already spends 2^-8 of the 4e-3 error budget, so the
+// weights are never rounded here.
 //
-//   warp 0      TMA producer: per 64-code stage, the x tile [NT tokens x 64]
-//               (128-byte swizzled, K-major: the UMMA B operand) and the packed
-//               W tile [128 rows x 64 codes], onto one mbarrier.
-//   warp 1      MMA issuer: tcgen05.mma kind::f16, A from tensor memory
-//               (dequantized W), B from shared memory (x), fp32 accumulator
-//               D [128 x NT] in tensor memory; tcgen05.commit releases stages.
-//   warps 2..9  dequantizers: thread <-> W row (TMEM lane), two warps per lane
-//               quarter split each stage's 64 codes; w' = s*q + b rounded once
-//               to bf16/f16 is written with tcgen05.st into an A slot.  The
-//               same warps run the epilogue (tcgen05.ld of D, convert, store y).
+// Roles ("weights-stationary": 128 rows of W are the MMA's M side, up to 128
+// tokens its N side):
+//   warp 0      TMA producer: per 64-code stage, the x tile [NT x 64] (128-byte
+//               swizzled, K-major UMMA B operand) and the packed W tile
+//               [128 rows x 64 codes], completing on one mbarrier.
+//   warp 1      MMA issuer: tcgen05.mma kind::f16, A (codes) from tensor
+//               memory, B from shared memory, D_g into one of two TMEM
+//               accumulators; tcgen05.commit releases stages, A slots and
+//               finished groups.
+//   warps 2..9  code expanders + epilogue: thread <-> W row (TMEM lane); two
+//               warps per lane quarter split each stage's 64 codes and, in the
+//               epilogue, the tile's tokens.  They expand packed codes into
+//               bf16/f16 integers with tcgen05.st, then for every finished
+//               group read D_g (tcgen05.ld) and update fp32 accumulators held
+//               in registers; at tile end they store y.
 //
-// Dequantizing into tensor memory instead of shared memory keeps the
-// shared-memory traffic at the packed weights plus the x tile; the per-group
-// scales/biases of a tile are brought in with asynchronous 4-byte copies.
+// Rows of the last W tile that fall past N read TMA zero fill and the clamped
+// last row's scale/bias and are simply not stored: no per-row check inside the
+// K loop (the partial-rows idea of "mlx PR #4516").
 //
-// Rows of the last W tile that fall past N are read as TMA zero fill (or as
-// the clamped last row's scale/bias) and simply not stored: no per-row check
-// inside the K loop (the partial-rows idea of "mlx PR #4516").
-//
-// Every mbarrier wait is bounded (2 s); on expiry the CTA raises an abort
-// flag, records an error word readable through aq_device_error(), drains its
-// own outstanding copies (bounded), frees its tensor memory and exits.
+// Every mbarrier wait is bounded (2 s); on expiry the CTA raises an abort flag,
+// records an error word readable through aq_device_error(), drains its own
+// outstanding copies and MMAs (bounded), frees its tensor memory and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "aq_internal.h"
 #include "device_common.cuh"
@@ -50,24 +60,30 @@ constexpr int SCW = 32;                   // groups per scale/bias chunk
 constexpr int SCP = SCW + 2;              // padded row pitch (halves) of a chunk in shared memory
 constexpr int MAX_STAGES = 16;
 constexpr int MAX_EXPERTS = 1024;
+constexpr int XTAB_MAX_BYTES = 48 * 1024; // sum-of-x table per token tile
+constexpr int NBMAX = 4;                  // group accumulators in tensor memory
+
+// group accumulators for a token-tile width: 4 while they fit beside the A slots
+__host__ __device__ constexpr int nbufs(int nt) { return nt <= 64 ? 4 : 2; }
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait
 constexpr int ERR_TIMEOUT = 1;
 
 struct MmaParams {
-    CUtensorMap tx;  // x: 4D {K, rows, nb1, nb0} u16, box {64, nt, 1, 1}, 128B swizzle
+    CUtensorMap tx;  // x: 4D {K, rows, nb1, nb0} u16, box {64, NT, 1, 1}, 128B swizzle
     CUtensorMap tw;  // W: 2D {K*bits/32, rows} u32, box {2*bits, 128}
+    const void* x;
     void* y;
     const uint16_t* scales;
     const uint16_t* biases;
     int64_t M, N, K;
-    int64_t y_row;
-    int64_t yb[2];
+    int64_t x_row, y_row;
+    int64_t xb[2], yb[2];
     int64_t nb1;
-    int nt;
     int n_wtiles, n_ttiles, nbatch;
-    int log2g;
+    int group, log2g;
     int stages;
     int kg;              // groups per row = K / group
+    int ydt;             // DT of y
     uint32_t tmem_cols;
     uint32_t idesc;
     const int64_t* offsets;  // grouped mode when non-null
@@ -80,7 +96,7 @@ struct TileInfo {
     int64_t wrow0;   // first W row of the tile in the W tensor (expert offset included)
     int64_t n0;      // first output column (row of W within the expert / matrix)
     int nvalid;      // valid W rows in this tile
-    int64_t xrow0;   // first x row (token) coordinate
+    int64_t xrow0;   // first x row (token) of the tile within its batch / the sorted rows
     int tvalid;      // valid tokens in this tile
     int b0, b1;      // launch batch (non-grouped)
 };
@@ -90,34 +106,41 @@ struct Smem {
     uint64_t* empty;
     uint64_t* afull;
     uint64_t* aempty;
-    uint64_t* dfull;
+    uint64_t* gfull;     // [NBMAX] group accumulator ready (MMA commit)
+    uint64_t* gempty;    // [NBMAX] group accumulator consumed (8 epilogue warps)
     uint64_t* sbar;      // [2] scale/bias chunk slots: 256 dequant-thread arrivals
+    uint64_t* xbar;      // sum-of-x table barrier: 256 arrivals
     uint64_t* mdone;     // all MMAs of this CTA retired (teardown)
     uint32_t* tmem_base;
     int* abort;
-    int* prefix;     // grouped: tile prefix sums [n_experts + 1]
-    uint8_t* xs;     // stages * nt * 128
-    uint8_t* ws;     // stages * 1024 * bits
-    uint16_t* sb;    // [2 slots][2 arrays][128][SCP]
+    int* prefix;         // grouped: tile prefix sums [n_experts + 1]
+    float* xtab;         // [kg][NT] sums of x per group and token
+    uint8_t* xs;         // stages * NT * 128
+    uint8_t* ws;         // stages * 1024 * bits
+    uint16_t* sb;        // [2 slots][2 arrays][128][SCP]
 };
 
-template <int BITS>
+template <int BITS, int NT>
 __device__ __forceinline__ Smem carve(uint8_t* base, const MmaParams& p) {
     Smem s;
     uint8_t* q = base;
     s.xs = q;
-    q += (size_t)p.stages * p.nt * 128;
+    q += (size_t)p.stages * NT * 128;
     s.ws = q;
     q += (size_t)p.stages * 1024 * BITS;
+    s.xtab = reinterpret_cast<float*>(q);
+    q += (size_t)p.kg * NT * 4;
     s.sb = reinterpret_cast<uint16_t*>(q);
     q += 2 * 2 * 128 * SCP * 2;
     s.full = reinterpret_cast<uint64_t*>(q);
     s.empty = s.full + MAX_STAGES;
     s.afull = s.empty + MAX_STAGES;
     s.aempty = s.afull + SA;
-    s.dfull = s.aempty + SA;
-    s.sbar = s.dfull + 1;
-    s.mdone = s.sbar + 2;
+    s.gfull = s.aempty + SA;
+    s.gempty = s.gfull + NBMAX;
+    s.sbar = s.gempty + NBMAX;
+    s.xbar = s.sbar + 2;
+    s.mdone = s.xbar + 1;
     s.tmem_base = reinterpret_cast<uint32_t*>(s.mdone + 1);
     s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
     s.prefix = s.abort + 1;
@@ -125,7 +148,7 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const MmaParams& p) {
 }
 
 __host__ __device__ constexpr size_t smem_fixed_bytes() {
-    return 2 * 2 * 128 * SCP * 2 + (2 * MAX_STAGES + 2 * SA + 4) * 8 + 8 + (MAX_EXPERTS + 1) * 4 + 1024 /*align*/;
+    return 2 * 2 * 128 * SCP * 2 + (2 * MAX_STAGES + 2 * SA + 2 * NBMAX + 5) * 8 + 8 + (MAX_EXPERTS + 1) * 4 + 1024 /*align*/;
 }
 
 __device__ __forceinline__ void raise_abort(int* abort) {
@@ -133,17 +156,16 @@ __device__ __forceinline__ void raise_abort(int* abort) {
     atomicExch(&g_device_error, ERR_TIMEOUT);
 }
 
-// total number of tiles (grouped mode reads the prefix sums in shared memory)
 __device__ __forceinline__ int total_tiles(const MmaParams& p, const Smem& s) {
     if (p.offsets) return s.prefix[p.n_experts];
     return p.n_wtiles * p.n_ttiles * p.nbatch;
 }
 
+template <int NT>
 __device__ __forceinline__ TileInfo tile_info(const MmaParams& p, const Smem& s, int t) {
     TileInfo ti;
     if (p.offsets) {
-        // expert e with prefix[e] <= t < prefix[e+1]
-        int lo = 0, hi = p.n_experts;
+        int lo = 0, hi = p.n_experts;  // expert e with prefix[e] <= t < prefix[e+1]
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
             if (s.prefix[mid] <= t) lo = mid; else hi = mid;
@@ -155,8 +177,8 @@ __device__ __forceinline__ TileInfo tile_info(const MmaParams& p, const Smem& s,
         ti.n0 = (int64_t)wt * 128;
         ti.wrow0 = (int64_t)e * p.N + ti.n0;
         ti.nvalid = (int)min64(128, p.N - ti.n0);
-        ti.xrow0 = off + (int64_t)tt * p.nt;
-        ti.tvalid = (int)min64(p.nt, cnt - (int64_t)tt * p.nt);
+        ti.xrow0 = off + (int64_t)tt * NT;
+        ti.tvalid = (int)min64(NT, cnt - (int64_t)tt * NT);
         ti.b0 = ti.b1 = 0;
     } else {
         const int wt = t % p.n_wtiles;
@@ -166,8 +188,8 @@ __device__ __forceinline__ TileInfo tile_info(const MmaParams& p, const Smem& s,
         ti.n0 = (int64_t)wt * 128;
         ti.wrow0 = ti.n0;
         ti.nvalid = (int)min64(128, p.N - ti.n0);
-        ti.xrow0 = (int64_t)tt * p.nt;
-        ti.tvalid = (int)min64(p.nt, p.M - ti.xrow0);
+        ti.xrow0 = (int64_t)tt * NT;
+        ti.tvalid = (int)min64(NT, p.M - ti.xrow0);
         ti.b1 = (int)(b % p.nb1);
         ti.b0 = (int)(b / p.nb1);
     }
@@ -175,14 +197,15 @@ __device__ __forceinline__ TileInfo tile_info(const MmaParams& p, const Smem& s,
 }
 
 // ---------------------------------------------------------------------------
-// dequantization of one thread's 32 codes into 16 packed A-operand pairs
+// code expansion: one thread's 32 packed codes -> 16 pairs of exact integers
+// in the 16-bit MMA type (low half = even code)
 // ---------------------------------------------------------------------------
 
 // swizzled byte offset of a 16-byte chunk written by TMA (bits 4.. XOR bits 7..)
 template <int BITS>
 __device__ __forceinline__ uint32_t wswz(uint32_t off) {
-    if constexpr (BITS == 4) return off ^ (((off >> 7) & 1u) << 4);   // 32-byte swizzle
-    else if constexpr (BITS == 8) return off ^ (((off >> 7) & 3u) << 4);  // 64-byte swizzle
+    if constexpr (BITS == 4) return off ^ (((off >> 7) & 1u) << 4);      // 32-byte swizzle
+    else if constexpr (BITS == 8) return off ^ (((off >> 7) & 3u) << 4); // 64-byte swizzle
     else return off;
 }
 
@@ -207,75 +230,57 @@ __device__ __forceinline__ void load_w32(const uint8_t* stage, int row, int h, u
     }
 }
 
-__device__ __forceinline__ uint32_t pack2(float lo, float hi, bf16_t) {
-    const __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&r);
-}
-__device__ __forceinline__ uint32_t pack2(float lo, float hi, f16_t) {
-    const __half2 r = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&r);
-}
-
-// (offset + q) pairs to s*q + b, rounded once, in the 16-bit type
-__device__ __forceinline__ uint32_t affine2(uint32_t qo, uint32_t s2, uint32_t b2, uint32_t off2, bf16_t) {
-    const __nv_bfloat162 q = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&qo),
+// (OFF + q0, OFF + q1) in both halves -> (q0, q1), exact
+__device__ __forceinline__ uint32_t sub_off(uint32_t v, uint32_t off2, bf16_t) {
+    const __nv_bfloat162 r = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&v),
                                      *reinterpret_cast<const __nv_bfloat162*>(&off2));
-    const __nv_bfloat162 r = __hfma2(*reinterpret_cast<const __nv_bfloat162*>(&s2), q,
-                                     *reinterpret_cast<const __nv_bfloat162*>(&b2));
     return *reinterpret_cast<const uint32_t*>(&r);
 }
-__device__ __forceinline__ uint32_t affine2(uint32_t qo, uint32_t s2, uint32_t b2, uint32_t off2, f16_t) {
-    const __half2 q = __hsub2(*reinterpret_cast<const __half2*>(&qo), *reinterpret_cast<const __half2*>(&off2));
-    const __half2 r = __hfma2(*reinterpret_cast<const __half2*>(&s2), q, *reinterpret_cast<const __half2*>(&b2));
+__device__ __forceinline__ uint32_t sub_off(uint32_t v, uint32_t off2, f16_t) {
+    const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&v), *reinterpret_cast<const __half2*>(&off2));
     return *reinterpret_cast<const uint32_t*>(&r);
 }
 
 template <int BITS, typename XT>
-__device__ __forceinline__ void dequant32(const uint32_t* w, uint16_t sbits, uint16_t bbits, uint32_t* out) {
-    const uint32_t s2 = (uint32_t)sbits | ((uint32_t)sbits << 16);
-    const uint32_t b2 = (uint32_t)bbits | ((uint32_t)bbits << 16);
+__device__ __forceinline__ void expand32(const uint32_t* w, uint32_t* out) {
     constexpr bool BF = std::is_same<XT, bf16_t>::value;
+    // 0x4300 = 128.0 in bf16 (7 mantissa bits), 0x6400 = 1024.0 in f16 (10 mantissa bits):
+    // OR-ing a code into the mantissa gives exactly OFF + q.
+    constexpr uint32_t MAGIC = BF ? 0x43004300u : 0x64006400u;
     if constexpr (BITS == 4) {
         // byte j of a word holds codes (2j, 2j+1); the word shifted by 4 holds code 2j+1 in
-        // the low nibble of byte j.  PRMT gathers both into the two halves, LOP3 makes
-        // (offset + q) in each half: 128 + q in bf16 (0x4300 | q), 1024 + q in f16 (0x6400 | q).
-        constexpr uint32_t MAGIC = BF ? 0x43004300u : 0x64006400u;
-        constexpr uint32_t OFF2 = MAGIC;
+        // the low nibble of byte j.  PRMT gathers both into the two halves.
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint32_t word = w[i], shifted = w[i] >> 4;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const uint32_t t = __byte_perm(word, shifted, j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12));
-                const uint32_t qo = (t & 0x000F000Fu) | MAGIC;
-                out[4 * i + j] = affine2(qo, s2, b2, OFF2, XT{});
+                out[4 * i + j] = sub_off((t & 0x000F000Fu) | MAGIC, MAGIC, XT{});
             }
         }
     } else if constexpr (BITS == 8 && !BF) {
-        // f16: 1024 + q is exact for every 8-bit code
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const uint32_t qo = __byte_perm(w[i], 0x64006400u, (2 * j) | (5 << 4) | ((2 * j + 1) << 8) | (7 << 12));
-                out[2 * i + j] = affine2(qo, s2, b2, 0x64006400u, XT{});
-            }
-        }
+            for (int j = 0; j < 2; ++j)
+                out[2 * i + j] = sub_off(
+                    __byte_perm(w[i], MAGIC, (2 * j) | (5 << 4) | ((2 * j + 1) << 8) | (7 << 12)), MAGIC, XT{});
     } else if constexpr (BITS == 8) {
-        // bf16 cannot hold 128 + q for q >= 128: go through fp32 (2^23 + q is exact there)
-        const float s = __uint_as_float((uint32_t)sbits << 16), b = __uint_as_float((uint32_t)bbits << 16);
+        // bf16 cannot hold 128 + q for q >= 128: form q exactly in fp32 (2^23 + q minus 2^23), then
+        // convert the pair (every q <= 255 is exact in bf16)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const float q0 = __uint_as_float(__byte_perm(w[i], 0x4B000000u, (2 * j) | (4 << 4) | (5 << 8) | (7 << 12))) - 8388608.0f;
                 const float q1 = __uint_as_float(__byte_perm(w[i], 0x4B000000u, (2 * j + 1) | (4 << 4) | (5 << 8) | (7 << 12))) - 8388608.0f;
-                out[2 * i + j] = pack2(fmaf(s, q0, b), fmaf(s, q1, b), XT{});
+                const __nv_bfloat162 r = __floats2bfloat162_rn(q0, q1);
+                out[2 * i + j] = *reinterpret_cast<const uint32_t*>(&r);
             }
         }
     } else {
-        // generic width (2, 6): funnel-shift extraction, fp32 affine, one rounding
-        const float s = half_bits_to_float(sbits, XT{}), b = half_bits_to_float(bbits, XT{});
+        // generic widths (2, 6): funnel-shift extraction of both codes of a pair
         constexpr uint32_t MASK = (1u << BITS) - 1u;
         uint32_t ww[BITS + 1];
 #pragma unroll
@@ -283,21 +288,16 @@ __device__ __forceinline__ void dequant32(const uint32_t* w, uint16_t sbits, uin
         ww[BITS] = 0;
 #pragma unroll
         for (int pr = 0; pr < 16; ++pr) {
-            float v[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int pos = (2 * pr + e) * BITS;
-                const int wi = pos >> 5, sh = pos & 31;
-                const uint32_t q = __funnelshift_r(ww[wi], ww[wi + 1], sh) & MASK;
-                v[e] = fmaf(s, (float)q, b);
-            }
-            out[pr] = pack2(v[0], v[1], XT{});
+            const int p0 = (2 * pr) * BITS, p1 = p0 + BITS;
+            const uint32_t q0 = __funnelshift_r(ww[p0 >> 5], ww[(p0 >> 5) + 1], p0 & 31) & MASK;
+            const uint32_t q1 = __funnelshift_r(ww[p1 >> 5], ww[(p1 >> 5) + 1], p1 & 31) & MASK;
+            out[pr] = sub_off(q0 | (q1 << 16) | MAGIC, MAGIC, XT{});
         }
     }
 }
 
 // ---------------------------------------------------------------------------
-// scale/bias chunk loads (dequant warps, asynchronous 4-byte copies)
+// scale/bias chunk loads (asynchronous 4-byte copies by the 256 expander threads)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void issue_sb_chunk(const MmaParams& p, const TileInfo& ti, int chunk, uint16_t* slot,
                                                int tid) {
@@ -316,19 +316,62 @@ __device__ __forceinline__ void issue_sb_chunk(const MmaParams& p, const TileInf
     }
 }
 
+// sum over each group of x[t, k] (widened to fp32 first) for the tile's tokens -> xtab[g][t]
+template <typename XT, int NT>
+__device__ __forceinline__ void build_xtab(const MmaParams& p, const TileInfo& ti, float* xtab, int tid) {
+    const XT* xb = (const XT*)p.x + (p.offsets ? 0 : (int64_t)ti.b0 * p.xb[0] + (int64_t)ti.b1 * p.xb[1]);
+    const int items = p.kg * NT;
+    const int vec_per_group = p.group >> 3;  // 16-byte vectors of 8 elements
+    for (int it = tid; it < items; it += DQ_THREADS) {
+        const int g = it / NT, t = it - g * NT;
+        float acc = 0.0f;
+        if (t < ti.tvalid) {
+            const XT* row = xb + (ti.xrow0 + t) * p.x_row + (int64_t)g * p.group;
+            for (int v = 0; v < vec_per_group; ++v) {
+                float f[8];
+                unpack8(__ldg(reinterpret_cast<const uint4*>(row) + v), f, XT{});
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc += f[e];
+            }
+        }
+        xtab[g * NT + t] = acc;
+    }
+}
+
+__device__ __forceinline__ void store_y(void* y, int64_t off, float v, int ydt, bf16_t) {
+    if (ydt == (int)DT::F32) store_out((float*)y + off, v);
+    else store_out((bf16_t*)y + off, v);
+}
+__device__ __forceinline__ void store_y(void* y, int64_t off, float v, int ydt, f16_t) {
+    if (ydt == (int)DT::F32) store_out((float*)y + off, v);
+    else store_out((f16_t*)y + off, v);
+}
+
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-template <int BITS, typename XT, typename YT>
+template <int BITS, typename XT, int NT>
 __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_constant__ MmaParams p) {
+    constexpr int H = NT / 2;            // tokens per epilogue thread
+    constexpr int NB = nbufs(NT);        // group accumulators
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const Smem s = carve<BITS>(base, p);
+    const Smem s = carve<BITS, NT>(base, p);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = p.stages;
     const int KBLK = (int)(p.K / KB);
+    const int G = p.group;
+    const int NG = p.kg;
     const int CS = (SCW << p.log2g) / KB;   // stages per scale/bias chunk
-    const int NCH = (p.kg + SCW - 1) / SCW; // chunks per tile
+    const int NCH = (NG + SCW - 1) / SCW;   // chunks per tile
+    // Epilogue lag in stages: group g is folded in once the expanders are LAG stages past
+    // its end, so the MMA of the stages in between overlaps code expansion.  The MMA of a
+    // stage reuses the accumulator of the group NB groups earlier, which must be folded by
+    // then: NB >= LAG * groups-per-stage.
+    const int gps = G < KB ? KB / G : 1;
+    int LAG = NB / gps;
+    if (LAG > 3) LAG = 3;
+    if (LAG < 1) LAG = 1;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
@@ -339,9 +382,13 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
             ptx::mbar_init(&s.afull[i], 8);
             ptx::mbar_init(&s.aempty[i], 1);
         }
-        ptx::mbar_init(s.dfull, 1);
+        for (int i = 0; i < NBMAX; ++i) {
+            ptx::mbar_init(&s.gfull[i], 1);
+            ptx::mbar_init(&s.gempty[i], 8);
+        }
         ptx::mbar_init(&s.sbar[0], DQ_THREADS);
         ptx::mbar_init(&s.sbar[1], DQ_THREADS);
+        ptx::mbar_init(s.xbar, DQ_THREADS);
         ptx::mbar_init(s.mdone, 1);
         *s.abort = 0;
         ptx::fence_mbar_init();
@@ -355,7 +402,7 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
         ptx::tmem_relinquish();
     }
     if (p.offsets && warp == 2) {
-        // tiles per expert: ceil(count / nt) * n_wtiles, prefix-summed
+        // tiles per expert: ceil(count / NT) * n_wtiles, prefix-summed
         if (lane == 0) s.prefix[0] = 0;
         __syncwarp();
         int carry = 0;
@@ -364,7 +411,7 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
             int v = 0;
             if (e < p.n_experts) {
                 const int64_t cnt = p.offsets[e + 1] - p.offsets[e];
-                v = (int)((cnt + p.nt - 1) / p.nt) * p.n_wtiles;
+                v = (int)((cnt + NT - 1) / NT) * p.n_wtiles;
             }
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -379,24 +426,23 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tbase = *s.tmem_base;
-    const uint32_t d_tmem = tbase + SA * 32;  // accumulator columns follow the A slots
+    const uint32_t d_tmem = tbase + SA * 32;  // NB group accumulators of NT columns follow the A slots
     const int ntiles = total_tiles(p, s);
 
     if (warp == 0) {
         // ======================= TMA producer =======================
         if (lane == 0) {
-            const uint32_t xbytes = (uint32_t)p.nt * 128;
-            const uint32_t wbytes = 1024u * BITS;
+            const uint32_t bytes = (uint32_t)NT * 128 + 1024u * BITS;
             uint32_t it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                const TileInfo ti = tile_info(p, s, t);
+                const TileInfo ti = tile_info<NT>(p, s, t);
                 for (int kb = 0; kb < KBLK; ++kb, ++it) {
                     const int st = it % S;
                     const uint32_t ph = (it / S) & 1;
                     if (!ptx::mbar_wait(&s.empty[st], ph ^ 1, s.abort, WAIT_NS)) { ok = false; break; }
-                    ptx::mbar_arrive_expect_tx(&s.full[st], xbytes + wbytes);
-                    ptx::tma_load_4d(s.xs + (size_t)st * p.nt * 128, &p.tx, &s.full[st], kb * KB, (int32_t)ti.xrow0,
+                    ptx::mbar_arrive_expect_tx(&s.full[st], bytes);
+                    ptx::tma_load_4d(s.xs + (size_t)st * NT * 128, &p.tx, &s.full[st], kb * KB, (int32_t)ti.xrow0,
                                      ti.b1, ti.b0);
                     ptx::tma_load_2d(s.ws + (size_t)st * 1024 * BITS, &p.tw, &s.full[st], kb * 2 * BITS,
                                      (int32_t)ti.wrow0);
@@ -415,10 +461,10 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
     } else if (warp == 1) {
         // ======================= MMA issuer =======================
         if (lane == 0) {
-            uint32_t it = 0;
+            uint32_t it = 0, gc = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                for (int kb = 0; kb < KBLK; ++kb, ++it) {
+                for (int kb = 0; kb < KBLK && ok; ++kb, ++it) {
                     const int st = it % S;
                     const uint32_t ph = (it / S) & 1;
                     const int a = it % SA;
@@ -429,16 +475,30 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
                         break;
                     }
                     ptx::tc_fence_after();
-                    const uint32_t xaddr = ptx::smem_u32(s.xs + (size_t)st * p.nt * 128);
+                    const uint32_t xaddr = ptx::smem_u32(s.xs + (size_t)st * NT * 128);
 #pragma unroll
                     for (int j = 0; j < KB / 16; ++j) {
+                        const int k = kb * KB + 16 * j;
+                        const bool gstart = (k & (G - 1)) == 0;
+                        const uint32_t buf = gc % NB;
+                        if (gstart) {
+                            // this accumulator's previous group must have been read by the epilogue
+                            if (!ptx::mbar_wait(&s.gempty[buf], ((gc / NB) & 1) ^ 1, s.abort, WAIT_NS)) {
+                                ok = false;
+                                break;
+                            }
+                            ptx::tc_fence_after();
+                        }
                         const uint64_t bdesc = ptx::smem_desc_sw128(xaddr + 32 * j);
-                        ptx::mma_ts(d_tmem, tbase + a * 32 + j * 8, bdesc, p.idesc, (kb | j) != 0 ? 1u : 0u);
+                        ptx::mma_ts(d_tmem + buf * NT, tbase + a * 32 + j * 8, bdesc, p.idesc, gstart ? 0u : 1u);
+                        if (((k + 16) & (G - 1)) == 0) {
+                            ptx::mma_commit(&s.gfull[buf]);
+                            ++gc;
+                        }
                     }
                     ptx::mma_commit(&s.empty[st]);
                     ptx::mma_commit(&s.aempty[a]);
                 }
-                if (ok) ptx::mma_commit(s.dfull);
             }
             if (!ok) raise_abort(s.abort);
             // every MMA this thread issued must retire before tensor memory is freed
@@ -448,48 +508,116 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
         }
         __syncwarp();
     } else {
-        // ======================= dequantizers + epilogue =======================
+        // ======================= code expanders + epilogue =======================
         const int q = warp & 3;                 // TMEM lane quarter
-        const int h = (warp - 2) >> 2;          // which 32 codes of each stage
+        const int h = (warp - 2) >> 2;          // which 32 codes of each stage / which half of the tokens
         const int row = 32 * q + lane;          // W row within the tile == TMEM lane
         const int tid = threadIdx.x - 64;       // 0..255
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        uint32_t it = 0;
+        uint32_t it = 0, ge = 0, xph = 0;
         int unit = 0;
         bool ok = true;
-        // first scale/bias chunk of the first tile
+        int64_t cur_x0 = -1;
+        int cur_b = -1, cur_tv = -1;
+        float2 acc[H / 2];
+
         if (blockIdx.x < ntiles) {
-            const TileInfo t0 = tile_info(p, s, blockIdx.x);
+            const TileInfo t0 = tile_info<NT>(p, s, blockIdx.x);
             issue_sb_chunk(p, t0, 0, s.sb, tid);
         }
         ptx::cp_async_commit();
-        int tile_iter = 0;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tile_iter) {
-            const TileInfo ti = tile_info(p, s, t);
-            const uint16_t* slot = s.sb;
-            int g_chunk0 = 0;
+
+        const uint16_t* slot = s.sb;
+        int g_chunk0 = 0;
+
+        // epilogue of group g of the current tile: acc += s*D_g + b*X_g
+        auto epilogue_group = [&](int g) -> bool {
+            const uint32_t buf = ge % NB;
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&s.gfull[buf], (ge / NB) & 1, s.abort, WAIT_NS)))
+                return false;
+            ptx::tc_fence_after();
+            const int gl = g - g_chunk0;
+            const float sv = half_bits_to_float(slot[row * SCP + gl], XT{});
+            const float bv = half_bits_to_float(slot[128 * SCP + row * SCP + gl], XT{});
+            const float2 s2 = make_float2(sv, sv), b2 = make_float2(bv, bv);
+            const float* xg = s.xtab + g * NT + h * H;
+#pragma unroll
+            for (int c0 = 0; c0 < H; c0 += 16) {
+                uint32_t v[16];
+                if constexpr (H >= 16) {
+                    ptx::tmem_ld16(d_tmem + buf * NT + lane_base + h * H + c0, v);
+                } else {
+                    ptx::tmem_ld8(d_tmem + buf * NT + lane_base + h * H + c0, v);
+                }
+                ptx::tc_wait_ld();
+                constexpr int CNT = H >= 16 ? 16 : H;
+#pragma unroll
+                for (int c = 0; c < CNT; c += 4) {
+                    const float4 xv = *reinterpret_cast<const float4*>(xg + c0 + c);
+                    float2& a0 = acc[(c0 + c) / 2];
+                    float2& a1 = acc[(c0 + c) / 2 + 1];
+                    a0 = ptx::ffma2(b2, make_float2(xv.x, xv.y), a0);
+                    a1 = ptx::ffma2(b2, make_float2(xv.z, xv.w), a1);
+                    a0 = ptx::ffma2(s2, make_float2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), a0);
+                    a1 = ptx::ffma2(s2, make_float2(__uint_as_float(v[c + 2]), __uint_as_float(v[c + 3])), a1);
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&s.gempty[buf]);
+            ++ge;
+            return true;
+        };
+
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const TileInfo ti = tile_info<NT>(p, s, t);
+            // ---- sums of x for this token tile (rebuilt only when the tokens change) ----
+            const int bkey = ti.b0 * 65536 + ti.b1;
+            if (ti.xrow0 != cur_x0 || bkey != cur_b || ti.tvalid != cur_tv) {
+                // everyone is done reading the previous table
+                ptx::mbar_arrive(s.xbar);
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_NS));
+                ++xph;
+                if (!ok) break;
+                build_xtab<XT, NT>(p, ti, s.xtab, tid);
+                ptx::mbar_arrive(s.xbar);
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_NS));
+                ++xph;
+                if (!ok) break;
+                cur_x0 = ti.xrow0;
+                cur_b = bkey;
+                cur_tv = ti.tvalid;
+            }
+#pragma unroll
+            for (int i = 0; i < H / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
+            int g_next = 0;  // next group of this tile awaiting its epilogue
             for (int kb = 0; kb < KBLK; ++kb, ++it) {
+                // (1) epilogues of the groups that ended LAG stages before this one
+                while (g_next < NG && (g_next + 1) * G <= (kb - LAG + 1) * KB) {
+                    if (!epilogue_group(g_next)) { ok = false; break; }
+                    ++g_next;
+                }
+                if (!ok) break;
+                // (2) next scale/bias chunk
                 if (kb % CS == 0) {
-                    // this chunk's copies were issued one chunk earlier: each thread waits for its
-                    // own, then the 256 dequant threads meet on the slot's mbarrier (release/acquire)
                     ptx::cp_async_wait_all();
                     ptx::mbar_arrive(&s.sbar[unit & 1]);
                     ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS));
                     if (!ok) break;
                     slot = s.sb + (unit & 1) * 2 * 128 * SCP;
-                    g_chunk0 = (kb / CS) * SCW;
-                    // prefetch the next chunk (this tile's next, or the next tile's first)
                     const int c = kb / CS;
+                    g_chunk0 = c * SCW;
                     uint16_t* nslot = s.sb + ((unit + 1) & 1) * 2 * 128 * SCP;
                     if (c + 1 < NCH) {
                         issue_sb_chunk(p, ti, c + 1, nslot, tid);
                     } else if (t + (int)gridDim.x < ntiles) {
-                        const TileInfo tn = tile_info(p, s, t + gridDim.x);
+                        const TileInfo tn = tile_info<NT>(p, s, t + gridDim.x);
                         issue_sb_chunk(p, tn, 0, nslot, tid);
                     }
                     ptx::cp_async_commit();
                     ++unit;
                 }
+                // (3) expand this stage's codes into an A slot
                 const int st = it % S;
                 const uint32_t ph = (it / S) & 1;
                 const int a = it % SA;
@@ -498,11 +626,8 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
                 if (!ok) break;
                 uint32_t wv[BITS];
                 load_w32<BITS>(s.ws + (size_t)st * 1024 * BITS, row, h, wv);
-                const int g = ((kb * KB + 32 * h) >> p.log2g) - g_chunk0;
-                const uint16_t sbits = slot[row * SCP + g];
-                const uint16_t bbits = slot[128 * SCP + row * SCP + g];
                 uint32_t out[16];
-                dequant32<BITS, XT>(wv, sbits, bbits, out);
+                expand32<BITS, XT>(wv, out);
                 ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.aempty[a], aph ^ 1, s.abort, WAIT_NS));
                 if (!ok) break;
                 ptx::tmem_st16(tbase + lane_base + a * 32 + 16 * h, out);
@@ -512,28 +637,23 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
                 if (lane == 0) ptx::mbar_arrive(&s.afull[a]);
             }
             if (!ok) break;
-            // ---- epilogue: D[128 x nt] -> y ----
-            ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.dfull, tile_iter & 1, s.abort, WAIT_NS));
+            while (g_next < NG) {
+                if (!epilogue_group(g_next)) { ok = false; break; }
+                ++g_next;
+            }
             if (!ok) break;
-            ptx::tc_fence_after();
-            const int half = p.nt >> 1;
-            const int c0 = h * half;
-            const int64_t n = ti.n0 + row;
-            const bool row_ok = row < ti.nvalid;
-            YT* ybase;
-            if (p.offsets) ybase = (YT*)p.y + ti.xrow0 * p.y_row + n;
-            else ybase = (YT*)p.y + ti.b0 * p.yb[0] + ti.b1 * p.yb[1] + ti.xrow0 * p.y_row + n;
-            for (int cc = 0; cc < half; cc += 8) {
-                uint32_t v[8];
-                ptx::tmem_ld8(d_tmem + lane_base + c0 + cc, v);
-                ptx::tc_wait_ld();
+            // ---- store this thread's row of y for its half of the tokens ----
+            if (row < ti.nvalid) {
+                const int64_t n = ti.n0 + row;
+                int64_t off = ti.xrow0 * p.y_row + n;
+                if (!p.offsets) off += (int64_t)ti.b0 * p.yb[0] + (int64_t)ti.b1 * p.yb[1];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int tok = c0 + cc + e;
-                    if (row_ok && tok < ti.tvalid) store_out(ybase + (int64_t)tok * p.y_row, __uint_as_float(v[e]));
+                for (int i = 0; i < H / 2; ++i) {
+                    const int tok = h * H + 2 * i;
+                    if (tok < ti.tvalid) store_y(p.y, off + (int64_t)tok * p.y_row, acc[i].x, p.ydt, XT{});
+                    if (tok + 1 < ti.tvalid) store_y(p.y, off + (int64_t)(tok + 1) * p.y_row, acc[i].y, p.ydt, XT{});
                 }
             }
-            ptx::tc_fence_before();
         }
         ptx::cp_async_wait_all();
         if (!ok) raise_abort(s.abort);
@@ -577,35 +697,32 @@ int num_sms() {
     return n[dev];
 }
 
+// tokens per tile: 16, 32, 64 or 128
 int pick_nt(const MmaProblem& p) {
-    int64_t m;
-    if (p.offsets) {
-        const int64_t avg = (p.M + p.n_experts - 1) / p.n_experts;
-        m = 2 * avg;
-        if (m > 128) m = 128;
-    } else {
-        m = p.M;
-    }
-    int64_t nt = (m + 15) / 16 * 16;
-    if (nt < 16) nt = 16;
-    if (nt > 256) nt = 256;
-    return (int)nt;
-}
-
-size_t smem_for(int nt, int bits, int stages) {
-    return (size_t)stages * ((size_t)nt * 128 + 1024 * (size_t)bits) + smem_fixed_bytes();
+    int64_t m = p.M;
+    if (p.offsets) m = 2 * ((p.M + p.n_experts - 1) / p.n_experts);
+    if (m <= 16) return 16;
+    if (m <= 32) return 32;
+    if (m <= 64) return 64;
+    return 128;
 }
 
 constexpr size_t SMEM_LIMIT = 227 * 1024;
 
-int pick_stages(int nt, int bits) {
+size_t smem_for(int nt, int bits, int stages, int64_t kg) {
+    return (size_t)stages * ((size_t)nt * 128 + 1024 * (size_t)bits) + (size_t)kg * nt * 4 + smem_fixed_bytes();
+}
+
+int pick_stages(int nt, int bits, int64_t kg) {
     const size_t per = (size_t)nt * 128 + 1024 * (size_t)bits;
-    int st = (int)((SMEM_LIMIT - smem_fixed_bytes()) / per);
+    const size_t fixed = (size_t)kg * nt * 4 + smem_fixed_bytes();
+    if (fixed >= SMEM_LIMIT) return 0;
+    int st = (int)((SMEM_LIMIT - fixed) / per);
     if (st > MAX_STAGES) st = MAX_STAGES;
     return st;
 }
 
-template <int BITS, typename XT, typename YT>
+template <int BITS, typename XT, int NT>
 cudaError_t launch_t(const MmaParams& prm, int grid, size_t smem, cudaStream_t s) {
     static std::mutex mu;
     static bool done[64] = {false};
@@ -616,23 +733,34 @@ cudaError_t launch_t(const MmaParams& prm, int grid, size_t smem, cudaStream_t s
     {
         std::lock_guard<std::mutex> lk(mu);
         if (!done[dev]) {
-            e = cudaFuncSetAttribute(qmm_tc_kernel<BITS, XT, YT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            e = cudaFuncSetAttribute(qmm_tc_kernel<BITS, XT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)SMEM_LIMIT);
             if (e != cudaSuccess) return e;
             done[dev] = true;
         }
     }
-    qmm_tc_kernel<BITS, XT, YT><<<grid, MMA_THREADS, smem, s>>>(prm);
+    qmm_tc_kernel<BITS, XT, NT><<<grid, MMA_THREADS, smem, s>>>(prm);
     return cudaGetLastError();
 }
 
-template <typename XT, typename YT>
-cudaError_t launch_bits(int bits, const MmaParams& prm, int grid, size_t smem, cudaStream_t s) {
+template <int BITS, typename XT>
+cudaError_t launch_nt(int nt, const MmaParams& prm, int grid, size_t smem, cudaStream_t s) {
+    switch (nt) {
+        case 16: return launch_t<BITS, XT, 16>(prm, grid, smem, s);
+        case 32: return launch_t<BITS, XT, 32>(prm, grid, smem, s);
+        case 64: return launch_t<BITS, XT, 64>(prm, grid, smem, s);
+        case 128: return launch_t<BITS, XT, 128>(prm, grid, smem, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <typename XT>
+cudaError_t launch_bits(int bits, int nt, const MmaParams& prm, int grid, size_t smem, cudaStream_t s) {
     switch (bits) {
-        case 2: return launch_t<2, XT, YT>(prm, grid, smem, s);
-        case 4: return launch_t<4, XT, YT>(prm, grid, smem, s);
-        case 6: return launch_t<6, XT, YT>(prm, grid, smem, s);
-        case 8: return launch_t<8, XT, YT>(prm, grid, smem, s);
+        case 2: return launch_nt<2, XT>(nt, prm, grid, smem, s);
+        case 4: return launch_nt<4, XT>(nt, prm, grid, smem, s);
+        case 6: return launch_nt<6, XT>(nt, prm, grid, smem, s);
+        case 8: return launch_nt<8, XT>(nt, prm, grid, smem, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -657,6 +785,9 @@ bool mma_supported(const MmaProblem& p, const char** why) {
     }
     if (p.M > INT32_MAX / 2 || p.N * (p.offsets ? p.n_experts : 1) > INT32_MAX / 2)
         return no("problem too large for 32-bit tile coordinates");
+    const int nt = pick_nt(p);
+    if ((size_t)kg * nt * 4 > XTAB_MAX_BYTES || pick_stages(nt, p.bits, kg) < 2)
+        return no("K/group too large for the sum-of-x table of the tensor-core kernel");
     if (!get_encode()) return no("driver entry point cuTensorMapEncodeTiled unavailable");
     return true;
 }
@@ -668,17 +799,17 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     memset(&prm, 0, sizeof prm);
     const int nt = pick_nt(pb);
     const int bits = pb.bits;
-    const int stages = pick_stages(nt, bits);
-    const int64_t rows_total = pb.offsets ? pb.M : pb.M;
+    const int64_t kg = pb.K / pb.group;
+    const int stages = pick_stages(nt, bits, kg);
+    if (stages < 2) return cudaErrorInvalidValue;
+    const int64_t rows_total = pb.M;
     // ---- x tensor map: {K, rows, nb1, nb0}
     {
         cuuint64_t dims[4] = {(cuuint64_t)pb.K, (cuuint64_t)rows_total, (cuuint64_t)pb.nb[1], (cuuint64_t)pb.nb[0]};
-        const int64_t rowb = pb.x_row * 2;
-        int64_t s1 = pb.nb[1] > 1 ? pb.xb[1] * 2 : rowb * (rows_total > 0 ? rows_total : 1);
-        int64_t s2 = pb.nb[0] > 1 ? pb.xb[0] * 2 : s1 * (int64_t)pb.nb[1];
-        if (rows_total <= 1) { /* a single row: any 16-byte multiple works as its stride */ }
-        cuuint64_t strides[3] = {(cuuint64_t)(rows_total > 1 ? rowb : ((pb.K * 2 + 15) / 16 * 16)),
-                                 (cuuint64_t)((s1 + 15) / 16 * 16), (cuuint64_t)((s2 + 15) / 16 * 16)};
+        const int64_t rowb = rows_total > 1 ? pb.x_row * 2 : (pb.K * 2 + 15) / 16 * 16;
+        const int64_t s1 = pb.nb[1] > 1 ? pb.xb[1] * 2 : rowb * rows_total;
+        const int64_t s2 = pb.nb[0] > 1 ? pb.xb[0] * 2 : s1 * (int64_t)pb.nb[1];
+        cuuint64_t strides[3] = {(cuuint64_t)rowb, (cuuint64_t)((s1 + 15) / 16 * 16), (cuuint64_t)((s2 + 15) / 16 * 16)};
         cuuint32_t box[4] = {64, (cuuint32_t)nt, 1, 1};
         cuuint32_t estr[4] = {1, 1, 1, 1};
         CUresult r = encode(&prm.tx, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(pb.x), dims, strides, box,
@@ -700,26 +831,31 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
+    prm.x = pb.x;
     prm.y = pb.y;
     prm.scales = (const uint16_t*)pb.scales;
     prm.biases = (const uint16_t*)pb.biases;
     prm.M = pb.M;
     prm.N = pb.N;
     prm.K = pb.K;
+    prm.x_row = pb.x_row;
     prm.y_row = pb.y_row;
+    prm.xb[0] = pb.xb[0];
+    prm.xb[1] = pb.xb[1];
     prm.yb[0] = pb.yb[0];
     prm.yb[1] = pb.yb[1];
     prm.nb1 = pb.nb[1];
-    prm.nt = nt;
     prm.n_wtiles = (int)((pb.N + 127) / 128);
     prm.n_ttiles = (int)((pb.M + nt - 1) / nt);
     prm.nbatch = (int)(pb.nb[0] * pb.nb[1]);
+    prm.group = pb.group;
     int lg = 0;
     while ((1 << lg) < pb.group) ++lg;
     prm.log2g = lg;
     prm.stages = stages;
-    prm.kg = (int)(pb.K / pb.group);
-    uint32_t cols = SA * 32 + nt, pw = 32;
+    prm.kg = (int)kg;
+    prm.ydt = (int)pb.ydt;
+    uint32_t cols = SA * 32 + nbufs(nt) * nt, pw = 32;
     while (pw < cols) pw <<= 1;
     prm.tmem_cols = pw;
     prm.idesc = ptx::idesc_f16(nt, pb.xdt == DT::BF16 ? 1 : 0);
@@ -734,13 +870,9 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
         const int64_t tiles = (int64_t)prm.n_wtiles * prm.n_ttiles * prm.nbatch;
         grid = (int)(tiles < sms ? tiles : sms);
     }
-    const size_t smem = smem_for(nt, bits, stages);
-    if (pb.xdt == DT::BF16) {
-        return pb.ydt == DT::F32 ? launch_bits<bf16_t, float>(bits, prm, grid, smem, stream)
-                                 : launch_bits<bf16_t, bf16_t>(bits, prm, grid, smem, stream);
-    }
-    return pb.ydt == DT::F32 ? launch_bits<f16_t, float>(bits, prm, grid, smem, stream)
-                             : launch_bits<f16_t, f16_t>(bits, prm, grid, smem, stream);
+    const size_t smem = smem_for(nt, bits, stages, kg);
+    if (pb.xdt == DT::BF16) return launch_bits<bf16_t>(bits, nt, prm, grid, smem, stream);
+    return launch_bits<f16_t>(bits, nt, prm, grid, smem, stream);
 }
 
 cudaError_t read_and_clear_device_error(int* value, cudaStream_t s) {

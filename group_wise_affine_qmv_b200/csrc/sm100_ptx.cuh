@@ -172,6 +172,18 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* v) {
 }
 
 // ---------------------------------------------------------------------------
+// packed fp32 pairs (sm_100): d = a * b + c on two lanes at once, round to nearest
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)),
+          "l"(*reinterpret_cast<const uint64_t*>(&c)));
+    return *reinterpret_cast<const float2*>(&d);
+}
+
+// ---------------------------------------------------------------------------
 // UMMA descriptors
 // ---------------------------------------------------------------------------
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row core groups

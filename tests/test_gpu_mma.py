@@ -32,9 +32,9 @@ def _regime(x, wq, sc, bi, group, bits):
 
 
 @pytest.mark.parametrize("bits", [2, 4, 6, 8])
-@pytest.mark.parametrize("M,N,K", [(5, 129, 64), (16, 128, 128), (17, 300, 256), (32, 1000, 1024),
-                                   (33, 257, 512), (64, 640, 1024), (100, 200, 192), (256, 384, 640),
-                                   (300, 131, 320)])
+@pytest.mark.parametrize("M,N,K", [(5, 129, 128), (16, 128, 128), (17, 300, 256), (32, 1000, 1024),
+                                   (33, 257, 512), (64, 640, 1024), (100, 200, 256), (256, 384, 640),
+                                   (300, 131, 384)])
 def test_mma_shapes(bits, M, N, K):
     group = 64
     w = inputs.normal((N, K), 0.02, seed=M * 7 + N + K + bits)
@@ -145,6 +145,17 @@ def test_grouped_moe_bank_shape():
         for r in list(range(lo, min(hi, lo + 3))):
             ref = oracle.linear_contig(xb[r:r + 1], "bf16", wd[e])
             assert np.all(row_errors(y[r:r + 1], ref) <= 4e-3), (e, r)
+
+
+def test_odd_group_count_takes_gemv():
+    """K/group odd (K=192, G=64) is served by the GEMV kernel, still to the same bar."""
+    w = inputs.normal((100, 192), 0.02, seed=41)
+    Q, (wq, sc, bi) = _q(w, 64, 4)
+    x = inputs.normal((20, 192), 1.0, torch.bfloat16, seed=42)
+    xd = x.to(DEV)
+    assert _regime(xd, wq, sc, bi, 64, 4) == "qmv"
+    y = aq.aq_qmm_t(xd, wq, sc, bi, 64, 4)
+    assert np.all(row_errors(y, oracle_linear_view(x, Q.dequant())) <= 4e-3)
 
 
 def test_device_error_word_clear():
