@@ -47,8 +47,10 @@ def _stale(obj: str, src: str, newest_header: float) -> bool:
     return t < os.path.getmtime(src) or t < newest_header
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra_flags=None, out: str = LIB,
+          build_dir: str = BUILD) -> str:
+    """Compile csrc/*.cu into `out` (objects under `build_dir`)."""
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     newest_header = max([os.path.getmtime(h) for h in _headers()] + [0.0])
     cc = nvcc()
@@ -56,7 +58,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
     jobs = []
     objs = []
     for src in srcs:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _stale(obj, src, newest_header):
             jobs.append([cc] + ARCH + flags + ["-c", src, "-o", obj])
@@ -73,11 +75,11 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
     if jobs:
         with cf.ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 4)) as ex:
             list(ex.map(run, jobs))
-    if jobs or force or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if jobs or force or not os.path.exists(out) or any(os.path.getmtime(o) > os.path.getmtime(out) for o in objs):
+        tmp = out + f".tmp{os.getpid()}"
         run([cc] + ARCH + ["-shared", "-o", tmp] + objs + ["-Xlinker", "--exclude-libs,ALL"])
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, out)
+    return out
 
 
 def main(argv=None):
@@ -85,9 +87,16 @@ def main(argv=None):
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-v", action="store_true", help="print register/smem usage per kernel")
+    ap.add_argument("--trace", metavar="OUT",
+                    help="build a tracing variant (-DAQ_TRACE: per-wait-site time counters, aq_trace_read) into OUT")
     args = ap.parse_args(argv)
     extra = ["-Xptxas", "-v"] if args.ptxas_v else []
-    path = build(force=args.force or args.ptxas_v, verbose=args.verbose or args.ptxas_v, extra_flags=extra)
+    if args.trace:
+        out = os.path.abspath(args.trace)
+        path = build(force=args.force, verbose=args.verbose, extra_flags=extra + ["-DAQ_TRACE"], out=out,
+                     build_dir=os.path.join(BUILD, "trace"))
+    else:
+        path = build(force=args.force or args.ptxas_v, verbose=args.verbose or args.ptxas_v, extra_flags=extra)
     print(path)
 
 

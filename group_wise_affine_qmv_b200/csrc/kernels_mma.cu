@@ -49,6 +49,9 @@
 namespace aq {
 
 __device__ int g_device_error = 0;
+#ifdef AQ_TRACE
+__device__ unsigned long long g_trace[64];
+#endif
 
 namespace {
 
@@ -440,7 +443,7 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
                 for (int kb = 0; kb < KBLK; ++kb, ++it) {
                     const int st = it % S;
                     const uint32_t ph = (it / S) & 1;
-                    if (!ptx::mbar_wait(&s.empty[st], ph ^ 1, s.abort, WAIT_NS)) { ok = false; break; }
+                    if (!ptx::mbar_wait(&s.empty[st], ph ^ 1, s.abort, WAIT_NS, 0)) { ok = false; break; }
                     ptx::mbar_arrive_expect_tx(&s.full[st], bytes);
                     ptx::tma_load_4d(s.xs + (size_t)st * NT * 128, &p.tx, &s.full[st], kb * KB, (int32_t)ti.xrow0,
                                      ti.b1, ti.b0);
@@ -469,8 +472,8 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
                     const uint32_t ph = (it / S) & 1;
                     const int a = it % SA;
                     const uint32_t aph = (it / SA) & 1;
-                    if (!ptx::mbar_wait(&s.full[st], ph, s.abort, WAIT_NS) ||
-                        !ptx::mbar_wait(&s.afull[a], aph, s.abort, WAIT_NS)) {
+                    if (!ptx::mbar_wait(&s.full[st], ph, s.abort, WAIT_NS, 1) ||
+                        !ptx::mbar_wait(&s.afull[a], aph, s.abort, WAIT_NS, 2)) {
                         ok = false;
                         break;
                     }
@@ -483,7 +486,7 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
                         const uint32_t buf = gc % NB;
                         if (gstart) {
                             // this accumulator's previous group must have been read by the epilogue
-                            if (!ptx::mbar_wait(&s.gempty[buf], ((gc / NB) & 1) ^ 1, s.abort, WAIT_NS)) {
+                            if (!ptx::mbar_wait(&s.gempty[buf], ((gc / NB) & 1) ^ 1, s.abort, WAIT_NS, 3)) {
                                 ok = false;
                                 break;
                             }
@@ -533,7 +536,7 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
         // epilogue of group g of the current tile: acc += s*D_g + b*X_g
         auto epilogue_group = [&](int g) -> bool {
             const uint32_t buf = ge % NB;
-            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&s.gfull[buf], (ge / NB) & 1, s.abort, WAIT_NS)))
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&s.gfull[buf], (ge / NB) & 1, s.abort, WAIT_NS, 6)))
                 return false;
             ptx::tc_fence_after();
             const int gl = g - g_chunk0;
@@ -549,7 +552,11 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
                 } else {
                     ptx::tmem_ld8(d_tmem + buf * NT + lane_base + h * H + c0, v);
                 }
+#ifdef AQ_TRACE
+                { const uint64_t w0 = ptx::globaltimer_ns(); ptx::tc_wait_ld(); AQ_TRACE_ADD(10, ptx::globaltimer_ns() - w0); }
+#else
                 ptx::tc_wait_ld();
+#endif
                 constexpr int CNT = H >= 16 ? 16 : H;
 #pragma unroll
                 for (int c = 0; c < CNT; c += 4) {
@@ -592,8 +599,10 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
             for (int i = 0; i < H / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
             int g_next = 0;  // next group of this tile awaiting its epilogue
             for (int kb = 0; kb < KBLK; ++kb, ++it) {
-                // (1) epilogues of the groups that ended LAG stages before this one
-                while (g_next < NG && (g_next + 1) * G <= (kb - LAG + 1) * KB) {
+                // (1) epilogues of the groups that ended LAG stages before this one; entering a
+                //     new scale/bias chunk, every group of the previous chunk (its slot is reused)
+                const int fold_end = (kb % CS == 0) ? kb * KB : (kb - LAG + 1) * KB;
+                while (g_next < NG && (g_next + 1) * G <= fold_end) {
                     if (!epilogue_group(g_next)) { ok = false; break; }
                     ++g_next;
                 }
@@ -602,7 +611,7 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
                 if (kb % CS == 0) {
                     ptx::cp_async_wait_all();
                     ptx::mbar_arrive(&s.sbar[unit & 1]);
-                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS));
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS, 7));
                     if (!ok) break;
                     slot = s.sb + (unit & 1) * 2 * 128 * SCP;
                     const int c = kb / CS;
@@ -622,16 +631,20 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
                 const uint32_t ph = (it / S) & 1;
                 const int a = it % SA;
                 const uint32_t aph = (it / SA) & 1;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.full[st], ph, s.abort, WAIT_NS));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.full[st], ph, s.abort, WAIT_NS, 4));
                 if (!ok) break;
                 uint32_t wv[BITS];
                 load_w32<BITS>(s.ws + (size_t)st * 1024 * BITS, row, h, wv);
                 uint32_t out[16];
                 expand32<BITS, XT>(wv, out);
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.aempty[a], aph ^ 1, s.abort, WAIT_NS));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.aempty[a], aph ^ 1, s.abort, WAIT_NS, 5));
                 if (!ok) break;
                 ptx::tmem_st16(tbase + lane_base + a * 32 + 16 * h, out);
+#ifdef AQ_TRACE
+                { const uint64_t w0 = ptx::globaltimer_ns(); ptx::tc_wait_st(); AQ_TRACE_ADD(9, ptx::globaltimer_ns() - w0); }
+#else
                 ptx::tc_wait_st();
+#endif
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&s.afull[a]);
@@ -874,6 +887,18 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     if (pb.xdt == DT::BF16) return launch_bits<bf16_t>(bits, nt, prm, grid, smem, stream);
     return launch_bits<f16_t>(bits, nt, prm, grid, smem, stream);
 }
+
+#ifdef AQ_TRACE
+extern "C" __attribute__((visibility("default"))) int aq_trace_read(unsigned long long* out, int reset) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    if (cudaMemcpyFromSymbol(out, g_trace, sizeof(unsigned long long) * 64) != cudaSuccess) return -1;
+    if (reset) {
+        unsigned long long z[64] = {0};
+        if (cudaMemcpyToSymbol(g_trace, z, sizeof z) != cudaSuccess) return -1;
+    }
+    return 0;
+}
+#endif
 
 cudaError_t read_and_clear_device_error(int* value, cudaStream_t s) {
     cudaError_t e = cudaStreamSynchronize(s);

@@ -53,11 +53,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
     return ok != 0;
 }
 
+#ifdef AQ_TRACE
+// Trace builds only: nanoseconds spent (lane 0 of each waiting warp) and number of
+// waits per wait site, accumulated over all CTAs; read back with aq_trace_read().
+extern __device__ unsigned long long g_trace[64];
+#define AQ_TRACE_ADD(site, ns)                                  \
+    do {                                                        \
+        if ((threadIdx.x & 31) == 0) {                          \
+            atomicAdd(&g_trace[(site)], (unsigned long long)(ns)); \
+            atomicAdd(&g_trace[32 + (site)], 1ull);             \
+        }                                                       \
+    } while (0)
+#endif
+
 // Wait for the phase of parity `parity` to complete.  Returns false if the
 // budget ran out or *abort became non-zero (another warp gave up).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint64_t budget_ns) {
+                                          uint64_t budget_ns, int site = -1) {
     const uint32_t a = smem_u32(bar);
+#ifdef AQ_TRACE
+    const uint64_t tt0 = globaltimer_ns();
+    bool done = mbar_try_wait(a, parity);
+    if (!done) {
+        for (uint32_t i = 1;; ++i) {
+            if (mbar_try_wait(a, parity)) { done = true; break; }
+            if ((i & 63u) == 0 && (*abort || globaltimer_ns() - tt0 > budget_ns)) break;
+        }
+    }
+    if (site >= 0) AQ_TRACE_ADD(site, globaltimer_ns() - tt0);
+    return done;
+#else
+    (void)site;
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
@@ -67,6 +93,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
             if (globaltimer_ns() - t0 > budget_ns) return false;
         }
     }
+#endif
 }
 
 // ---------------------------------------------------------------------------
