@@ -49,22 +49,30 @@
 namespace aq {
 
 __device__ int g_device_error = 0;
-#ifdef AQ_TRACE
-__device__ unsigned long long g_trace[64];
-#endif
 
 namespace {
 
 constexpr int MMA_THREADS = 320;          // 10 warps
 constexpr int DQ_THREADS = 256;           // warps 2..9
-constexpr int KB = 64;                    // codes per pipeline stage
+constexpr int KB = 64;                    // codes per MMA sub-step (4 tcgen05.mma of K = 16)
 constexpr int SA = 4;                     // A slots in tensor memory, 32 columns each
 constexpr int SCW = 32;                   // groups per scale/bias chunk
 constexpr int SCP = SCW + 2;              // padded row pitch (halves) of a chunk in shared memory
 constexpr int MAX_STAGES = 16;
+constexpr int MAX_XSLOTS = 16;
 constexpr int MAX_EXPERTS = 1024;
 constexpr int XTAB_MAX_BYTES = 48 * 1024; // sum-of-x table per token tile
 constexpr int NBMAX = 4;                  // group accumulators in tensor memory
+
+// One pipeline stage of W is 128 rows x ROWB bytes: a full 128-byte swizzle atom per row for
+// 2/4/8-bit codes (so each TMA request moves a 128-byte line), 96 bytes for 6-bit.  A stage
+// holds SUB sub-steps of 64 codes.
+template <int BITS> struct WStage {
+    static constexpr int ROWB = BITS == 6 ? 96 : 128;
+    static constexpr int CODES = ROWB * 8 / BITS;
+    static constexpr int SUB = CODES / KB;
+    static constexpr int BYTES = 128 * ROWB;
+};
 
 // group accumulators for a token-tile width: 4 while they fit beside the A slots
 __host__ __device__ constexpr int nbufs(int nt) { return nt <= 64 ? 4 : 2; }
@@ -86,6 +94,9 @@ struct MmaParams {
     int group, log2g;
     int stages;
     int kg;              // groups per row = K / group
+    int xres;            // 1: the CTA's single x tile stays resident in shared memory
+    int xslots;          // streaming x: ring slots of [NT x 64] (one per MMA sub-step)
+    int n_wstages;       // W pipeline stages per tile
     int ydt;             // DT of y
     uint32_t tmem_cols;
     uint32_t idesc;
@@ -114,12 +125,15 @@ struct Smem {
     uint64_t* sbar;      // [2] scale/bias chunk slots: 256 dequant-thread arrivals
     uint64_t* xbar;      // sum-of-x table barrier: 256 arrivals
     uint64_t* mdone;     // all MMAs of this CTA retired (teardown)
+    uint64_t* xfull;     // resident x tile landed
+    uint64_t* xsfull;    // [MAX_XSLOTS] streaming x slot landed (TMA)
+    uint64_t* xsempty;   // [MAX_XSLOTS] streaming x slot consumed (MMA commit)
     uint32_t* tmem_base;
     int* abort;
     int* prefix;         // grouped: tile prefix sums [n_experts + 1]
     float* xtab;         // [kg][NT] sums of x per group and token
-    uint8_t* xs;         // stages * NT * 128
-    uint8_t* ws;         // stages * 1024 * bits
+    uint8_t* xs;         // resident: [K/64][NT][128 B]; streaming: xslots x [NT][128 B]
+    uint8_t* ws;         // stages x [128 rows][ROWB]
     uint16_t* sb;        // [2 slots][2 arrays][128][SCP]
 };
 
@@ -128,9 +142,9 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const MmaParams& p) {
     Smem s;
     uint8_t* q = base;
     s.xs = q;
-    q += (size_t)p.stages * NT * 128;
+    q += p.xres ? (size_t)(p.K / KB) * NT * 128 : (size_t)p.xslots * NT * 128;
     s.ws = q;
-    q += (size_t)p.stages * 1024 * BITS;
+    q += (size_t)p.stages * WStage<BITS>::BYTES;
     s.xtab = reinterpret_cast<float*>(q);
     q += (size_t)p.kg * NT * 4;
     s.sb = reinterpret_cast<uint16_t*>(q);
@@ -144,14 +158,17 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const MmaParams& p) {
     s.sbar = s.gempty + NBMAX;
     s.xbar = s.sbar + 2;
     s.mdone = s.xbar + 1;
-    s.tmem_base = reinterpret_cast<uint32_t*>(s.mdone + 1);
+    s.xfull = s.mdone + 1;
+    s.xsfull = s.xfull + 1;
+    s.xsempty = s.xsfull + MAX_XSLOTS;
+    s.tmem_base = reinterpret_cast<uint32_t*>(s.xsempty + MAX_XSLOTS);
     s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
     s.prefix = s.abort + 1;
     return s;
 }
 
 __host__ __device__ constexpr size_t smem_fixed_bytes() {
-    return 2 * 2 * 128 * SCP * 2 + (2 * MAX_STAGES + 2 * SA + 2 * NBMAX + 5) * 8 + 8 + (MAX_EXPERTS + 1) * 4 + 1024 /*align*/;
+    return 2 * 2 * 128 * SCP * 2 + (2 * MAX_STAGES + 2 * MAX_XSLOTS + 2 * SA + 2 * NBMAX + 6) * 8 + 8 + (MAX_EXPERTS + 1) * 4 + 1024 /*align*/;
 }
 
 __device__ __forceinline__ void raise_abort(int* abort) {
@@ -204,30 +221,29 @@ __device__ __forceinline__ TileInfo tile_info(const MmaParams& p, const Smem& s,
 // in the 16-bit MMA type (low half = even code)
 // ---------------------------------------------------------------------------
 
-// swizzled byte offset of a 16-byte chunk written by TMA (bits 4.. XOR bits 7..)
+// This thread's 32 codes (sub-step j, half h) of W row `row` in a stage.  Rows are ROWB bytes
+// apart; with a 128-byte swizzle, 16-byte chunk c of row r sits at chunk c ^ (r & 7).
 template <int BITS>
-__device__ __forceinline__ uint32_t wswz(uint32_t off) {
-    if constexpr (BITS == 4) return off ^ (((off >> 7) & 1u) << 4);      // 32-byte swizzle
-    else if constexpr (BITS == 8) return off ^ (((off >> 7) & 3u) << 4); // 64-byte swizzle
-    else return off;
-}
-
-template <int BITS>
-__device__ __forceinline__ void load_w32(const uint8_t* stage, int row, int h, uint32_t* w) {
-    constexpr uint32_t RB = 8 * BITS;  // bytes per row per stage (64 codes)
-    const uint32_t base = (uint32_t)row * RB + (uint32_t)h * (RB / 2);
+__device__ __forceinline__ void load_w32(const uint8_t* stage, int row, int j, int h, uint32_t* w) {
+    constexpr int ROWB = WStage<BITS>::ROWB;
+    const uint32_t b = (uint32_t)(j * KB + 32 * h) * BITS / 8;  // byte offset within the row
+    const uint8_t* r = stage + (uint32_t)row * ROWB;
+    const uint32_t sw = ROWB == 128 ? ((uint32_t)(row & 7) << 4) : 0u;
     if constexpr (BITS == 4) {
-        const uint4 v = *reinterpret_cast<const uint4*>(stage + wswz<4>(base));
+        const uint4 v = *reinterpret_cast<const uint4*>(r + (b ^ sw));
         w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
     } else if constexpr (BITS == 8) {
-        const uint4 v0 = *reinterpret_cast<const uint4*>(stage + wswz<8>(base));
-        const uint4 v1 = *reinterpret_cast<const uint4*>(stage + wswz<8>(base + 16));
+        const uint4 v0 = *reinterpret_cast<const uint4*>(r + (b ^ sw));
+        const uint4 v1 = *reinterpret_cast<const uint4*>(r + ((b + 16) ^ sw));
         w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
         w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+    } else if constexpr (BITS == 2) {
+        const uint2 v = *reinterpret_cast<const uint2*>(r + (((b & ~15u) ^ sw) | (b & 15u)));
+        w[0] = v.x; w[1] = v.y;
     } else {
 #pragma unroll
         for (int i = 0; i < BITS / 2; ++i) {
-            const uint2 v = *reinterpret_cast<const uint2*>(stage + base + 8 * i);
+            const uint2 v = *reinterpret_cast<const uint2*>(r + b + 8 * i);
             w[2 * i] = v.x; w[2 * i + 1] = v.y;
         }
     }
@@ -357,6 +373,8 @@ template <int BITS, typename XT, int NT>
 __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_constant__ MmaParams p) {
     constexpr int H = NT / 2;            // tokens per epilogue thread
     constexpr int NB = nbufs(NT);        // group accumulators
+    constexpr int SUB = WStage<BITS>::SUB;
+    const int NWS = p.n_wstages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const Smem s = carve<BITS, NT>(base, p);
@@ -376,6 +394,9 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
     if (LAG > 3) LAG = 3;
     if (LAG < 1) LAG = 1;
 
+#ifdef AQ_TRACE
+    if (threadIdx.x < 64) ::aq_trace_smem[threadIdx.x] = 0;
+#endif
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
             ptx::mbar_init(&s.full[i], 1);
@@ -393,6 +414,11 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
         ptx::mbar_init(&s.sbar[1], DQ_THREADS);
         ptx::mbar_init(s.xbar, DQ_THREADS);
         ptx::mbar_init(s.mdone, 1);
+        ptx::mbar_init(s.xfull, 1);
+        for (int i = 0; i < p.xslots; ++i) {
+            ptx::mbar_init(&s.xsfull[i], 1);
+            ptx::mbar_init(&s.xsempty[i], 1);
+        }
         *s.abort = 0;
         ptx::fence_mbar_init();
     }
@@ -435,72 +461,115 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
     if (warp == 0) {
         // ======================= TMA producer =======================
         if (lane == 0) {
-            const uint32_t bytes = (uint32_t)NT * 128 + 1024u * BITS;
-            uint32_t it = 0;
+            const uint32_t bytes = WStage<BITS>::BYTES;
+            const int SX = p.xslots;
+            uint32_t wit = 0, xit = 0;
             bool ok = true;
+            if (p.xres && (int)blockIdx.x < ntiles) {
+                // the CTA's only token tile: all of K, once
+                const TileInfo t0 = tile_info<NT>(p, s, blockIdx.x);
+                ptx::mbar_arrive_expect_tx(s.xfull, (uint32_t)KBLK * NT * 128);
+                for (int kb = 0; kb < KBLK; ++kb)
+                    ptx::tma_load_4d(s.xs + (size_t)kb * NT * 128, &p.tx, s.xfull, kb * KB, (int32_t)t0.xrow0, t0.b1,
+                                     t0.b0);
+            }
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 const TileInfo ti = tile_info<NT>(p, s, t);
-                for (int kb = 0; kb < KBLK; ++kb, ++it) {
-                    const int st = it % S;
-                    const uint32_t ph = (it / S) & 1;
+                for (int w = 0; w < NWS; ++w, ++wit) {
+                    const int st = wit % S;
+                    const uint32_t ph = (wit / S) & 1;
                     if (!ptx::mbar_wait(&s.empty[st], ph ^ 1, s.abort, WAIT_NS, 0)) { ok = false; break; }
                     ptx::mbar_arrive_expect_tx(&s.full[st], bytes);
-                    ptx::tma_load_4d(s.xs + (size_t)st * NT * 128, &p.tx, &s.full[st], kb * KB, (int32_t)ti.xrow0,
-                                     ti.b1, ti.b0);
-                    ptx::tma_load_2d(s.ws + (size_t)st * 1024 * BITS, &p.tw, &s.full[st], kb * 2 * BITS,
-                                     (int32_t)ti.wrow0);
+                    ptx::tma_load_2d(s.ws + (size_t)st * WStage<BITS>::BYTES, &p.tw, &s.full[st],
+                                     w * (WStage<BITS>::ROWB / 4), (int32_t)ti.wrow0);
+                    if (!p.xres) {
+                        for (int j = 0; j < SUB && ok; ++j, ++xit) {
+                            const int kb = w * SUB + j;
+                            if (kb >= KBLK) break;
+                            const int xsl = xit % SX;
+                            if (!ptx::mbar_wait(&s.xsempty[xsl], ((xit / SX) & 1) ^ 1, s.abort, WAIT_NS, 0)) {
+                                ok = false;
+                                break;
+                            }
+                            ptx::mbar_arrive_expect_tx(&s.xsfull[xsl], (uint32_t)NT * 128);
+                            ptx::tma_load_4d(s.xs + (size_t)xsl * NT * 128, &p.tx, &s.xsfull[xsl], kb * KB,
+                                             (int32_t)ti.xrow0, ti.b1, ti.b0);
+                        }
+                    }
                 }
             }
             if (!ok) {
                 raise_abort(s.abort);
                 // drain: the copies of every issued stage must land before the CTA exits
                 volatile int never = 0;
-                const uint32_t first = it >= (uint32_t)S ? it - S : 0;
-                for (uint32_t j = first; j < it; ++j)
-                    ptx::mbar_wait(&s.full[j % S], (j / S) & 1, &never, 200000000ull);
+                const uint32_t first = wit >= (uint32_t)S ? wit - S : 0;
+                for (uint32_t jj = first; jj < wit; ++jj)
+                    ptx::mbar_wait(&s.full[jj % S], (jj / S) & 1, &never, 200000000ull);
+                const uint32_t xfirst = xit >= (uint32_t)SX ? xit - SX : 0;
+                for (uint32_t jj = xfirst; jj < xit; ++jj)
+                    ptx::mbar_wait(&s.xsfull[jj % SX], (jj / SX) & 1, &never, 200000000ull);
+            }
+            if (p.xres && (int)blockIdx.x < ntiles) {
+                volatile int never = 0;
+                ptx::mbar_wait(s.xfull, 0, &never, 200000000ull);
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         // ======================= MMA issuer =======================
         if (lane == 0) {
-            uint32_t it = 0, gc = 0;
+            uint32_t it = 0, gc = 0, wit = 0, xit = 0;
+            const int SX = p.xslots;
             bool ok = true;
+            if (p.xres && (int)blockIdx.x < ntiles)
+                ok = ptx::mbar_wait(s.xfull, 0, s.abort, WAIT_NS, 1);
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                for (int kb = 0; kb < KBLK && ok; ++kb, ++it) {
-                    const int st = it % S;
-                    const uint32_t ph = (it / S) & 1;
-                    const int a = it % SA;
-                    const uint32_t aph = (it / SA) & 1;
-                    if (!ptx::mbar_wait(&s.full[st], ph, s.abort, WAIT_NS, 1) ||
-                        !ptx::mbar_wait(&s.afull[a], aph, s.abort, WAIT_NS, 2)) {
-                        ok = false;
-                        break;
-                    }
-                    ptx::tc_fence_after();
-                    const uint32_t xaddr = ptx::smem_u32(s.xs + (size_t)st * NT * 128);
+                for (int w = 0; w < NWS && ok; ++w, ++wit) {
+                    const int st = wit % S;
+                    const uint32_t ph = (wit / S) & 1;
+                    (void)ph;
+                    for (int j = 0; j < SUB && ok; ++j) {
+                        const int kb = w * SUB + j;
+                        if (kb >= KBLK) break;
+                        const int a = it % SA;
+                        const uint32_t aph = (it / SA) & 1;
+                        const int xsl = xit % SX;
+                        if (!p.xres && !ptx::mbar_wait(&s.xsfull[xsl], (xit / SX) & 1, s.abort, WAIT_NS, 1)) {
+                            ok = false;
+                            break;
+                        }
+                        if (!ptx::mbar_wait(&s.afull[a], aph, s.abort, WAIT_NS, 2)) { ok = false; break; }
+                        ptx::tc_fence_after();
+                        const uint32_t xaddr =
+                            ptx::smem_u32(p.xres ? s.xs + (size_t)kb * NT * 128 : s.xs + (size_t)xsl * NT * 128);
 #pragma unroll
-                    for (int j = 0; j < KB / 16; ++j) {
-                        const int k = kb * KB + 16 * j;
-                        const bool gstart = (k & (G - 1)) == 0;
-                        const uint32_t buf = gc % NB;
-                        if (gstart) {
-                            // this accumulator's previous group must have been read by the epilogue
-                            if (!ptx::mbar_wait(&s.gempty[buf], ((gc / NB) & 1) ^ 1, s.abort, WAIT_NS, 3)) {
-                                ok = false;
-                                break;
+                        for (int kk = 0; kk < KB / 16; ++kk) {
+                            const int k = kb * KB + 16 * kk;
+                            const bool gstart = (k & (G - 1)) == 0;
+                            const uint32_t buf = gc % NB;
+                            if (gstart) {
+                                // this accumulator's previous group must have been read by the epilogue
+                                if (!ptx::mbar_wait(&s.gempty[buf], ((gc / NB) & 1) ^ 1, s.abort, WAIT_NS, 3)) {
+                                    ok = false;
+                                    break;
+                                }
+                                ptx::tc_fence_after();
                             }
-                            ptx::tc_fence_after();
+                            const uint64_t bdesc = ptx::smem_desc_sw128(xaddr + 32 * kk);
+                            ptx::mma_ts(d_tmem + buf * NT, tbase + a * 32 + kk * 8, bdesc, p.idesc, gstart ? 0u : 1u);
+                            if (((k + 16) & (G - 1)) == 0) {
+                                ptx::mma_commit(&s.gfull[buf]);
+                                ++gc;
+                            }
                         }
-                        const uint64_t bdesc = ptx::smem_desc_sw128(xaddr + 32 * j);
-                        ptx::mma_ts(d_tmem + buf * NT, tbase + a * 32 + j * 8, bdesc, p.idesc, gstart ? 0u : 1u);
-                        if (((k + 16) & (G - 1)) == 0) {
-                            ptx::mma_commit(&s.gfull[buf]);
-                            ++gc;
+                        ptx::mma_commit(&s.aempty[a]);
+                        if (!p.xres) {
+                            ptx::mma_commit(&s.xsempty[xsl]);
+                            ++xit;
                         }
+                        ++it;
                     }
                     ptx::mma_commit(&s.empty[st]);
-                    ptx::mma_commit(&s.aempty[a]);
                 }
             }
             if (!ok) raise_abort(s.abort);
@@ -517,7 +586,7 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
         const int row = 32 * q + lane;          // W row within the tile == TMEM lane
         const int tid = threadIdx.x - 64;       // 0..255
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        uint32_t it = 0, ge = 0, xph = 0;
+        uint32_t it = 0, ge = 0, xph = 0, wit = 0;
         int unit = 0;
         bool ok = true;
         int64_t cur_x0 = -1;
@@ -598,56 +667,62 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
 #pragma unroll
             for (int i = 0; i < H / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
             int g_next = 0;  // next group of this tile awaiting its epilogue
-            for (int kb = 0; kb < KBLK; ++kb, ++it) {
-                // (1) epilogues of the groups that ended LAG stages before this one; entering a
-                //     new scale/bias chunk, every group of the previous chunk (its slot is reused)
-                const int fold_end = (kb % CS == 0) ? kb * KB : (kb - LAG + 1) * KB;
-                while (g_next < NG && (g_next + 1) * G <= fold_end) {
-                    if (!epilogue_group(g_next)) { ok = false; break; }
-                    ++g_next;
-                }
-                if (!ok) break;
-                // (2) next scale/bias chunk
-                if (kb % CS == 0) {
-                    ptx::cp_async_wait_all();
-                    ptx::mbar_arrive(&s.sbar[unit & 1]);
-                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS, 7));
-                    if (!ok) break;
-                    slot = s.sb + (unit & 1) * 2 * 128 * SCP;
-                    const int c = kb / CS;
-                    g_chunk0 = c * SCW;
-                    uint16_t* nslot = s.sb + ((unit + 1) & 1) * 2 * 128 * SCP;
-                    if (c + 1 < NCH) {
-                        issue_sb_chunk(p, ti, c + 1, nslot, tid);
-                    } else if (t + (int)gridDim.x < ntiles) {
-                        const TileInfo tn = tile_info<NT>(p, s, t + gridDim.x);
-                        issue_sb_chunk(p, tn, 0, nslot, tid);
-                    }
-                    ptx::cp_async_commit();
-                    ++unit;
-                }
-                // (3) expand this stage's codes into an A slot
-                const int st = it % S;
-                const uint32_t ph = (it / S) & 1;
-                const int a = it % SA;
-                const uint32_t aph = (it / SA) & 1;
+            for (int w = 0; w < NWS && ok; ++w, ++wit) {
+                const int st = wit % S;
+                const uint32_t ph = (wit / S) & 1;
                 ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.full[st], ph, s.abort, WAIT_NS, 4));
                 if (!ok) break;
-                uint32_t wv[BITS];
-                load_w32<BITS>(s.ws + (size_t)st * 1024 * BITS, row, h, wv);
-                uint32_t out[16];
-                expand32<BITS, XT>(wv, out);
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.aempty[a], aph ^ 1, s.abort, WAIT_NS, 5));
-                if (!ok) break;
-                ptx::tmem_st16(tbase + lane_base + a * 32 + 16 * h, out);
+                const uint8_t* wstage = s.ws + (size_t)st * WStage<BITS>::BYTES;
+                for (int j = 0; j < SUB; ++j, ++it) {
+                    const int kb = w * SUB + j;
+                    if (kb >= KBLK) break;
+                    // (1) epilogues of the groups that ended LAG sub-steps before this one; entering a
+                    //     new scale/bias chunk, every group of the previous chunk (its slot is reused)
+                    const int fold_end = (kb % CS == 0) ? kb * KB : (kb - LAG + 1) * KB;
+                    while (g_next < NG && (g_next + 1) * G <= fold_end) {
+                        if (!epilogue_group(g_next)) { ok = false; break; }
+                        ++g_next;
+                    }
+                    if (!ok) break;
+                    // (2) next scale/bias chunk
+                    if (kb % CS == 0) {
+                        ptx::cp_async_wait_all();
+                        ptx::mbar_arrive(&s.sbar[unit & 1]);
+                        ok = __all_sync(0xffffffffu,
+                                        ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS, 7));
+                        if (!ok) break;
+                        slot = s.sb + (unit & 1) * 2 * 128 * SCP;
+                        const int c = kb / CS;
+                        g_chunk0 = c * SCW;
+                        uint16_t* nslot = s.sb + ((unit + 1) & 1) * 2 * 128 * SCP;
+                        if (c + 1 < NCH) {
+                            issue_sb_chunk(p, ti, c + 1, nslot, tid);
+                        } else if (t + (int)gridDim.x < ntiles) {
+                            const TileInfo tn = tile_info<NT>(p, s, t + gridDim.x);
+                            issue_sb_chunk(p, tn, 0, nslot, tid);
+                        }
+                        ptx::cp_async_commit();
+                        ++unit;
+                    }
+                    // (3) expand this sub-step's codes into an A slot
+                    const int a = it % SA;
+                    const uint32_t aph = (it / SA) & 1;
+                    uint32_t wv[BITS];
+                    load_w32<BITS>(wstage, row, j, h, wv);
+                    uint32_t out[16];
+                    expand32<BITS, XT>(wv, out);
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.aempty[a], aph ^ 1, s.abort, WAIT_NS, 5));
+                    if (!ok) break;
+                    ptx::tmem_st16(tbase + lane_base + a * 32 + 16 * h, out);
 #ifdef AQ_TRACE
-                { const uint64_t w0 = ptx::globaltimer_ns(); ptx::tc_wait_st(); AQ_TRACE_ADD(9, ptx::globaltimer_ns() - w0); }
+                    { const uint64_t w0 = ptx::globaltimer_ns(); ptx::tc_wait_st(); AQ_TRACE_ADD(9, ptx::globaltimer_ns() - w0); }
 #else
-                ptx::tc_wait_st();
+                    ptx::tc_wait_st();
 #endif
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&s.afull[a]);
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&s.afull[a]);
+                }
             }
             if (!ok) break;
             while (g_next < NG) {
@@ -678,6 +753,9 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tbase, p.tmem_cols);
     }
+#ifdef AQ_TRACE
+    if (threadIdx.x < 64) atomicAdd(&::aq_trace_ns[threadIdx.x], ::aq_trace_smem[threadIdx.x]);
+#endif
 }
 
 // ---------------------------------------------------------------------------
@@ -720,19 +798,45 @@ int pick_nt(const MmaProblem& p) {
     return 128;
 }
 
+#ifdef AQ_TRACE
+constexpr size_t SMEM_LIMIT = 226 * 1024;  // the trace counters take static shared memory
+#else
 constexpr size_t SMEM_LIMIT = 227 * 1024;
+#endif
 
-size_t smem_for(int nt, int bits, int stages, int64_t kg) {
-    return (size_t)stages * ((size_t)nt * 128 + 1024 * (size_t)bits) + (size_t)kg * nt * 4 + smem_fixed_bytes();
+int wstage_rowb(int bits) { return bits == 6 ? 96 : 128; }
+int wstage_sub(int bits) { return wstage_rowb(bits) * 8 / bits / KB; }
+
+// shared memory of one pipeline stage, and of the parts that do not depend on the stage count
+size_t stage_bytes(int bits) { return (size_t)128 * wstage_rowb(bits); }
+size_t fixed_bytes(int nt, int64_t K, int64_t kg, int xres, int xslots) {
+    return (xres ? (size_t)(K / KB) * nt * 128 : (size_t)xslots * nt * 128) + (size_t)kg * nt * 4 +
+           smem_fixed_bytes();
 }
-
-int pick_stages(int nt, int bits, int64_t kg) {
-    const size_t per = (size_t)nt * 128 + 1024 * (size_t)bits;
-    const size_t fixed = (size_t)kg * nt * 4 + smem_fixed_bytes();
+size_t smem_for(int nt, int bits, int stages, int64_t K, int64_t kg, int xres, int xslots) {
+    return (size_t)stages * stage_bytes(bits) + fixed_bytes(nt, K, kg, xres, xslots);
+}
+int pick_stages(int nt, int bits, int64_t K, int64_t kg, int xres, int xslots) {
+    const size_t fixed = fixed_bytes(nt, K, kg, xres, xslots);
     if (fixed >= SMEM_LIMIT) return 0;
-    int st = (int)((SMEM_LIMIT - fixed) / per);
+    int st = (int)((SMEM_LIMIT - fixed) / stage_bytes(bits));
     if (st > MAX_STAGES) st = MAX_STAGES;
     return st;
+}
+constexpr int MIN_STAGES = 3;
+constexpr int MIN_XSLOTS = 4;
+// streaming x: as many [NT x 64] slots as leave MIN_STAGES + 1 W stages (at most MAX_XSLOTS)
+int pick_xslots(int nt, int bits, int64_t K, int64_t kg) {
+    int best = 0;
+    for (int xs = MIN_XSLOTS; xs <= MAX_XSLOTS; ++xs)
+        if (pick_stages(nt, bits, K, kg, 0, xs) >= MIN_STAGES + 1) best = xs;
+    if (best == 0 && pick_stages(nt, bits, K, kg, 0, MIN_XSLOTS) >= MIN_STAGES) best = MIN_XSLOTS;
+    return best;
+}
+// x stays resident when a CTA sees one token tile and it leaves room for the W pipeline
+int pick_xres(const MmaProblem& p, int nt, int64_t kg) {
+    if (p.offsets || p.M > nt || p.nb[0] * p.nb[1] != 1) return 0;
+    return pick_stages(nt, p.bits, p.K, kg, 1, 0) >= MIN_STAGES + 1 ? 1 : 0;
 }
 
 template <int BITS, typename XT, int NT>
@@ -799,7 +903,7 @@ bool mma_supported(const MmaProblem& p, const char** why) {
     if (p.M > INT32_MAX / 2 || p.N * (p.offsets ? p.n_experts : 1) > INT32_MAX / 2)
         return no("problem too large for 32-bit tile coordinates");
     const int nt = pick_nt(p);
-    if ((size_t)kg * nt * 4 > XTAB_MAX_BYTES || pick_stages(nt, p.bits, kg) < 2)
+    if ((size_t)kg * nt * 4 > XTAB_MAX_BYTES || (pick_xres(p, nt, kg) == 0 && pick_xslots(nt, p.bits, p.K, kg) == 0))
         return no("K/group too large for the sum-of-x table of the tensor-core kernel");
     if (!get_encode()) return no("driver entry point cuTensorMapEncodeTiled unavailable");
     return true;
@@ -813,8 +917,10 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     const int nt = pick_nt(pb);
     const int bits = pb.bits;
     const int64_t kg = pb.K / pb.group;
-    const int stages = pick_stages(nt, bits, kg);
-    if (stages < 2) return cudaErrorInvalidValue;
+    const int xres = pick_xres(pb, nt, kg);
+    const int xslots = xres ? 0 : pick_xslots(nt, bits, pb.K, kg);
+    const int stages = pick_stages(nt, bits, pb.K, kg, xres, xslots);
+    if (stages < MIN_STAGES || (!xres && xslots < MIN_XSLOTS)) return cudaErrorInvalidValue;
     const int64_t rows_total = pb.M;
     // ---- x tensor map: {K, rows, nb1, nb0}
     {
@@ -835,10 +941,9 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
         const int64_t wrows = pb.offsets ? pb.N * pb.n_experts : pb.N;
         cuuint64_t dims[2] = {(cuuint64_t)(pb.K * bits / 32), (cuuint64_t)wrows};
         cuuint64_t strides[1] = {(cuuint64_t)(pb.w_row * 4)};
-        cuuint32_t box[2] = {(cuuint32_t)(2 * bits), 128};
+        cuuint32_t box[2] = {(cuuint32_t)(wstage_rowb(bits) / 4), 128};
         cuuint32_t estr[2] = {1, 1};
-        CUtensorMapSwizzle sw = bits == 4 ? CU_TENSOR_MAP_SWIZZLE_32B
-                                : bits == 8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
+        CUtensorMapSwizzle sw = wstage_rowb(bits) == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
         CUresult r = encode(&prm.tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(pb.wq), dims, strides,
                             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -867,6 +972,9 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     prm.log2g = lg;
     prm.stages = stages;
     prm.kg = (int)kg;
+    prm.xres = xres;
+    prm.xslots = xslots;
+    prm.n_wstages = (int)((pb.K / KB + wstage_sub(bits) - 1) / wstage_sub(bits));
     prm.ydt = (int)pb.ydt;
     uint32_t cols = SA * 32 + nbufs(nt) * nt, pw = 32;
     while (pw < cols) pw <<= 1;
@@ -883,7 +991,7 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
         const int64_t tiles = (int64_t)prm.n_wtiles * prm.n_ttiles * prm.nbatch;
         grid = (int)(tiles < sms ? tiles : sms);
     }
-    const size_t smem = smem_for(nt, bits, stages, kg);
+    const size_t smem = smem_for(nt, bits, stages, pb.K, kg, xres, xslots);
     if (pb.xdt == DT::BF16) return launch_bits<bf16_t>(bits, nt, prm, grid, smem, stream);
     return launch_bits<f16_t>(bits, nt, prm, grid, smem, stream);
 }
@@ -891,10 +999,10 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
 #ifdef AQ_TRACE
 extern "C" __attribute__((visibility("default"))) int aq_trace_read(unsigned long long* out, int reset) {
     if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-    if (cudaMemcpyFromSymbol(out, g_trace, sizeof(unsigned long long) * 64) != cudaSuccess) return -1;
+    if (cudaMemcpyFromSymbol(out, ::aq_trace_ns, sizeof(unsigned long long) * 64) != cudaSuccess) return -1;
     if (reset) {
         unsigned long long z[64] = {0};
-        if (cudaMemcpyToSymbol(g_trace, z, sizeof z) != cudaSuccess) return -1;
+        if (cudaMemcpyToSymbol(::aq_trace_ns, z, sizeof z) != cudaSuccess) return -1;
     }
     return 0;
 }

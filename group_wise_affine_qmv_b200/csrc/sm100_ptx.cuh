@@ -1,12 +1,17 @@
 // sm100_ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA, tcgen05.
 //
-// Every wait here is bounded: it gives up after a wall-clock budget (read from
-// %globaltimer) or as soon as another warp of the CTA has raised the abort
-// flag, and reports failure instead of spinning forever.
+// Every wait here is bounded: it gives up after a budget of SM clock cycles or
+// as soon as another warp of the CTA has raised the abort flag, and reports
+// failure instead of spinning forever.
 #pragma once
 
 #include <cuda.h>
 #include <stdint.h>
+
+#ifdef AQ_TRACE
+__device__ unsigned long long aq_trace_ns[64];     // one translation unit includes this header
+__shared__ unsigned long long aq_trace_smem[64];   // per-CTA accumulation, flushed at exit
+#endif
 
 namespace aq {
 namespace ptx {
@@ -56,44 +61,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 #ifdef AQ_TRACE
 // Trace builds only: nanoseconds spent (lane 0 of each waiting warp) and number of
 // waits per wait site, accumulated over all CTAs; read back with aq_trace_read().
-extern __device__ unsigned long long g_trace[64];
-#define AQ_TRACE_ADD(site, ns)                                  \
-    do {                                                        \
-        if ((threadIdx.x & 31) == 0) {                          \
-            atomicAdd(&g_trace[(site)], (unsigned long long)(ns)); \
-            atomicAdd(&g_trace[32 + (site)], 1ull);             \
-        }                                                       \
+#define AQ_TRACE_ADD(site, ns)                                         \
+    do {                                                               \
+        if ((threadIdx.x & 31) == 0) {                                 \
+            atomicAdd(&::aq_trace_smem[(site)], (unsigned long long)(ns)); \
+            atomicAdd(&::aq_trace_smem[32 + (site)], 1ull);              \
+        }                                                              \
     } while (0)
 #endif
 
 // Wait for the phase of parity `parity` to complete.  Returns false if the
-// budget ran out or *abort became non-zero (another warp gave up).
+// budget ran out or *abort became non-zero (another warp gave up).  The budget is
+// counted in SM clock cycles (clock64, cheap to read; at most ~2 GHz, so
+// 2 cycles per nanosecond of budget never undercounts the wall time).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t budget_ns, int site = -1) {
     const uint32_t a = smem_u32(bar);
 #ifdef AQ_TRACE
     const uint64_t tt0 = globaltimer_ns();
+#endif
     bool done = mbar_try_wait(a, parity);
     if (!done) {
+        const long long c0 = clock64();
+        const long long limit = (long long)(budget_ns * 2ull);
         for (uint32_t i = 1;; ++i) {
             if (mbar_try_wait(a, parity)) { done = true; break; }
-            if ((i & 63u) == 0 && (*abort || globaltimer_ns() - tt0 > budget_ns)) break;
+            if ((i & 63u) == 0 && (*abort || clock64() - c0 > limit)) break;
         }
     }
+#ifdef AQ_TRACE
     if (site >= 0) AQ_TRACE_ADD(site, globaltimer_ns() - tt0);
-    return done;
 #else
     (void)site;
-    if (mbar_try_wait(a, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(a, parity)) return true;
-        if ((i & 63u) == 0) {
-            if (*abort) return false;
-            if (globaltimer_ns() - t0 > budget_ns) return false;
-        }
-    }
 #endif
+    return done;
 }
 
 // ---------------------------------------------------------------------------
