@@ -7,26 +7,32 @@
 // The tensor core computes D_g with the INTEGER codes as its A operand (exact
 // in bf16/f16) and x as B, one fresh fp32 accumulator per group; the epilogue
 // warps fold s and b in with fp32 FMAs.  X_g is summed from x widened to fp32
-// before any addition ("mlx PR #4516", load_vector fix).  Rounding w to
-// bf16 before the MMA would cost ~2e-3 of max|y| on its own, while the output
+// before any addition ("mlx PR #4516", load_vector fix).  Rounding w to bf16
+// before the MMA would cost ~2e-3 of max|y| on its own, while the output
 // rounding to bf16 already spends 2^-8 of the 4e-3 error budget, so the
 // weights are never rounded here.
 //
-// Roles ("weights-stationary": 128 rows of W are the MMA's M side, up to 128
-// tokens its N side):
-//   warp 0      TMA producer: per 64-code stage, the x tile [NT x 64] (128-byte
-//               swizzled, K-major UMMA B operand) and the packed W tile
-//               [128 rows x 64 codes], completing on one mbarrier.
-//   warp 1      MMA issuer: tcgen05.mma kind::f16, A (codes) from tensor
-//               memory, B from shared memory, D_g into one of two TMEM
-//               accumulators; tcgen05.commit releases stages, A slots and
-//               finished groups.
-//   warps 2..9  code expanders + epilogue: thread <-> W row (TMEM lane); two
-//               warps per lane quarter split each stage's 64 codes and, in the
-//               epilogue, the tile's tokens.  They expand packed codes into
-//               bf16/f16 integers with tcgen05.st, then for every finished
-//               group read D_g (tcgen05.ld) and update fp32 accumulators held
-//               in registers; at tile end they store y.
+// "Weights-stationary" tiles: 128 rows of W are the MMA's M side, up to 32
+// tokens its N side.  The pipeline advances one W stage at a time (128 rows x
+// WSC codes, WSC = 128 or 256 so that a stage row is a 64..128-byte TMA line)
+// and every hand-off between roles happens once per stage:
+//   warp 0      W producer: TMA of each W stage onto wfull[s] (ring of up to 12).
+//   warp 10     x producer: the CTA's token tile once (resident x), or per W
+//               stage its x block (SUB boxes of [NT x 64], 128-byte swizzle, the
+//               UMMA B operand) onto a ring of up to 4 x stages.
+//   warp 1      MMA issuer (warp-wide loop, one lane issues): waits for the
+//               expanded codes of the stage (afull) and for its accumulators to
+//               be free (dfree), then issues SUB*4 tcgen05.mma kind::f16 with A
+//               from tensor memory, one fresh accumulator per group, and one
+//               tcgen05.commit (sdone[w % 2]; a second one frees a streamed x stage).
+//   warps 2..9  code expanders + epilogue: thread <-> W row (TMEM lane), two
+//               warps per lane quarter split each 64 codes.  Per stage they
+//               expand the packed codes into bf16/f16 integers (tcgen05.st into
+//               A block w % 2), release the shared-memory stage (wfree), then
+//               fold the previous stage's groups into fp32 registers
+//               (tcgen05.ld of D, + s*D + b*X) and release its accumulators.
+// Tensor memory: [A block 0 | A block 1 | D: 2 x GPS group accumulators of NT
+// columns]; with GPS = WSC / group <= 4 this fits 512 columns.
 //
 // Rows of the last W tile that fall past N read TMA zero fill and the clamped
 // last row's scale/bias and are simply not stored: no per-row check inside the
@@ -52,36 +58,22 @@ __device__ int g_device_error = 0;
 
 namespace {
 
-constexpr int MMA_THREADS = 320;          // 10 warps
+constexpr int MMA_THREADS = 352;          // 11 warps
 constexpr int DQ_THREADS = 256;           // warps 2..9
 constexpr int KB = 64;                    // codes per MMA sub-step (4 tcgen05.mma of K = 16)
-constexpr int SA = 4;                     // A slots in tensor memory, 32 columns each
 constexpr int SCW = 32;                   // groups per scale/bias chunk
 constexpr int SCP = SCW + 2;              // padded row pitch (halves) of a chunk in shared memory
-constexpr int MAX_STAGES = 16;
-constexpr int MAX_XSLOTS = 16;
+constexpr int MAX_STAGES = 12;
+constexpr int MAX_XST = 4;                // streamed x stages
 constexpr int MAX_EXPERTS = 1024;
-constexpr int XTAB_MAX_BYTES = 48 * 1024; // sum-of-x table per token tile
-constexpr int NBMAX = 4;                  // group accumulators in tensor memory
-
-// One pipeline stage of W is 128 rows x ROWB bytes: a full 128-byte swizzle atom per row for
-// 2/4/8-bit codes (so each TMA request moves a 128-byte line), 96 bytes for 6-bit.  A stage
-// holds SUB sub-steps of 64 codes.
-template <int BITS> struct WStage {
-    static constexpr int ROWB = BITS == 6 ? 96 : 128;
-    static constexpr int CODES = ROWB * 8 / BITS;
-    static constexpr int SUB = CODES / KB;
-    static constexpr int BYTES = 128 * ROWB;
-};
-
-// group accumulators for a token-tile width: 4 while they fit beside the A slots
-__host__ __device__ constexpr int nbufs(int nt) { return nt <= 64 ? 4 : 2; }
+constexpr int XTAB_MAX_BYTES = 32 * 1024; // sum-of-x table per token tile
+constexpr int NT_MAX = 32;                // tokens per tile
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait
 constexpr int ERR_TIMEOUT = 1;
 
 struct MmaParams {
     CUtensorMap tx;  // x: 4D {K, rows, nb1, nb0} u16, box {64, NT, 1, 1}, 128B swizzle
-    CUtensorMap tw;  // W: 2D {K*bits/32, rows} u32, box {2*bits, 128}
+    CUtensorMap tw;  // W: 2D {K*bits/32, rows} u32, box {rowb/4, 128}
     const void* x;
     void* y;
     const uint16_t* scales;
@@ -92,12 +84,18 @@ struct MmaParams {
     int64_t nb1;
     int n_wtiles, n_ttiles, nbatch;
     int group, log2g;
-    int stages;
     int kg;              // groups per row = K / group
-    int xres;            // 1: the CTA's single x tile stays resident in shared memory
-    int xslots;          // streaming x: ring slots of [NT x 64] (one per MMA sub-step)
-    int n_wstages;       // W pipeline stages per tile
     int ydt;             // DT of y
+    int wsc;             // codes per W stage (128 or 256)
+    int rowb;            // bytes per W row per stage
+    int sub;             // 64-code MMA sub-steps per stage
+    int gps;             // groups per stage
+    uint32_t swz;        // swizzle mask of the W stage (see swz_addr)
+    int n_wstages;       // W stages per tile
+    int stages;          // W ring depth
+    int cs_w;            // W stages per scale/bias chunk
+    int xres;            // 1: the CTA's single x tile stays resident in shared memory
+    int xst;             // streamed x ring depth (x stages of SUB boxes) when not resident
     uint32_t tmem_cols;
     uint32_t idesc;
     const int64_t* offsets;  // grouped mode when non-null
@@ -116,59 +114,58 @@ struct TileInfo {
 };
 
 struct Smem {
-    uint64_t* full;
-    uint64_t* empty;
-    uint64_t* afull;
-    uint64_t* aempty;
-    uint64_t* gfull;     // [NBMAX] group accumulator ready (MMA commit)
-    uint64_t* gempty;    // [NBMAX] group accumulator consumed (8 epilogue warps)
-    uint64_t* sbar;      // [2] scale/bias chunk slots: 256 dequant-thread arrivals
-    uint64_t* xbar;      // sum-of-x table barrier: 256 arrivals
-    uint64_t* mdone;     // all MMAs of this CTA retired (teardown)
-    uint64_t* xfull;     // resident x tile landed
-    uint64_t* xsfull;    // [MAX_XSLOTS] streaming x slot landed (TMA)
-    uint64_t* xsempty;   // [MAX_XSLOTS] streaming x slot consumed (MMA commit)
+    uint64_t* wfull;     // [MAX_STAGES] W stage landed (TMA)
+    uint64_t* wfree;     // [MAX_STAGES] W stage read by the 8 expander warps
+    uint64_t* xfull;     // [MAX_XST] streamed x stage landed (TMA)
+    uint64_t* xfree;     // [MAX_XST] streamed x stage read by its MMAs (commit)
+    uint64_t* afull;     // [2] A block written (8 expander warps)
+    uint64_t* sdone;     // [2] MMAs of a W stage complete (commit)
+    uint64_t* dfree;     // [2] group accumulators of a W stage read (8 epilogue warps)
+    uint64_t* sbar;      // [2] scale/bias chunk slots: 256 arrivals
+    uint64_t* xbar;      // sum-of-x table: 256 arrivals
+    uint64_t* xres_full; // resident x landed
+    uint64_t* mdone;     // teardown: all MMAs retired
     uint32_t* tmem_base;
     int* abort;
     int* prefix;         // grouped: tile prefix sums [n_experts + 1]
     float* xtab;         // [kg][NT] sums of x per group and token
-    uint8_t* xs;         // resident: [K/64][NT][128 B]; streaming: xslots x [NT][128 B]
-    uint8_t* ws;         // stages x [128 rows][ROWB]
+    uint8_t* xs;         // resident: [K/64][NT][128 B]; streamed: [xst][SUB][NT][128 B]
+    uint8_t* ws;         // [stages][128 rows][rowb]
     uint16_t* sb;        // [2 slots][2 arrays][128][SCP]
 };
 
-template <int BITS, int NT>
+template <int NT>
 __device__ __forceinline__ Smem carve(uint8_t* base, const MmaParams& p) {
     Smem s;
     uint8_t* q = base;
     s.xs = q;
-    q += p.xres ? (size_t)(p.K / KB) * NT * 128 : (size_t)p.xslots * NT * 128;
+    q += p.xres ? (size_t)(p.K / KB) * NT * 128 : (size_t)p.xst * p.sub * NT * 128;
     s.ws = q;
-    q += (size_t)p.stages * WStage<BITS>::BYTES;
+    q += (size_t)p.stages * 128 * p.rowb;
+    q = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(q) + 1023) & ~uintptr_t(1023));
     s.xtab = reinterpret_cast<float*>(q);
     q += (size_t)p.kg * NT * 4;
     s.sb = reinterpret_cast<uint16_t*>(q);
     q += 2 * 2 * 128 * SCP * 2;
-    s.full = reinterpret_cast<uint64_t*>(q);
-    s.empty = s.full + MAX_STAGES;
-    s.afull = s.empty + MAX_STAGES;
-    s.aempty = s.afull + SA;
-    s.gfull = s.aempty + SA;
-    s.gempty = s.gfull + NBMAX;
-    s.sbar = s.gempty + NBMAX;
+    s.wfull = reinterpret_cast<uint64_t*>(q);
+    s.wfree = s.wfull + MAX_STAGES;
+    s.xfull = s.wfree + MAX_STAGES;
+    s.xfree = s.xfull + MAX_XST;
+    s.afull = s.xfree + MAX_XST;
+    s.sdone = s.afull + 2;
+    s.dfree = s.sdone + 2;
+    s.sbar = s.dfree + 2;
     s.xbar = s.sbar + 2;
-    s.mdone = s.xbar + 1;
-    s.xfull = s.mdone + 1;
-    s.xsfull = s.xfull + 1;
-    s.xsempty = s.xsfull + MAX_XSLOTS;
-    s.tmem_base = reinterpret_cast<uint32_t*>(s.xsempty + MAX_XSLOTS);
+    s.xres_full = s.xbar + 1;
+    s.mdone = s.xres_full + 1;
+    s.tmem_base = reinterpret_cast<uint32_t*>(s.mdone + 1);
     s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
     s.prefix = s.abort + 1;
     return s;
 }
 
 __host__ __device__ constexpr size_t smem_fixed_bytes() {
-    return 2 * 2 * 128 * SCP * 2 + (2 * MAX_STAGES + 2 * MAX_XSLOTS + 2 * SA + 2 * NBMAX + 6) * 8 + 8 + (MAX_EXPERTS + 1) * 4 + 1024 /*align*/;
+    return 2 * 2 * 128 * SCP * 2 + (2 * MAX_STAGES + 2 * MAX_XST + 2 * 4 + 3) * 8 + 8 + (MAX_EXPERTS + 1) * 4 + 2 * 1024 /*align*/;
 }
 
 __device__ __forceinline__ void raise_abort(int* abort) {
@@ -221,29 +218,31 @@ __device__ __forceinline__ TileInfo tile_info(const MmaParams& p, const Smem& s,
 // in the 16-bit MMA type (low half = even code)
 // ---------------------------------------------------------------------------
 
-// This thread's 32 codes (sub-step j, half h) of W row `row` in a stage.  Rows are ROWB bytes
-// apart; with a 128-byte swizzle, 16-byte chunk c of row r sits at chunk c ^ (r & 7).
+// This thread's 32 codes (sub-step j, half h) of W row `row` in a stage whose rows are
+// `rowb` bytes apart.  TMA wrote the stage with a swizzle that XORs byte-address bits
+// [4..6] with bits [7..9] under `swz` (7: 128-byte, 3: 64-byte, 1: 32-byte, 0: none);
+// the stage base is 1024-byte aligned, so stage-relative addresses swizzle the same way.
+__device__ __forceinline__ uint32_t swz_addr(uint32_t a, uint32_t swz) { return a ^ (((a >> 7) & swz) << 4); }
+
 template <int BITS>
-__device__ __forceinline__ void load_w32(const uint8_t* stage, int row, int j, int h, uint32_t* w) {
-    constexpr int ROWB = WStage<BITS>::ROWB;
-    const uint32_t b = (uint32_t)(j * KB + 32 * h) * BITS / 8;  // byte offset within the row
-    const uint8_t* r = stage + (uint32_t)row * ROWB;
-    const uint32_t sw = ROWB == 128 ? ((uint32_t)(row & 7) << 4) : 0u;
+__device__ __forceinline__ void load_w32(const uint8_t* stage, int rowb, uint32_t swz, int row, int j, int h,
+                                         uint32_t* w) {
+    const uint32_t a = (uint32_t)row * rowb + (uint32_t)(j * KB + 32 * h) * BITS / 8;
     if constexpr (BITS == 4) {
-        const uint4 v = *reinterpret_cast<const uint4*>(r + (b ^ sw));
+        const uint4 v = *reinterpret_cast<const uint4*>(stage + swz_addr(a, swz));
         w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
     } else if constexpr (BITS == 8) {
-        const uint4 v0 = *reinterpret_cast<const uint4*>(r + (b ^ sw));
-        const uint4 v1 = *reinterpret_cast<const uint4*>(r + ((b + 16) ^ sw));
+        const uint4 v0 = *reinterpret_cast<const uint4*>(stage + swz_addr(a, swz));
+        const uint4 v1 = *reinterpret_cast<const uint4*>(stage + swz_addr(a + 16, swz));
         w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
         w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
     } else if constexpr (BITS == 2) {
-        const uint2 v = *reinterpret_cast<const uint2*>(r + (((b & ~15u) ^ sw) | (b & 15u)));
+        const uint2 v = *reinterpret_cast<const uint2*>(stage + swz_addr(a, swz));
         w[0] = v.x; w[1] = v.y;
     } else {
 #pragma unroll
         for (int i = 0; i < BITS / 2; ++i) {
-            const uint2 v = *reinterpret_cast<const uint2*>(r + b + 8 * i);
+            const uint2 v = *reinterpret_cast<const uint2*>(stage + swz_addr(a + 8 * i, swz));
             w[2 * i] = v.x; w[2 * i + 1] = v.y;
         }
     }
@@ -372,53 +371,41 @@ __device__ __forceinline__ void store_y(void* y, int64_t off, float v, int ydt, 
 template <int BITS, typename XT, int NT>
 __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_constant__ MmaParams p) {
     constexpr int H = NT / 2;            // tokens per epilogue thread
-    constexpr int NB = nbufs(NT);        // group accumulators
-    constexpr int SUB = WStage<BITS>::SUB;
-    const int NWS = p.n_wstages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const Smem s = carve<BITS, NT>(base, p);
+    const Smem s = carve<NT>(base, p);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = p.stages;
     const int KBLK = (int)(p.K / KB);
     const int G = p.group;
     const int NG = p.kg;
-    const int CS = (SCW << p.log2g) / KB;   // stages per scale/bias chunk
-    const int NCH = (NG + SCW - 1) / SCW;   // chunks per tile
-    // Epilogue lag in stages: group g is folded in once the expanders are LAG stages past
-    // its end, so the MMA of the stages in between overlaps code expansion.  The MMA of a
-    // stage reuses the accumulator of the group NB groups earlier, which must be folded by
-    // then: NB >= LAG * groups-per-stage.
-    const int gps = G < KB ? KB / G : 1;
-    int LAG = NB / gps;
-    if (LAG > 3) LAG = 3;
-    if (LAG < 1) LAG = 1;
+    const int NWS = p.n_wstages;
+    const int SUB = p.sub;
+    const int GPS = p.gps;
+    const int ACOLS = p.wsc / 2;            // tensor-memory columns of one A block
+    const int NCH = (NG + SCW - 1) / SCW;   // scale/bias chunks per tile
 
 #ifdef AQ_TRACE
     if (threadIdx.x < 64) ::aq_trace_smem[threadIdx.x] = 0;
 #endif
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
-            ptx::mbar_init(&s.full[i], 1);
-            ptx::mbar_init(&s.empty[i], 1);
+            ptx::mbar_init(&s.wfull[i], 1);
+            ptx::mbar_init(&s.wfree[i], 8);
         }
-        for (int i = 0; i < SA; ++i) {
+        for (int i = 0; i < MAX_XST; ++i) {
+            ptx::mbar_init(&s.xfull[i], 1);
+            ptx::mbar_init(&s.xfree[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&s.afull[i], 8);
-            ptx::mbar_init(&s.aempty[i], 1);
+            ptx::mbar_init(&s.sdone[i], 1);
+            ptx::mbar_init(&s.dfree[i], 8);
+            ptx::mbar_init(&s.sbar[i], DQ_THREADS);
         }
-        for (int i = 0; i < NBMAX; ++i) {
-            ptx::mbar_init(&s.gfull[i], 1);
-            ptx::mbar_init(&s.gempty[i], 8);
-        }
-        ptx::mbar_init(&s.sbar[0], DQ_THREADS);
-        ptx::mbar_init(&s.sbar[1], DQ_THREADS);
         ptx::mbar_init(s.xbar, DQ_THREADS);
+        ptx::mbar_init(s.xres_full, 1);
         ptx::mbar_init(s.mdone, 1);
-        ptx::mbar_init(s.xfull, 1);
-        for (int i = 0; i < p.xslots; ++i) {
-            ptx::mbar_init(&s.xsfull[i], 1);
-            ptx::mbar_init(&s.xsempty[i], 1);
-        }
         *s.abort = 0;
         ptx::fence_mbar_init();
     }
@@ -455,125 +442,134 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tbase = *s.tmem_base;
-    const uint32_t d_tmem = tbase + SA * 32;  // NB group accumulators of NT columns follow the A slots
+    const uint32_t d_tmem = tbase + (uint32_t)p.wsc;  // 2 x GPS group accumulators follow the two A blocks
     const int ntiles = total_tiles(p, s);
+    const bool has_tiles = (int)blockIdx.x < ntiles;
 
     if (warp == 0) {
-        // ======================= TMA producer =======================
-        if (lane == 0) {
-            const uint32_t bytes = WStage<BITS>::BYTES;
-            const int SX = p.xslots;
-            uint32_t wit = 0, xit = 0;
-            bool ok = true;
-            if (p.xres && (int)blockIdx.x < ntiles) {
+        // ======================= W producer =======================
+        // Warp-wide loop (uniform coordinates and barrier phases); one lane issues the copies.
+        const bool leader = lane == 0;
+        const uint32_t wbytes = 128u * (uint32_t)p.rowb;
+        uint32_t wg = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const TileInfo ti = tile_info<NT>(p, s, t);
+            for (int w = 0; w < NWS; ++w) {
+                const int st = wg % S;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfree[st], ((wg / S) & 1) ^ 1, s.abort, WAIT_NS, 0));
+                if (!ok) break;
+                if (leader) {
+                    // columns past K (a partial last stage) read as zero fill
+                    ptx::mbar_arrive_expect_tx(&s.wfull[st], wbytes);
+                    ptx::tma_load_2d(s.ws + (size_t)st * 128 * p.rowb, &p.tw, &s.wfull[st], w * (p.rowb / 4),
+                                     (int32_t)ti.wrow0);
+                }
+                ++wg;
+            }
+        }
+        if (leader && !ok) {
+            raise_abort(s.abort);
+            // drain: the copies of every issued stage must land before the CTA exits
+            volatile int never = 0;
+            for (uint32_t j = wg >= (uint32_t)S ? wg - S : 0; j < wg; ++j)
+                ptx::mbar_wait(&s.wfull[j % S], (j / S) & 1, &never, 200000000ull);
+        }
+        __syncwarp();
+    } else if (warp == 10) {
+        // ======================= x producer =======================
+        const bool leader = lane == 0;
+        bool ok = true;
+        uint32_t wg = 0;
+        if (p.xres) {
+            if (has_tiles && leader) {
                 // the CTA's only token tile: all of K, once
                 const TileInfo t0 = tile_info<NT>(p, s, blockIdx.x);
-                ptx::mbar_arrive_expect_tx(s.xfull, (uint32_t)KBLK * NT * 128);
+                ptx::mbar_arrive_expect_tx(s.xres_full, (uint32_t)KBLK * NT * 128);
                 for (int kb = 0; kb < KBLK; ++kb)
-                    ptx::tma_load_4d(s.xs + (size_t)kb * NT * 128, &p.tx, s.xfull, kb * KB, (int32_t)t0.xrow0, t0.b1,
-                                     t0.b0);
+                    ptx::tma_load_4d(s.xs + (size_t)kb * NT * 128, &p.tx, s.xres_full, kb * KB, (int32_t)t0.xrow0,
+                                     t0.b1, t0.b0);
+                volatile int never = 0;
+                ptx::mbar_wait(s.xres_full, 0, &never, 200000000ull);
             }
+        } else {
+            const int XS = p.xst;
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 const TileInfo ti = tile_info<NT>(p, s, t);
-                for (int w = 0; w < NWS; ++w, ++wit) {
-                    const int st = wit % S;
-                    const uint32_t ph = (wit / S) & 1;
-                    if (!ptx::mbar_wait(&s.empty[st], ph ^ 1, s.abort, WAIT_NS, 0)) { ok = false; break; }
-                    ptx::mbar_arrive_expect_tx(&s.full[st], bytes);
-                    ptx::tma_load_2d(s.ws + (size_t)st * WStage<BITS>::BYTES, &p.tw, &s.full[st],
-                                     w * (WStage<BITS>::ROWB / 4), (int32_t)ti.wrow0);
-                    if (!p.xres) {
-                        for (int j = 0; j < SUB && ok; ++j, ++xit) {
-                            const int kb = w * SUB + j;
-                            if (kb >= KBLK) break;
-                            const int xsl = xit % SX;
-                            if (!ptx::mbar_wait(&s.xsempty[xsl], ((xit / SX) & 1) ^ 1, s.abort, WAIT_NS, 0)) {
-                                ok = false;
-                                break;
-                            }
-                            ptx::mbar_arrive_expect_tx(&s.xsfull[xsl], (uint32_t)NT * 128);
-                            ptx::tma_load_4d(s.xs + (size_t)xsl * NT * 128, &p.tx, &s.xsfull[xsl], kb * KB,
-                                             (int32_t)ti.xrow0, ti.b1, ti.b0);
-                        }
+                for (int w = 0; w < NWS; ++w) {
+                    const int xs = wg % XS;
+                    ok = __all_sync(0xffffffffu,
+                                    ptx::mbar_wait(&s.xfree[xs], ((wg / XS) & 1) ^ 1, s.abort, WAIT_NS, 9));
+                    if (!ok) break;
+                    if (leader) {
+                        const int nsub = min(SUB, KBLK - w * SUB);
+                        ptx::mbar_arrive_expect_tx(&s.xfull[xs], (uint32_t)nsub * NT * 128);
+                        for (int j = 0; j < nsub; ++j)
+                            ptx::tma_load_4d(s.xs + ((size_t)xs * SUB + j) * NT * 128, &p.tx, &s.xfull[xs],
+                                             (w * SUB + j) * KB, (int32_t)ti.xrow0, ti.b1, ti.b0);
                     }
+                    ++wg;
                 }
             }
-            if (!ok) {
+            if (leader && !ok) {
                 raise_abort(s.abort);
-                // drain: the copies of every issued stage must land before the CTA exits
                 volatile int never = 0;
-                const uint32_t first = wit >= (uint32_t)S ? wit - S : 0;
-                for (uint32_t jj = first; jj < wit; ++jj)
-                    ptx::mbar_wait(&s.full[jj % S], (jj / S) & 1, &never, 200000000ull);
-                const uint32_t xfirst = xit >= (uint32_t)SX ? xit - SX : 0;
-                for (uint32_t jj = xfirst; jj < xit; ++jj)
-                    ptx::mbar_wait(&s.xsfull[jj % SX], (jj / SX) & 1, &never, 200000000ull);
-            }
-            if (p.xres && (int)blockIdx.x < ntiles) {
-                volatile int never = 0;
-                ptx::mbar_wait(s.xfull, 0, &never, 200000000ull);
+                for (uint32_t j = wg >= (uint32_t)XS ? wg - XS : 0; j < wg; ++j)
+                    ptx::mbar_wait(&s.xfull[j % XS], (j / XS) & 1, &never, 200000000ull);
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         // ======================= MMA issuer =======================
-        if (lane == 0) {
-            uint32_t it = 0, gc = 0, wit = 0, xit = 0;
-            const int SX = p.xslots;
-            bool ok = true;
-            if (p.xres && (int)blockIdx.x < ntiles)
-                ok = ptx::mbar_wait(s.xfull, 0, s.abort, WAIT_NS, 1);
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                for (int w = 0; w < NWS && ok; ++w, ++wit) {
-                    const int st = wit % S;
-                    const uint32_t ph = (wit / S) & 1;
-                    (void)ph;
-                    for (int j = 0; j < SUB && ok; ++j) {
-                        const int kb = w * SUB + j;
-                        if (kb >= KBLK) break;
-                        const int a = it % SA;
-                        const uint32_t aph = (it / SA) & 1;
-                        const int xsl = xit % SX;
-                        if (!p.xres && !ptx::mbar_wait(&s.xsfull[xsl], (xit / SX) & 1, s.abort, WAIT_NS, 1)) {
-                            ok = false;
-                            break;
-                        }
-                        if (!ptx::mbar_wait(&s.afull[a], aph, s.abort, WAIT_NS, 2)) { ok = false; break; }
-                        ptx::tc_fence_after();
-                        const uint32_t xaddr =
-                            ptx::smem_u32(p.xres ? s.xs + (size_t)kb * NT * 128 : s.xs + (size_t)xsl * NT * 128);
+        // Warp-wide loop so barrier phases, tensor-memory addresses and descriptors stay
+        // warp-uniform; one lane issues the tcgen05 operations.
+        const bool leader = lane == 0;
+        uint32_t wg = 0;
+        bool ok = true;
+        if (p.xres && has_tiles) ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xres_full, 0, s.abort, WAIT_NS, 1));
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            for (int w = 0; w < NWS; ++w, ++wg) {
+                const int slot = wg & 1;
+                const uint32_t ph = (wg >> 1) & 1;
+                const int xs = p.xres ? 0 : (int)(wg % (uint32_t)p.xst);
+                if (!p.xres) {
+                    ok = __all_sync(0xffffffffu,
+                                    ptx::mbar_wait(&s.xfull[xs], (wg / p.xst) & 1, s.abort, WAIT_NS, 1));
+                    if (!ok) break;
+                }
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.afull[slot], ph, s.abort, WAIT_NS, 2));
+                if (!ok) break;
+                // the epilogue has read this slot's accumulators (stage wg - 2)
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.dfree[slot], ph ^ 1, s.abort, WAIT_NS, 3));
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t a_blk = tbase + (uint32_t)(slot * ACOLS);
+                const uint32_t d_blk = d_tmem + (uint32_t)(slot * GPS * NT);
+                for (int j = 0; j < SUB; ++j) {
+                    const int kb = w * SUB + j;
+                    if (kb >= KBLK) break;
+                    const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(
+                        p.xres ? s.xs + (size_t)kb * NT * 128 : s.xs + ((size_t)xs * SUB + j) * NT * 128));
 #pragma unroll
-                        for (int kk = 0; kk < KB / 16; ++kk) {
-                            const int k = kb * KB + 16 * kk;
-                            const bool gstart = (k & (G - 1)) == 0;
-                            const uint32_t buf = gc % NB;
-                            if (gstart) {
-                                // this accumulator's previous group must have been read by the epilogue
-                                if (!ptx::mbar_wait(&s.gempty[buf], ((gc / NB) & 1) ^ 1, s.abort, WAIT_NS, 3)) {
-                                    ok = false;
-                                    break;
-                                }
-                                ptx::tc_fence_after();
-                            }
-                            const uint64_t bdesc = ptx::smem_desc_sw128(xaddr + 32 * kk);
-                            ptx::mma_ts(d_tmem + buf * NT, tbase + a * 32 + kk * 8, bdesc, p.idesc, gstart ? 0u : 1u);
-                            if (((k + 16) & (G - 1)) == 0) {
-                                ptx::mma_commit(&s.gfull[buf]);
-                                ++gc;
-                            }
-                        }
-                        ptx::mma_commit(&s.aempty[a]);
-                        if (!p.xres) {
-                            ptx::mma_commit(&s.xsempty[xsl]);
-                            ++xit;
-                        }
-                        ++it;
+                    for (int kk = 0; kk < KB / 16; ++kk) {
+                        const int ks = j * KB + 16 * kk;            // code offset within the stage
+                        const uint32_t lg = (uint32_t)(ks >> p.log2g);  // group within the stage
+                        const bool gstart = (ks & (G - 1)) == 0;
+                        // descriptor start address advances 32 bytes (2 units of 16 B) per K = 16 step
+                        if (leader)
+                            ptx::mma_ts(d_blk + lg * NT, a_blk + (uint32_t)(j * 32 + kk * 8), bdesc + (uint64_t)(2 * kk),
+                                        p.idesc, gstart ? 0u : 1u);
                     }
-                    ptx::mma_commit(&s.empty[st]);
+                }
+                if (leader) {
+                    ptx::mma_commit(&s.sdone[slot]);
+                    if (!p.xres) ptx::mma_commit(&s.xfree[xs]);
                 }
             }
-            if (!ok) raise_abort(s.abort);
-            // every MMA this thread issued must retire before tensor memory is freed
+        }
+        if (!ok && leader) raise_abort(s.abort);
+        // every MMA this warp issued must retire before tensor memory is freed
+        if (leader) {
             ptx::mma_commit(s.mdone);
             volatile int never = 0;
             ptx::mbar_wait(s.mdone, 0, &never, 200000000ull);
@@ -582,56 +578,69 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
     } else {
         // ======================= code expanders + epilogue =======================
         const int q = warp & 3;                 // TMEM lane quarter
-        const int h = (warp - 2) >> 2;          // which 32 codes of each stage / which half of the tokens
+        const int h = (warp - 2) >> 2;          // which 32 codes of each 64 / which half of the tokens
         const int row = 32 * q + lane;          // W row within the tile == TMEM lane
         const int tid = threadIdx.x - 64;       // 0..255
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        uint32_t it = 0, ge = 0, xph = 0, wit = 0;
+        uint32_t wg = 0, xph = 0;
         int unit = 0;
         bool ok = true;
         int64_t cur_x0 = -1;
         int cur_b = -1, cur_tv = -1;
         float2 acc[H / 2];
 
-        if (blockIdx.x < ntiles) {
+        if (has_tiles) {
             const TileInfo t0 = tile_info<NT>(p, s, blockIdx.x);
             issue_sb_chunk(p, t0, 0, s.sb, tid);
         }
         ptx::cp_async_commit();
-
-        const uint16_t* slot = s.sb;
+        const uint16_t* sbslot = s.sb;
         int g_chunk0 = 0;
 
-        // epilogue of group g of the current tile: acc += s*D_g + b*X_g
-        auto epilogue_group = [&](int g) -> bool {
-            const uint32_t buf = ge % NB;
-            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&s.gfull[buf], (ge / NB) & 1, s.abort, WAIT_NS, 6)))
+        // fold the groups of W stage `wl` (global stage counter wgE) of tile `ti` into acc
+        auto epilogue_stage = [&](uint32_t wgE, int wl, const TileInfo& ti, int t) -> bool {
+            if (wl % p.cs_w == 0) {
+                // this stage opens a scale/bias chunk: its copies were issued a chunk earlier
+                ptx::cp_async_wait_all();
+                ptx::mbar_arrive(&s.sbar[unit & 1]);
+                if (!__all_sync(0xffffffffu,
+                                ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS, 7)))
+                    return false;
+                sbslot = s.sb + (unit & 1) * 2 * 128 * SCP;
+                const int c = wl / p.cs_w;
+                g_chunk0 = c * SCW;
+                uint16_t* nslot = s.sb + ((unit + 1) & 1) * 2 * 128 * SCP;
+                if (c + 1 < NCH) {
+                    issue_sb_chunk(p, ti, c + 1, nslot, tid);
+                } else if (t + (int)gridDim.x < ntiles) {
+                    const TileInfo tn = tile_info<NT>(p, s, t + gridDim.x);
+                    issue_sb_chunk(p, tn, 0, nslot, tid);
+                }
+                ptx::cp_async_commit();
+                ++unit;
+            }
+            const int slot = wgE & 1;
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&s.sdone[slot], (wgE >> 1) & 1, s.abort, WAIT_NS, 6)))
                 return false;
             ptx::tc_fence_after();
-            const int gl = g - g_chunk0;
-            const float sv = half_bits_to_float(slot[row * SCP + gl], XT{});
-            const float bv = half_bits_to_float(slot[128 * SCP + row * SCP + gl], XT{});
-            const float2 s2 = make_float2(sv, sv), b2 = make_float2(bv, bv);
-            const float* xg = s.xtab + g * NT + h * H;
-#pragma unroll
-            for (int c0 = 0; c0 < H; c0 += 16) {
+            for (int lg = 0; lg < GPS; ++lg) {
+                const int g = wl * GPS + lg;
+                if (g >= NG) break;
+                const int gl = g - g_chunk0;
+                const float sv = half_bits_to_float(sbslot[row * SCP + gl], XT{});
+                const float bv = half_bits_to_float(sbslot[128 * SCP + row * SCP + gl], XT{});
+                const float2 s2 = make_float2(sv, sv), b2 = make_float2(bv, bv);
+                const float* xg = s.xtab + g * NT + h * H;
+                const uint32_t dcol = d_tmem + (uint32_t)((slot * GPS + lg) * NT + h * H);
                 uint32_t v[16];
-                if constexpr (H >= 16) {
-                    ptx::tmem_ld16(d_tmem + buf * NT + lane_base + h * H + c0, v);
-                } else {
-                    ptx::tmem_ld8(d_tmem + buf * NT + lane_base + h * H + c0, v);
-                }
-#ifdef AQ_TRACE
-                { const uint64_t w0 = ptx::globaltimer_ns(); ptx::tc_wait_ld(); AQ_TRACE_ADD(10, ptx::globaltimer_ns() - w0); }
-#else
+                if constexpr (H >= 16) ptx::tmem_ld16(dcol + lane_base, v);
+                else ptx::tmem_ld8(dcol + lane_base, v);
                 ptx::tc_wait_ld();
-#endif
-                constexpr int CNT = H >= 16 ? 16 : H;
 #pragma unroll
-                for (int c = 0; c < CNT; c += 4) {
-                    const float4 xv = *reinterpret_cast<const float4*>(xg + c0 + c);
-                    float2& a0 = acc[(c0 + c) / 2];
-                    float2& a1 = acc[(c0 + c) / 2 + 1];
+                for (int c = 0; c < H; c += 4) {
+                    const float4 xv = *reinterpret_cast<const float4*>(xg + c);
+                    float2& a0 = acc[c / 2];
+                    float2& a1 = acc[c / 2 + 1];
                     a0 = ptx::ffma2(b2, make_float2(xv.x, xv.y), a0);
                     a1 = ptx::ffma2(b2, make_float2(xv.z, xv.w), a1);
                     a0 = ptx::ffma2(s2, make_float2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), a0);
@@ -640,8 +649,7 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
             }
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&s.gempty[buf]);
-            ++ge;
+            if (lane == 0) ptx::mbar_arrive(&s.dfree[slot]);
             return true;
         };
 
@@ -650,14 +658,13 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
             // ---- sums of x for this token tile (rebuilt only when the tokens change) ----
             const int bkey = ti.b0 * 65536 + ti.b1;
             if (ti.xrow0 != cur_x0 || bkey != cur_b || ti.tvalid != cur_tv) {
-                // everyone is done reading the previous table
-                ptx::mbar_arrive(s.xbar);
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_NS));
+                ptx::mbar_arrive(s.xbar);  // everyone is done reading the previous table
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_NS, 8));
                 ++xph;
                 if (!ok) break;
                 build_xtab<XT, NT>(p, ti, s.xtab, tid);
                 ptx::mbar_arrive(s.xbar);
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_NS));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_NS, 8));
                 ++xph;
                 if (!ok) break;
                 cur_x0 = ti.xrow0;
@@ -666,69 +673,37 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) qmm_tc_kernel(const __grid_con
             }
 #pragma unroll
             for (int i = 0; i < H / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
-            int g_next = 0;  // next group of this tile awaiting its epilogue
-            for (int w = 0; w < NWS && ok; ++w, ++wit) {
-                const int st = wit % S;
-                const uint32_t ph = (wit / S) & 1;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.full[st], ph, s.abort, WAIT_NS, 4));
+            for (int w = 0; w < NWS && ok; ++w, ++wg) {
+                const int st = wg % S;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfull[st], (wg / S) & 1, s.abort, WAIT_NS, 4));
                 if (!ok) break;
-                const uint8_t* wstage = s.ws + (size_t)st * WStage<BITS>::BYTES;
-                for (int j = 0; j < SUB; ++j, ++it) {
-                    const int kb = w * SUB + j;
-                    if (kb >= KBLK) break;
-                    // (1) epilogues of the groups that ended LAG sub-steps before this one; entering a
-                    //     new scale/bias chunk, every group of the previous chunk (its slot is reused)
-                    const int fold_end = (kb % CS == 0) ? kb * KB : (kb - LAG + 1) * KB;
-                    while (g_next < NG && (g_next + 1) * G <= fold_end) {
-                        if (!epilogue_group(g_next)) { ok = false; break; }
-                        ++g_next;
-                    }
-                    if (!ok) break;
-                    // (2) next scale/bias chunk
-                    if (kb % CS == 0) {
-                        ptx::cp_async_wait_all();
-                        ptx::mbar_arrive(&s.sbar[unit & 1]);
-                        ok = __all_sync(0xffffffffu,
-                                        ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS, 7));
-                        if (!ok) break;
-                        slot = s.sb + (unit & 1) * 2 * 128 * SCP;
-                        const int c = kb / CS;
-                        g_chunk0 = c * SCW;
-                        uint16_t* nslot = s.sb + ((unit + 1) & 1) * 2 * 128 * SCP;
-                        if (c + 1 < NCH) {
-                            issue_sb_chunk(p, ti, c + 1, nslot, tid);
-                        } else if (t + (int)gridDim.x < ntiles) {
-                            const TileInfo tn = tile_info<NT>(p, s, t + gridDim.x);
-                            issue_sb_chunk(p, tn, 0, nslot, tid);
-                        }
-                        ptx::cp_async_commit();
-                        ++unit;
-                    }
-                    // (3) expand this sub-step's codes into an A slot
-                    const int a = it % SA;
-                    const uint32_t aph = (it / SA) & 1;
+                // A block wg & 1 was last read by the MMAs of stage wg - 2, whose completion the
+                // epilogue of that stage has already waited for (it ran before this expansion)
+                const uint8_t* wstage = s.ws + (size_t)st * 128 * p.rowb;
+                const uint32_t a_blk = tbase + lane_base + (uint32_t)((wg & 1) * ACOLS);
+                for (int j = 0; j < SUB; ++j) {
+                    if (w * SUB + j >= KBLK) break;
                     uint32_t wv[BITS];
-                    load_w32<BITS>(wstage, row, j, h, wv);
+                    load_w32<BITS>(wstage, p.rowb, p.swz, row, j, h, wv);
                     uint32_t out[16];
                     expand32<BITS, XT>(wv, out);
-                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.aempty[a], aph ^ 1, s.abort, WAIT_NS, 5));
+                    ptx::tmem_st16(a_blk + (uint32_t)(j * 32 + 16 * h), out);
+                }
+                ptx::tc_wait_st();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(&s.wfree[st]);
+                    ptx::mbar_arrive(&s.afull[wg & 1]);
+                }
+                // fold the previous stage while this one is being multiplied
+                if (w > 0) {
+                    ok = epilogue_stage(wg - 1, w - 1, ti, t);
                     if (!ok) break;
-                    ptx::tmem_st16(tbase + lane_base + a * 32 + 16 * h, out);
-#ifdef AQ_TRACE
-                    { const uint64_t w0 = ptx::globaltimer_ns(); ptx::tc_wait_st(); AQ_TRACE_ADD(9, ptx::globaltimer_ns() - w0); }
-#else
-                    ptx::tc_wait_st();
-#endif
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&s.afull[a]);
                 }
             }
             if (!ok) break;
-            while (g_next < NG) {
-                if (!epilogue_group(g_next)) { ok = false; break; }
-                ++g_next;
-            }
+            ok = epilogue_stage(wg - 1, NWS - 1, ti, t);
             if (!ok) break;
             // ---- store this thread's row of y for its half of the tokens ----
             if (row < ti.nvalid) {
@@ -788,14 +763,11 @@ int num_sms() {
     return n[dev];
 }
 
-// tokens per tile: 16, 32, 64 or 128
+// tokens per tile: 16 or 32 (more tokens take more token tiles)
 int pick_nt(const MmaProblem& p) {
     int64_t m = p.M;
     if (p.offsets) m = 2 * ((p.M + p.n_experts - 1) / p.n_experts);
-    if (m <= 16) return 16;
-    if (m <= 32) return 32;
-    if (m <= 64) return 64;
-    return 128;
+    return m <= 16 ? 16 : 32;
 }
 
 #ifdef AQ_TRACE
@@ -803,40 +775,67 @@ constexpr size_t SMEM_LIMIT = 226 * 1024;  // the trace counters take static sha
 #else
 constexpr size_t SMEM_LIMIT = 227 * 1024;
 #endif
+constexpr int MIN_STAGES = 3;
 
-int wstage_rowb(int bits) { return bits == 6 ? 96 : 128; }
-int wstage_sub(int bits) { return wstage_rowb(bits) * 8 / bits / KB; }
+// W stage geometry: WSC codes per row per stage, at most 4 groups per stage and a row of at most
+// one 128-byte swizzle atom (two A blocks plus 2 x 4 accumulators of 32 columns fill 512 columns).
+struct Geom {
+    int wsc, rowb, sub, gps;
+    uint32_t swz;
+    CUtensorMapSwizzle tma_swz;
+};
+Geom geometry(int bits, int group) {
+    Geom g;
+    int wsc = bits == 6 ? 128 : 1024 / bits;
+    if (wsc > 256) wsc = 256;
+    if (wsc > 4 * group) wsc = 4 * group;
+    g.wsc = wsc;
+    g.rowb = wsc * bits / 8;
+    g.sub = wsc / KB;
+    g.gps = wsc / group;
+    switch (g.rowb) {
+        case 128: g.swz = 7; g.tma_swz = CU_TENSOR_MAP_SWIZZLE_128B; break;
+        case 64: g.swz = 3; g.tma_swz = CU_TENSOR_MAP_SWIZZLE_64B; break;
+        case 32: g.swz = 1; g.tma_swz = CU_TENSOR_MAP_SWIZZLE_32B; break;
+        default: g.swz = 0; g.tma_swz = CU_TENSOR_MAP_SWIZZLE_NONE; break;
+    }
+    return g;
+}
 
-// shared memory of one pipeline stage, and of the parts that do not depend on the stage count
-size_t stage_bytes(int bits) { return (size_t)128 * wstage_rowb(bits); }
-size_t fixed_bytes(int nt, int64_t K, int64_t kg, int xres, int xslots) {
-    return (xres ? (size_t)(K / KB) * nt * 128 : (size_t)xslots * nt * 128) + (size_t)kg * nt * 4 +
+// x in shared memory: all of K when resident, else `xst` x stages of SUB boxes
+size_t fixed_bytes(int nt, int64_t K, int64_t kg, int xres, int xst, const Geom& g) {
+    return (xres ? (size_t)(K / KB) * nt * 128 : (size_t)xst * g.sub * nt * 128) + (size_t)kg * nt * 4 +
            smem_fixed_bytes();
 }
-size_t smem_for(int nt, int bits, int stages, int64_t K, int64_t kg, int xres, int xslots) {
-    return (size_t)stages * stage_bytes(bits) + fixed_bytes(nt, K, kg, xres, xslots);
+size_t smem_for(int nt, int stages, int64_t K, int64_t kg, int xres, int xst, const Geom& g) {
+    return (size_t)stages * 128 * g.rowb + fixed_bytes(nt, K, kg, xres, xst, g);
 }
-int pick_stages(int nt, int bits, int64_t K, int64_t kg, int xres, int xslots) {
-    const size_t fixed = fixed_bytes(nt, K, kg, xres, xslots);
+int pick_stages(int nt, int64_t K, int64_t kg, int xres, int xst, const Geom& g) {
+    const size_t fixed = fixed_bytes(nt, K, kg, xres, xst, g);
     if (fixed >= SMEM_LIMIT) return 0;
-    int st = (int)((SMEM_LIMIT - fixed) / stage_bytes(bits));
+    int st = (int)((SMEM_LIMIT - fixed) / ((size_t)128 * g.rowb));
     if (st > MAX_STAGES) st = MAX_STAGES;
     return st;
 }
-constexpr int MIN_STAGES = 3;
-constexpr int MIN_XSLOTS = 4;
-// streaming x: as many [NT x 64] slots as leave MIN_STAGES + 1 W stages (at most MAX_XSLOTS)
-int pick_xslots(int nt, int bits, int64_t K, int64_t kg) {
-    int best = 0;
-    for (int xs = MIN_XSLOTS; xs <= MAX_XSLOTS; ++xs)
-        if (pick_stages(nt, bits, K, kg, 0, xs) >= MIN_STAGES + 1) best = xs;
-    if (best == 0 && pick_stages(nt, bits, K, kg, 0, MIN_XSLOTS) >= MIN_STAGES) best = MIN_XSLOTS;
-    return best;
-}
-// x stays resident when a CTA sees one token tile and it leaves room for the W pipeline
-int pick_xres(const MmaProblem& p, int nt, int64_t kg) {
-    if (p.offsets || p.M > nt || p.nb[0] * p.nb[1] != 1) return 0;
-    return pick_stages(nt, p.bits, p.K, kg, 1, 0) >= MIN_STAGES + 1 ? 1 : 0;
+// x stays resident when a CTA sees one token tile and that leaves a deep enough W pipeline;
+// otherwise the deepest x ring (<= 4) that keeps at least 4 W stages
+struct XPlan {
+    int xres, xst, stages;
+};
+XPlan pick_x(const MmaProblem& p, int nt, int64_t kg, const Geom& g) {
+    XPlan r{0, 2, 0};
+    if (!p.offsets && p.M <= nt && p.nb[0] * p.nb[1] == 1 && pick_stages(nt, p.K, kg, 1, 0, g) >= 6) {
+        r.xres = 1;
+        r.xst = 0;
+    } else {
+        for (int xst = MAX_XST; xst > 2; --xst)
+            if (pick_stages(nt, p.K, kg, 0, xst, g) >= 4) {
+                r.xst = xst;
+                break;
+            }
+    }
+    r.stages = pick_stages(nt, p.K, kg, r.xres, r.xst, g);
+    return r;
 }
 
 template <int BITS, typename XT, int NT>
@@ -862,13 +861,7 @@ cudaError_t launch_t(const MmaParams& prm, int grid, size_t smem, cudaStream_t s
 
 template <int BITS, typename XT>
 cudaError_t launch_nt(int nt, const MmaParams& prm, int grid, size_t smem, cudaStream_t s) {
-    switch (nt) {
-        case 16: return launch_t<BITS, XT, 16>(prm, grid, smem, s);
-        case 32: return launch_t<BITS, XT, 32>(prm, grid, smem, s);
-        case 64: return launch_t<BITS, XT, 64>(prm, grid, smem, s);
-        case 128: return launch_t<BITS, XT, 128>(prm, grid, smem, s);
-    }
-    return cudaErrorInvalidValue;
+    return nt == 16 ? launch_t<BITS, XT, 16>(prm, grid, smem, s) : launch_t<BITS, XT, 32>(prm, grid, smem, s);
 }
 
 template <typename XT>
@@ -903,7 +896,8 @@ bool mma_supported(const MmaProblem& p, const char** why) {
     if (p.M > INT32_MAX / 2 || p.N * (p.offsets ? p.n_experts : 1) > INT32_MAX / 2)
         return no("problem too large for 32-bit tile coordinates");
     const int nt = pick_nt(p);
-    if ((size_t)kg * nt * 4 > XTAB_MAX_BYTES || (pick_xres(p, nt, kg) == 0 && pick_xslots(nt, p.bits, p.K, kg) == 0))
+    const Geom g = geometry(p.bits, p.group);
+    if ((size_t)kg * nt * 4 > XTAB_MAX_BYTES || pick_stages(nt, p.K, kg, 0, 2, g) < MIN_STAGES)
         return no("K/group too large for the sum-of-x table of the tensor-core kernel");
     if (!get_encode()) return no("driver entry point cuTensorMapEncodeTiled unavailable");
     return true;
@@ -917,10 +911,10 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     const int nt = pick_nt(pb);
     const int bits = pb.bits;
     const int64_t kg = pb.K / pb.group;
-    const int xres = pick_xres(pb, nt, kg);
-    const int xslots = xres ? 0 : pick_xslots(nt, bits, pb.K, kg);
-    const int stages = pick_stages(nt, bits, pb.K, kg, xres, xslots);
-    if (stages < MIN_STAGES || (!xres && xslots < MIN_XSLOTS)) return cudaErrorInvalidValue;
+    const Geom geo = geometry(bits, pb.group);
+    const XPlan xp = pick_x(pb, nt, kg, geo);
+    const int stages = xp.stages;
+    if (stages < MIN_STAGES) return cudaErrorInvalidValue;
     const int64_t rows_total = pb.M;
     // ---- x tensor map: {K, rows, nb1, nb0}
     {
@@ -936,16 +930,15 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
-    // ---- W tensor map: {K*bits/32 words, rows}
+    // ---- W tensor map: {K*bits/32 words, rows}, box {rowb/4 words, 128 rows}
     {
         const int64_t wrows = pb.offsets ? pb.N * pb.n_experts : pb.N;
         cuuint64_t dims[2] = {(cuuint64_t)(pb.K * bits / 32), (cuuint64_t)wrows};
         cuuint64_t strides[1] = {(cuuint64_t)(pb.w_row * 4)};
-        cuuint32_t box[2] = {(cuuint32_t)(wstage_rowb(bits) / 4), 128};
+        cuuint32_t box[2] = {(cuuint32_t)(geo.rowb / 4), 128};
         cuuint32_t estr[2] = {1, 1};
-        CUtensorMapSwizzle sw = wstage_rowb(bits) == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
         CUresult r = encode(&prm.tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(pb.wq), dims, strides,
-                            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, geo.tma_swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
@@ -970,13 +963,19 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     int lg = 0;
     while ((1 << lg) < pb.group) ++lg;
     prm.log2g = lg;
-    prm.stages = stages;
     prm.kg = (int)kg;
-    prm.xres = xres;
-    prm.xslots = xslots;
-    prm.n_wstages = (int)((pb.K / KB + wstage_sub(bits) - 1) / wstage_sub(bits));
     prm.ydt = (int)pb.ydt;
-    uint32_t cols = SA * 32 + nbufs(nt) * nt, pw = 32;
+    prm.wsc = geo.wsc;
+    prm.rowb = geo.rowb;
+    prm.sub = geo.sub;
+    prm.gps = geo.gps;
+    prm.swz = geo.swz;
+    prm.n_wstages = (int)((pb.K + geo.wsc - 1) / geo.wsc);
+    prm.stages = stages;
+    prm.cs_w = SCW / geo.gps;
+    prm.xres = xp.xres;
+    prm.xst = xp.xst;
+    uint32_t cols = (uint32_t)(geo.wsc + 2 * geo.gps * nt), pw = 32;
     while (pw < cols) pw <<= 1;
     prm.tmem_cols = pw;
     prm.idesc = ptx::idesc_f16(nt, pb.xdt == DT::BF16 ? 1 : 0);
@@ -991,7 +990,7 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
         const int64_t tiles = (int64_t)prm.n_wtiles * prm.n_ttiles * prm.nbatch;
         grid = (int)(tiles < sms ? tiles : sms);
     }
-    const size_t smem = smem_for(nt, bits, stages, pb.K, kg, xres, xslots);
+    const size_t smem = smem_for(nt, stages, pb.K, kg, xp.xres, xp.xst, geo);
     if (pb.xdt == DT::BF16) return launch_bits<bf16_t>(bits, nt, prm, grid, smem, stream);
     return launch_bits<f16_t>(bits, nt, prm, grid, smem, stream);
 }
