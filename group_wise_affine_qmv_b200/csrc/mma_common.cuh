@@ -1,0 +1,92 @@
+// mma_common.cuh -- definitions shared by the host side of the tensor-core kernel
+// (kernels_mma.cu) and its device code (mma_kernel.cuh, instantiated once per bit width in
+// kernels_mma_b{2,4,6,8}.cu so that the four compile in parallel).
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace aq {
+namespace mma {
+
+// ---- warp roles ----
+constexpr int EXP_WARPS = 8;                              // warps 2..9: code expanders
+constexpr int FOLD_WARPS = 8;                             // warps 10..17: s*D + b*X folds
+constexpr int FOLD_THREADS = 32 * FOLD_WARPS;
+constexpr int XPROD_WARP = 2 + EXP_WARPS + FOLD_WARPS;    // warp 18: x producer
+constexpr int THREADS = 32 * (XPROD_WARP + 1);            // 608
+
+// ---- tiling ----
+constexpr int NT = 32;                    // tokens per tile (the MMA's N)
+constexpr int KB = 64;                    // codes per MMA sub-step (4 tcgen05.mma of K = 16)
+constexpr int SCW = 32;                   // groups per scale/bias chunk
+constexpr int SCP = SCW + 2;              // padded row pitch (halves) of a chunk in shared memory
+constexpr int MAX_STAGES = 12;            // W ring
+constexpr int MAX_XST = 4;                // streamed x ring
+constexpr int MAX_EXPERTS = 1024;
+constexpr int XTAB_MAX_BYTES = 32 * 1024; // sums of x per group and token of one token tile
+constexpr int XV = 2;                     // 16-byte loads in flight per thread while summing x
+constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait
+constexpr int ERR_TIMEOUT = 1;
+
+// W stage geometry.  A stage is 128 rows x WSC codes: at most 4 groups (so that two A blocks
+// of WSC/2 columns and two sets of 4 group accumulators of NT columns fit the 512 tensor-memory
+// columns) and a row of at most one 128-byte swizzle atom (96 bytes for 6-bit codes).
+__host__ __device__ constexpr int stage_codes(int bits, int group) {
+    return bits == 6 ? 128 : (1024 / bits < 256 ? (1024 / bits < 4 * group ? 1024 / bits : 4 * group)
+                                                : (256 < 4 * group ? 256 : 4 * group));
+}
+__host__ __device__ constexpr int stage_rowb(int bits, int group) { return stage_codes(bits, group) * bits / 8; }
+// XOR mask of the TMA swizzle on byte-address bits [4..6] from bits [7..9]
+__host__ __device__ constexpr uint32_t stage_swz(int rowb) {
+    return rowb == 128 ? 7u : rowb == 64 ? 3u : rowb == 32 ? 1u : 0u;
+}
+
+struct Params {
+    CUtensorMap tx;  // x: 4D {K, rows, nb1, nb0} u16, box {64, NT, 1, 1}, 128-byte swizzle
+    CUtensorMap tw;  // W: 2D {K*bits/32, rows} u32, box {rowb/4, 128}, swizzle by row bytes
+    const void* x;
+    void* y;
+    const uint16_t* scales;
+    const uint16_t* biases;
+    int64_t M, N, K;
+    int64_t x_row, y_row;
+    int64_t xb[2], yb[2];
+    int64_t nb1;
+    int n_wtiles, n_ttiles, nbatch;
+    int kg;              // groups per row = K / group
+    int ydt;             // DT of y
+    int n_wstages;       // W stages per tile
+    int stages;          // W ring depth
+    int xres;            // 1: the CTA's single x tile stays resident in shared memory
+    int xst;             // streamed x ring depth (x stages of SUB boxes) when not resident
+    uint32_t tmem_cols;
+    uint32_t idesc;
+    const int64_t* offsets;  // grouped mode when non-null
+    int n_experts;
+    int* err;                    // device error word (set on a timed-out wait)
+    unsigned long long* trace;   // instrumented builds only: per-site counters [64]
+    long long* tl;               // instrumented builds only: event timeline [16][512]
+};
+
+// shared memory besides the x buffer, the W ring and the sum-of-x table
+__host__ __device__ constexpr size_t smem_fixed_bytes() {
+    return 2 * 2 * 128 * SCP * 2                                  // scale/bias chunk slots
+           + (2 * MAX_STAGES + 2 * MAX_XST + 2 * 4 + 3) * 8 + 8  // mbarriers, TMEM base, abort flag
+           + (MAX_EXPERTS + 1) * 4                               // grouped tile prefix sums
+           + 2 * 1024;                                           // alignment
+}
+
+// defined in mma_kernel.cuh, instantiated in kernels_mma_b<BITS>.cu
+template <int BITS>
+cudaError_t launch(bool bf16, int group, const Params& prm, int grid, size_t smem, cudaStream_t stream);
+extern template cudaError_t launch<2>(bool, int, const Params&, int, size_t, cudaStream_t);
+extern template cudaError_t launch<4>(bool, int, const Params&, int, size_t, cudaStream_t);
+extern template cudaError_t launch<6>(bool, int, const Params&, int, size_t, cudaStream_t);
+extern template cudaError_t launch<8>(bool, int, const Params&, int, size_t, cudaStream_t);
+
+}  // namespace mma
+}  // namespace aq

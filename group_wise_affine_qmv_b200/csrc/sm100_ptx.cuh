@@ -9,8 +9,7 @@
 #include <stdint.h>
 
 #ifdef AQ_TRACE
-__device__ unsigned long long aq_trace_ns[64];     // one translation unit includes this header
-__shared__ unsigned long long aq_trace_smem[64];   // per-CTA accumulation, flushed at exit
+static __shared__ unsigned long long aq_trace_smem[64];   // per-CTA accumulation, flushed at exit
 #endif
 
 namespace aq {
@@ -154,15 +153,14 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16 (bf16/f16 inputs, fp32 accumulate)
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16 (bf16/f16 inputs, fp32 accumulate); the accumulate
+// flag is an immediate (ACC = 0: D = A.B, 1: D += A.B)
+template <int ACC>
+__device__ __forceinline__ void mma_ts_imm(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc) {
+    asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, %4;"
+                 ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "n"(ACC)
+                 : "memory");
 }
 
 // arrive on `bar` when all previously issued tcgen05 async operations of this thread complete
