@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "aq_internal.h"
@@ -95,16 +96,20 @@ Geom geometry(int bits, int group) {
     return g;
 }
 
-// x in shared memory: all of K when resident, else `xst` x stages of SUB boxes
-size_t fixed_bytes(int64_t K, int64_t kg, int xres, int xst, const Geom& g) {
-    return (xres ? (size_t)(K / KB) * NT * 128 : (size_t)xst * g.sub * NT * 128) + (size_t)kg * NT * 4 +
-           smem_fixed_bytes();
+// Shared memory of one CTA whose K range spans at most `ms` W stages: x (that range when
+// resident, else `xst` x stages of SUB boxes), the sum-of-x table of the range, the partial
+// tile of a split, and the fixed part.
+size_t fixed_bytes(int64_t K, int64_t kg, int ms, int split, int xres, int xst, const Geom& g) {
+    const int64_t boxes = std::min<int64_t>((int64_t)ms * g.sub, K / KB);
+    const int64_t groups = std::min<int64_t>((int64_t)ms * (g.wsc / (K / kg)), kg);
+    return (xres ? (size_t)boxes * NT * 128 : (size_t)xst * g.sub * NT * 128) + (size_t)groups * NT * 4 +
+           (split > 1 ? (size_t)RED_BYTES : 0) + smem_fixed_bytes();
 }
-size_t smem_for(int stages, int64_t K, int64_t kg, int xres, int xst, const Geom& g) {
-    return (size_t)stages * 128 * g.rowb + fixed_bytes(K, kg, xres, xst, g);
+size_t smem_for(int stages, int64_t K, int64_t kg, int ms, int split, int xres, int xst, const Geom& g) {
+    return (size_t)stages * 128 * g.rowb + fixed_bytes(K, kg, ms, split, xres, xst, g);
 }
-int pick_stages(int64_t K, int64_t kg, int xres, int xst, const Geom& g) {
-    const size_t fixed = fixed_bytes(K, kg, xres, xst, g);
+int pick_stages(int64_t K, int64_t kg, int ms, int split, int xres, int xst, const Geom& g) {
+    const size_t fixed = fixed_bytes(K, kg, ms, split, xres, xst, g);
     if (fixed >= SMEM_LIMIT) return 0;
     int st = (int)((SMEM_LIMIT - fixed) / ((size_t)128 * g.rowb));
     if (st > MAX_STAGES) st = MAX_STAGES;
@@ -115,20 +120,31 @@ int pick_stages(int64_t K, int64_t kg, int xres, int xst, const Geom& g) {
 struct XPlan {
     int xres, xst, stages;
 };
-XPlan pick_x(const MmaProblem& p, int64_t kg, const Geom& g) {
+XPlan pick_x(const MmaProblem& p, int64_t kg, int ms, int split, const Geom& g) {
     XPlan r{0, 2, 0};
-    if (!p.offsets && p.M <= NT && p.nb[0] * p.nb[1] == 1 && pick_stages(p.K, kg, 1, 0, g) >= 6) {
+    if (!p.offsets && p.M <= NT && p.nb[0] * p.nb[1] == 1 && pick_stages(p.K, kg, ms, split, 1, 0, g) >= 6) {
         r.xres = 1;
         r.xst = 0;
     } else {
         for (int xst = MAX_XST; xst > 2; --xst)
-            if (pick_stages(p.K, kg, 0, xst, g) >= 4) {
+            if (pick_stages(p.K, kg, ms, split, 0, xst, g) >= 4) {
                 r.xst = xst;
                 break;
             }
     }
-    r.stages = pick_stages(p.K, kg, r.xres, r.xst, g);
+    r.stages = pick_stages(p.K, kg, ms, split, r.xres, r.xst, g);
     return r;
+}
+
+// CTAs per cluster splitting each tile's K: when the tiles alone would leave most SMs idle,
+// the largest power of two <= 8 that keeps the grid within the SMs and gives every rank
+// at least one W stage (two when a stage holds one group)
+int pick_split(int64_t tiles, int nws, int gps, int sms) {
+    const int u = gps == 1 ? 2 : 1;
+    const int nu = (nws + u - 1) / u;
+    int cs = 1;
+    while (cs < 8 && tiles * cs * 2 <= sms && cs * 2 <= nu) cs *= 2;
+    return cs;
 }
 
 }  // namespace
@@ -153,7 +169,8 @@ bool mma_supported(const MmaProblem& p, const char** why) {
     if (p.M > INT32_MAX / 2 || p.N * (p.offsets ? p.n_experts : 1) > INT32_MAX / 2)
         return no("problem too large for 32-bit tile coordinates");
     const Geom g = geometry(p.bits, p.group);
-    if ((size_t)kg * NT * 4 > XTAB_MAX_BYTES || pick_stages(p.K, kg, 0, 2, g) < MIN_STAGES)
+    if ((size_t)kg * NT * 4 > XTAB_MAX_BYTES ||
+        pick_stages(p.K, kg, (int)((p.K + g.wsc - 1) / g.wsc), 1, 0, 2, g) < MIN_STAGES)
         return no("K/group too large for the sum-of-x table of the tensor-core kernel");
     if (!get_encode()) return no("driver entry point cuTensorMapEncodeTiled unavailable");
     return true;
@@ -167,7 +184,13 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     const int bits = pb.bits;
     const int64_t kg = pb.K / pb.group;
     const Geom geo = geometry(bits, pb.group);
-    const XPlan xp = pick_x(pb, kg, geo);
+    const int nws = (int)((pb.K + geo.wsc - 1) / geo.wsc);
+    const int gps = geo.wsc / pb.group;
+    const int sms = num_sms();
+    const int64_t tiles = pb.offsets ? 0 : ((pb.N + 127) / 128) * ((pb.M + NT - 1) / NT) * pb.nb[0] * pb.nb[1];
+    const int split = pb.offsets ? 1 : pick_split(tiles, nws, gps, sms);
+    const int ms = split > 1 ? split_max_stages(nws, gps, split) : nws;
+    const XPlan xp = pick_x(pb, kg, ms, split, geo);
     const int stages = xp.stages;
     if (stages < MIN_STAGES) return cudaErrorInvalidValue;
     const int64_t rows_total = pb.M;
@@ -216,7 +239,8 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     prm.nbatch = (int)(pb.nb[0] * pb.nb[1]);
     prm.kg = (int)kg;
     prm.ydt = (int)pb.ydt;
-    prm.n_wstages = (int)((pb.K + geo.wsc - 1) / geo.wsc);
+    prm.n_wstages = nws;
+    prm.ksplit = split;
     prm.stages = stages;
     prm.xres = xp.xres;
     prm.xst = xp.xst;
@@ -248,15 +272,11 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     }
 #endif
 
-    const int sms = num_sms();
     int grid;
-    if (pb.offsets) {
-        grid = sms;
-    } else {
-        const int64_t tiles = (int64_t)prm.n_wtiles * prm.n_ttiles * prm.nbatch;
-        grid = (int)(tiles < sms ? tiles : sms);
-    }
-    const size_t smem = smem_for(stages, pb.K, kg, xp.xres, xp.xst, geo);
+    if (pb.offsets) grid = sms;
+    else if (split > 1) grid = (int)tiles * split;   // one tile per cluster
+    else grid = (int)(tiles < sms ? tiles : sms);
+    const size_t smem = smem_for(stages, pb.K, kg, ms, split, xp.xres, xp.xst, geo);
     const bool bf = pb.xdt == DT::BF16;
     switch (bits) {
         case 2: return launch<2>(bf, pb.group, prm, grid, smem, stream);

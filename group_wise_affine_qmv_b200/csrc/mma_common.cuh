@@ -67,15 +67,35 @@ struct Params {
     uint32_t idesc;
     const int64_t* offsets;  // grouped mode when non-null
     int n_experts;
+    int ksplit;                  // CTAs per cluster splitting each tile's K (1: no split)
     int* err;                    // device error word (set on a timed-out wait)
     unsigned long long* trace;   // instrumented builds only: per-site counters [64]
     long long* tl;               // instrumented builds only: event timeline [16][512]
 };
 
+// W stages [w0, w1) of the tile handled by rank `rank` of `cs` CTAs splitting K.  Ranges
+// start at an even group (4-byte scale/bias copies), so with one group per stage they move
+// in units of two stages.
+__host__ __device__ inline void split_range(int nws, int gps, int cs, int rank, int* w0, int* w1) {
+    const int u = gps == 1 ? 2 : 1;
+    const int nu = (nws + u - 1) / u;
+    const int a = u * (nu * rank / cs), b = u * (nu * (rank + 1) / cs);
+    *w0 = a < nws ? a : nws;
+    *w1 = b < nws ? b : nws;
+}
+// the most W stages any rank gets
+__host__ __device__ inline int split_max_stages(int nws, int gps, int cs) {
+    const int u = gps == 1 ? 2 : 1;
+    const int nu = (nws + u - 1) / u;
+    const int m = u * ((nu + cs - 1) / cs);
+    return m < nws ? m : nws;
+}
+constexpr int RED_BYTES = FOLD_THREADS * (NT / 2) * 4;  // one CTA's partial y tile (fp32)
+
 // shared memory besides the x buffer, the W ring and the sum-of-x table
 __host__ __device__ constexpr size_t smem_fixed_bytes() {
     return 2 * 2 * 128 * SCP * 2                                  // scale/bias chunk slots
-           + (2 * MAX_STAGES + 2 * MAX_XST + 2 * 4 + 3) * 8 + 8  // mbarriers, TMEM base, abort flag
+           + (2 * MAX_STAGES + 2 * MAX_XST + 2 * 4 + 5) * 8 + 8  // mbarriers, TMEM base, abort flag
            + (MAX_EXPERTS + 1) * 4                               // grouped tile prefix sums
            + 2 * 1024;                                           // alignment
 }

@@ -62,10 +62,11 @@ namespace mma {
 #define AQ_TSTOP(site, v)
 #endif
 #ifdef AQ_TIMELINE
-// timeline builds: clock64 of events in CTA 0, relative to its start
+// timeline builds: clock64 of events in CTAs 0 and 1, relative to each CTA's start
 #define AQ_TL(ev, idx, cond)                                                                         \
     do {                                                                                             \
-        if (blockIdx.x == 0 && (cond) && (idx) < 512) p.tl[(ev) * 512 + (idx)] = clock64() - tl0; \
+        if (blockIdx.x < 2 && (cond) && (idx) >= 0 && (idx) < 256)                                   \
+            p.tl[(ev) * 512 + 256 * blockIdx.x + (idx)] = clock64() - tl0;                             \
     } while (0)
 #else
 #define AQ_TL(ev, idx, cond)
@@ -94,26 +95,33 @@ struct Smem {
     uint64_t* xbar;      // sum-of-x table (fold threads)
     uint64_t* xres_full; // resident x landed
     uint64_t* mdone;     // teardown: all MMAs retired
+    uint64_t* red_full;  // split K: every rank's part of this CTA's rows has arrived (fold warps)
+    uint64_t* red_done;  // (unused)
     uint32_t* tmem_base;
     int* abort;
     int* prefix;         // grouped: tile prefix sums [n_experts + 1]
-    float* xtab;         // [kg][NT] sums of x per group and token
+    float* xtab;         // [groups of this CTA's K range][NT] sums of x per group and token
+    float* red;          // split K: partial sums of this CTA's rows [ranks][128 / ranks][NT] from every rank
     uint8_t* xs;         // resident: [K/64][NT][128 B]; streamed: [xst][SUB][NT][128 B]
     uint8_t* ws;         // [stages][128 rows][ROWB]
     uint16_t* sb;        // [2 slots][2 arrays][128][SCP]
 };
 
-template <int SUB, int ROWB>
-__device__ __forceinline__ Smem carve(uint8_t* base, const Params& p) {
+// ms: the most W stages of one CTA's K range
+template <int SUB, int ROWB, int GPS>
+__device__ __forceinline__ Smem carve(uint8_t* base, const Params& p, int ms) {
     Smem s;
     uint8_t* q = base;
     s.xs = q;
-    q += p.xres ? (size_t)(p.K / KB) * NT * 128 : (size_t)p.xst * SUB * NT * 128;
+    const int64_t boxes = min64((int64_t)ms * SUB, p.K / KB);
+    q += p.xres ? (size_t)boxes * NT * 128 : (size_t)p.xst * SUB * NT * 128;
     s.ws = q;
     q += (size_t)p.stages * 128 * ROWB;
     q = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(q) + 1023) & ~uintptr_t(1023));
     s.xtab = reinterpret_cast<float*>(q);
-    q += (size_t)p.kg * NT * 4;
+    q += (size_t)min(ms * GPS, p.kg) * NT * 4;
+    s.red = reinterpret_cast<float*>(q);
+    if (p.ksplit > 1) q += RED_BYTES;
     s.sb = reinterpret_cast<uint16_t*>(q);
     q += 2 * 2 * 128 * SCP * 2;
     s.wfull = reinterpret_cast<uint64_t*>(q);
@@ -127,7 +135,9 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const Params& p) {
     s.xbar = s.sbar + 2;
     s.xres_full = s.xbar + 1;
     s.mdone = s.xres_full + 1;
-    s.tmem_base = reinterpret_cast<uint32_t*>(s.mdone + 1);
+    s.red_full = s.mdone + 1;
+    s.red_done = s.red_full + 1;
+    s.tmem_base = reinterpret_cast<uint32_t*>(s.red_done + 1);
     s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
     s.prefix = s.abort + 1;
     return s;
@@ -292,13 +302,12 @@ __device__ __forceinline__ void expand32(const uint32_t* w, uint32_t* out) {
 }
 
 // ---------------------------------------------------------------------------
-// scale/bias chunk loads: fold thread tid copies groups [32c, 32c + 32) of row tid % 128,
-// scales for tid < 128 and biases above, with 4-byte asynchronous copies
+// scale/bias chunk loads: fold thread tid copies groups [g0, min(g0 + 32, g_end)) of row
+// tid % 128, scales for tid < 128 and biases above, with 4-byte asynchronous copies
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void issue_sb_chunk(const Params& p, const TileInfo& ti, int chunk, uint16_t* slot,
-                                               int tid) {
-    const int g0 = chunk * SCW;
-    const int pairs = min(SCW, p.kg - g0) >> 1;  // kg even, SCW even
+__device__ __forceinline__ void issue_sb_chunk(const Params& p, const TileInfo& ti, int g0, int g_end,
+                                               uint16_t* slot, int tid) {
+    const int pairs = min(SCW, g_end - g0) >> 1;  // g0 and g_end even
     const int r = tid & 127, arr = tid >> 7;
     const int64_t row = ti.wrow0 + min(r, ti.nvalid - 1);
     const uint16_t* src = (arr ? p.biases : p.scales) + row * p.kg + g0;
@@ -309,12 +318,13 @@ __device__ __forceinline__ void issue_sb_chunk(const Params& p, const TileInfo& 
 // sum over each group of x[t, k] (widened to fp32 first, added in k order) for the tile's
 // tokens -> xtab[g][t], from global memory
 template <typename XT, int G>
-__device__ __forceinline__ void build_xtab(const Params& p, const TileInfo& ti, float* xtab, int tid) {
+__device__ __forceinline__ void build_xtab(const Params& p, const TileInfo& ti, int g_lo, int g_hi, float* xtab,
+                                           int tid) {
     const XT* xb = (const XT*)p.x + (p.offsets ? 0 : (int64_t)ti.b0 * p.xb[0] + (int64_t)ti.b1 * p.xb[1]);
-    const int items = p.kg * NT;
+    const int items = (g_hi - g_lo) * NT;
     constexpr int VPG = G / 8;  // 16-byte vectors of 8 elements per group
     for (int it = tid; it < items; it += FOLD_THREADS) {
-        const int g = it / NT, t = it - g * NT;
+        const int gr = it / NT, t = it - gr * NT, g = g_lo + gr;
         float acc = 0.0f;
         if (t < ti.tvalid) {
             const uint4* row = reinterpret_cast<const uint4*>(xb + (ti.xrow0 + t) * p.x_row + (int64_t)g * G);
@@ -332,15 +342,16 @@ __device__ __forceinline__ void build_xtab(const Params& p, const TileInfo& ti, 
                 }
             }
         }
-        xtab[g * NT + t] = acc;
+        xtab[gr * NT + t] = acc;
     }
 }
 
 // the same sums from the resident x tile ([K/64][NT][128 B], 128-byte swizzle: 16-byte chunk
 // c of token row t sits at chunk c ^ (t & 7)); rows past the valid tokens are zero fill
+// (the resident buffer starts at group g_lo)
 template <typename XT, int G>
-__device__ __forceinline__ void build_xtab_smem(const Params& p, const uint8_t* xs, float* xtab, int tid) {
-    const int items = p.kg * NT;
+__device__ __forceinline__ void build_xtab_smem(int ngroups, const uint8_t* xs, float* xtab, int tid) {
+    const int items = ngroups * NT;
     constexpr int VPG = G / 8;
     for (int it = tid; it < items; it += FOLD_THREADS) {
         const int g = it / NT, t = it - g * NT;
@@ -392,7 +403,9 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const Smem s = carve<SUB, ROWB>(base, p);
+    const int NWS = p.n_wstages;
+    const int cs = p.ksplit;   // CTAs of a cluster splitting each tile's K (1: none)
+    const Smem s = carve<SUB, ROWB, GPS>(base, p, cs > 1 ? split_max_stages(NWS, GPS, cs) : NWS);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     AQ_TSTART(t_kernel);
 #ifdef AQ_TIMELINE
@@ -401,8 +414,6 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
     const int S = p.stages;
     const int KBLK = (int)(p.K / KB);
     const int NG = p.kg;
-    const int NWS = p.n_wstages;
-    const int NCH = (NG + SCW - 1) / SCW;   // scale/bias chunks per tile
 
 #ifdef AQ_TRACE
     if (threadIdx.x < 64) aq_trace_smem[threadIdx.x] = 0;
@@ -425,6 +436,9 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         ptx::mbar_init(s.xbar, FOLD_THREADS);
         ptx::mbar_init(s.xres_full, 1);
         ptx::mbar_init(s.mdone, 1);
+        if (cs > 1) {
+            ptx::mbar_init(s.red_full, cs * FOLD_WARPS);
+        }
         *s.abort = 0;
         ptx::fence_mbar_init();
     }
@@ -436,6 +450,11 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         ptx::tmem_alloc(s.tmem_base, p.tmem_cols);
         ptx::tmem_relinquish();
     }
+    // Programmatic dependent launch: the next kernel in the stream may start its own prologue
+    // now; this grid reads nothing an earlier kernel may write (x, W, scales, biases, offsets)
+    // and writes no y before the earlier grids have completed.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     if (p.offsets && warp == 2) {
         // tiles per expert: ceil(count / NT) * n_wtiles, prefix-summed
         if (lane == 0) s.prefix[0] = 0;
@@ -460,11 +479,24 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
+    if (cs > 1) {
+        // every CTA of the cluster has initialised its barriers before any remote arrival
+        asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    }
     const uint32_t tbase = *s.tmem_base;
     const uint32_t d_tmem = tbase + (uint32_t)WSC;  // 2 x GPS group accumulators follow the two A blocks
     const int ntiles = total_tiles(p, s);
-    const bool has_tiles = (int)blockIdx.x < ntiles;
+    // split K: cluster c takes tile c, its rank r the W stages [w0, w1); otherwise the CTA walks
+    // tiles blockIdx.x, blockIdx.x + gridDim.x, ... over all stages
+    const int rank = cs > 1 ? (int)(blockIdx.x % cs) : 0;
+    const int tile0 = cs > 1 ? (int)(blockIdx.x / cs) : (int)blockIdx.x;
+    const int tstep = cs > 1 ? ntiles : (int)gridDim.x;
+    int w0 = 0, w1 = NWS;
+    if (cs > 1) split_range(NWS, GPS, cs, rank, &w0, &w1);
+    const int g_lo = w0 * GPS, g_hi = min(w1 * GPS, NG);
+    const bool has_tiles = tile0 < ntiles;
     if (warp == 1) AQ_TSTOP(15, t_kernel);
+    AQ_TL(10, 1, threadIdx.x == 32);
 
     if (warp == 0) {
         // ======================= W producer =======================
@@ -472,9 +504,9 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         const bool leader = lane == 0;
         uint32_t wg = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        for (int t = tile0; t < ntiles && ok; t += tstep) {
             const TileInfo ti = tile_info(p, s, t);
-            for (int w = 0; w < NWS; ++w) {
+            for (int w = w0; w < w1; ++w) {
                 const int st = wg % S;
                 ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfree[st], ((wg / S) & 1) ^ 1, s.abort, WAIT_NS, 0));
                 if (!ok) break;
@@ -504,19 +536,21 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         if (p.xres) {
             if (has_tiles && leader) {
                 // the CTA's only token tile: all of K, once
-                const TileInfo t0 = tile_info(p, s, blockIdx.x);
-                ptx::mbar_arrive_expect_tx(s.xres_full, (uint32_t)KBLK * NT * 128);
-                for (int kb = 0; kb < KBLK; ++kb)
-                    ptx::tma_load_4d(s.xs + (size_t)kb * NT * 128, &p.tx, s.xres_full, kb * KB, (int32_t)t0.xrow0,
-                                     t0.b1, t0.b0);
+                // the CTA's only token tile: its K range, once
+                const TileInfo t0 = tile_info(p, s, tile0);
+                const int kb0 = w0 * SUB, kb1 = min(w1 * SUB, KBLK);
+                ptx::mbar_arrive_expect_tx(s.xres_full, (uint32_t)(kb1 - kb0) * NT * 128);
+                for (int kb = kb0; kb < kb1; ++kb)
+                    ptx::tma_load_4d(s.xs + (size_t)(kb - kb0) * NT * 128, &p.tx, s.xres_full, kb * KB,
+                                     (int32_t)t0.xrow0, t0.b1, t0.b0);
                 volatile int never = 0;
                 ptx::mbar_wait(s.xres_full, 0, &never, 200000000ull);
             }
         } else {
             const int XS = p.xst;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            for (int t = tile0; t < ntiles && ok; t += tstep) {
                 const TileInfo ti = tile_info(p, s, t);
-                for (int w = 0; w < NWS; ++w) {
+                for (int w = w0; w < w1; ++w) {
                     const int xs = wg % XS;
                     ok = __all_sync(0xffffffffu,
                                     ptx::mbar_wait(&s.xfree[xs], ((wg / XS) & 1) ^ 1, s.abort, WAIT_NS, 9));
@@ -547,8 +581,8 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         uint32_t wg = 0;
         bool ok = true;
         if (p.xres && has_tiles) ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xres_full, 0, s.abort, WAIT_NS, 1));
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            for (int w = 0; w < NWS; ++w, ++wg) {
+        for (int t = tile0; t < ntiles && ok; t += tstep) {
+            for (int w = w0; w < w1; ++w, ++wg) {
                 const int slot = wg & 1;
                 const uint32_t ph = (wg >> 1) & 1;
                 const int xs = p.xres ? 0 : (int)(wg % (uint32_t)p.xst);
@@ -571,7 +605,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                     const uint32_t d_blk = d_tmem + (uint32_t)(slot * GPS * NT);
                     // B operand: the stage's first 64-code box; boxes are NT*128 bytes apart
                     const uint64_t bdesc = ptx::smem_desc_sw128(ptx::smem_u32(
-                        p.xres ? s.xs + (size_t)w * SUB * NT * 128 : s.xs + (size_t)xs * SUB * NT * 128));
+                        p.xres ? s.xs + (size_t)(w - w0) * SUB * NT * 128 : s.xs + (size_t)xs * SUB * NT * 128));
                     const int nsub = min(SUB, KBLK - w * SUB);
 #pragma unroll
                     for (int j = 0; j < SUB; ++j) {
@@ -614,8 +648,8 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         uint32_t wg = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            for (int w = 0; w < NWS; ++w, ++wg) {
+        for (int t = tile0; t < ntiles && ok; t += tstep) {
+            for (int w = w0; w < w1; ++w, ++wg) {
                 const int st = wg % S;
                 ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfull[st], (wg / S) & 1, s.abort, WAIT_NS, 4));
                 if (!ok) break;
@@ -673,8 +707,8 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         bool ok = true;
 
         if (has_tiles) {
-            const TileInfo t0 = tile_info(p, s, blockIdx.x);
-            issue_sb_chunk(p, t0, 0, s.sb, tid);
+            const TileInfo t0 = tile_info(p, s, tile0);
+            issue_sb_chunk(p, t0, g_lo, g_hi, s.sb, tid);
         }
         ptx::cp_async_commit();
         const uint16_t* sbslot = s.sb;
@@ -682,7 +716,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         int64_t cur_x0 = -1;
         int cur_b0 = -1, cur_b1 = -1, cur_tv = -1;
 
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        for (int t = tile0; t < ntiles && ok; t += tstep) {
             const TileInfo ti = tile_info(p, s, t);
             AQ_TL(8, (t - (int)blockIdx.x) / (int)gridDim.x, threadIdx.x == 320);
             if (ti.xrow0 != cur_x0 || ti.b0 != cur_b0 || ti.b1 != cur_b1 || ti.tvalid != cur_tv) {
@@ -694,9 +728,9 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 if (p.xres) {
                     ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xres_full, 0, s.abort, WAIT_NS, 8));
                     if (!ok) break;
-                    build_xtab_smem<XT, G>(p, s.xs, s.xtab, tid);
+                    build_xtab_smem<XT, G>(g_hi - g_lo, s.xs, s.xtab, tid);
                 } else {
-                    build_xtab<XT, G>(p, ti, s.xtab, tid);
+                    build_xtab<XT, G>(p, ti, g_lo, g_hi, s.xtab, tid);
                 }
                 ptx::mbar_arrive(s.xbar);
                 ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_NS, 8));
@@ -710,8 +744,8 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
             float2 acc[H / 2];
 #pragma unroll
             for (int i = 0; i < H / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
-            for (int w = 0; w < NWS; ++w, ++wg) {
-                if (w % CS_W == 0) {
+            for (int w = w0; w < w1; ++w, ++wg) {
+                if ((w - w0) % CS_W == 0) {
                     // this stage opens a scale/bias chunk: its copies were issued a chunk earlier
                     ptx::cp_async_wait_all();
                     ptx::mbar_arrive(&s.sbar[unit & 1]);
@@ -719,14 +753,13 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                                     ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS, 7));
                     if (!ok) break;
                     sbslot = s.sb + (unit & 1) * 2 * 128 * SCP;
-                    const int c = w / CS_W;
-                    g_chunk0 = c * SCW;
+                    g_chunk0 = g_lo + ((w - w0) / CS_W) * SCW;
                     uint16_t* nslot = s.sb + ((unit + 1) & 1) * 2 * 128 * SCP;
-                    if (c + 1 < NCH) {
-                        issue_sb_chunk(p, ti, c + 1, nslot, tid);
-                    } else if (t + (int)gridDim.x < ntiles) {
-                        const TileInfo tn = tile_info(p, s, t + gridDim.x);
-                        issue_sb_chunk(p, tn, 0, nslot, tid);
+                    if (g_chunk0 + SCW < g_hi) {
+                        issue_sb_chunk(p, ti, g_chunk0 + SCW, g_hi, nslot, tid);
+                    } else if (t + tstep < ntiles) {
+                        const TileInfo tn = tile_info(p, s, t + tstep);
+                        issue_sb_chunk(p, tn, g_lo, g_hi, nslot, tid);
                     }
                     ptx::cp_async_commit();
                     ++unit;
@@ -748,7 +781,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                         const float bv = half_bits_to_float(sbslot[128 * SCP + row * SCP + gl], XT{});
                         const float bo = OFF == 0.0f ? bv : fmaf(-OFF, sv, bv);   // b - OFF*s
                         const float2 s2 = make_float2(sv, sv), b2 = make_float2(bo, bo);
-                        const float* xg = s.xtab + g * NT + th * H;
+                        const float* xg = s.xtab + (g - g_lo) * NT + th * H;
                         ptx::tc_wait_ld();
 #pragma unroll
                         for (int c = 0; c < H; c += 4) {
@@ -769,6 +802,40 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 AQ_TL(7, wg, threadIdx.x == 320);
             }
             if (!ok) break;
+            if (cs > 1) {
+                // ---- split K: rank r owns rows [r*RPR, (r+1)*RPR) of the tile.  Every rank pushes
+                //      its partial sums of each row into the owner's buffer (distributed shared
+                //      memory stores), then the owner adds the ranks' parts in rank order
+                //      (deterministic) and stores its rows.  One remote arrival per warp and owner:
+                //      the warp barrier orders every lane's stores before lane 0's release. ----
+                const int rpr = 128 / cs;
+                const int owner = row / rpr;
+                const uint32_t dst = ptx::mapa(
+                    ptx::smem_u32(s.red + ((size_t)rank * rpr + (row - owner * rpr)) * NT + th * H), (uint32_t)owner);
+#pragma unroll
+                for (int i = 0; i < H / 4; ++i)
+                    ptx::st_cluster_f4(dst + 16 * i, make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x,
+                                                                 acc[2 * i + 1].y));
+                __syncwarp();
+                if (lane == 0)
+                    for (int r = 0; r < cs; ++r) ptx::mbar_arrive_cluster(ptx::mapa(ptx::smem_u32(s.red_full), (uint32_t)r));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait_cluster(s.red_full, 0, s.abort, WAIT_NS));
+                if (!ok) break;
+                // this thread: elements [tid*F, tid*F + F) of the owned [rpr][NT] block
+                const int F = (128 * NT) / (cs * FOLD_THREADS);
+                for (int f = 0; f < F; ++f) {
+                    const int e = tid * F + f;
+                    float v = 0.0f;
+                    for (int r = 0; r < cs; ++r) v += s.red[(size_t)r * rpr * NT + e];
+                    const int rloc = rank * rpr + e / NT, tok = e % NT;
+                    if (rloc < ti.nvalid && tok < ti.tvalid) {
+                        int64_t off = (ti.xrow0 + tok) * p.y_row + ti.n0 + rloc;
+                        if (!p.offsets) off += (int64_t)ti.b0 * p.yb[0] + (int64_t)ti.b1 * p.yb[1];
+                        store_y(p.y, off, v, p.ydt, XT{});
+                    }
+                }
+                break;   // one tile per cluster
+            }
             // ---- this thread's row of y for its half of the tokens ----
             AQ_TSTART(t_store);
             if (row < ti.nvalid) {
@@ -828,8 +895,23 @@ cudaError_t launch_t(const Params& prm, int grid, size_t smem, cudaStream_t s) {
             done[dev] = true;
         }
     }
-    qmm_tc_kernel<BITS, XT, G><<<grid, THREADS, smem, s>>>(prm);
-    return cudaGetLastError();
+    // launched as a programmatic dependent of the previous kernel in the stream (see the kernel's
+    // prologue for what it does before the previous grid completes)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)prm.ksplit;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, qmm_tc_kernel<BITS, XT, G>, prm);
 }
 
 template <int BITS, typename XT>
