@@ -176,7 +176,135 @@ bool mma_supported(const MmaProblem& p, const char** why) {
     return true;
 }
 
+namespace {
+
+CUtensorMapSwizzle swizzle_for(int rowb) {
+    switch (rowb) {
+        case 128: return CU_TENSOR_MAP_SWIZZLE_128B;
+        case 64: return CU_TENSOR_MAP_SWIZZLE_64B;
+        case 32: return CU_TENSOR_MAP_SWIZZLE_32B;
+        default: return CU_TENSOR_MAP_SWIZZLE_NONE;
+    }
+}
+
+// x viewed as {K, rows, nb1, nb0} bf16/f16 bits, box {64 codes, `box_rows` tokens}, 128-byte swizzle
+CUresult encode_x(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap* m, const MmaProblem& pb, int box_rows) {
+    const int64_t rows_total = pb.M;
+    cuuint64_t dims[4] = {(cuuint64_t)pb.K, (cuuint64_t)rows_total, (cuuint64_t)pb.nb[1], (cuuint64_t)pb.nb[0]};
+    const int64_t rowb = rows_total > 1 ? pb.x_row * 2 : (pb.K * 2 + 15) / 16 * 16;
+    const int64_t s1 = pb.nb[1] > 1 ? pb.xb[1] * 2 : rowb * rows_total;
+    const int64_t s2 = pb.nb[0] > 1 ? pb.xb[0] * 2 : s1 * (int64_t)pb.nb[1];
+    cuuint64_t strides[3] = {(cuuint64_t)rowb, (cuuint64_t)((s1 + 15) / 16 * 16), (cuuint64_t)((s2 + 15) / 16 * 16)};
+    cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(pb.x), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+// W viewed as {K*bits/32 words, rows}, box {rowb/4 words, 128 rows}
+CUresult encode_w(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap* m, const MmaProblem& pb, int rowb) {
+    const int64_t wrows = pb.offsets ? pb.N * pb.n_experts : pb.N;
+    cuuint64_t dims[2] = {(cuuint64_t)(pb.K * pb.bits / 32), (cuuint64_t)wrows};
+    cuuint64_t strides[1] = {(cuuint64_t)(pb.w_row * 4)};
+    cuuint32_t box[2] = {(cuuint32_t)(rowb / 4), 128};
+    cuuint32_t estr[2] = {1, 1};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(pb.wq), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(rowb), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+void fill_common(Params& prm, const MmaProblem& pb) {
+    prm.x = pb.x;
+    prm.y = pb.y;
+    prm.scales = (const uint16_t*)pb.scales;
+    prm.biases = (const uint16_t*)pb.biases;
+    prm.M = pb.M;
+    prm.N = pb.N;
+    prm.K = pb.K;
+    prm.x_row = pb.x_row;
+    prm.y_row = pb.y_row;
+    prm.xb[0] = pb.xb[0];
+    prm.xb[1] = pb.xb[1];
+    prm.yb[0] = pb.yb[0];
+    prm.yb[1] = pb.yb[1];
+    prm.nb1 = pb.nb[1];
+    prm.n_wtiles = (int)((pb.N + 127) / 128);
+    prm.nbatch = (int)(pb.nb[0] * pb.nb[1]);
+    prm.kg = (int)(pb.K / pb.group);
+    prm.ydt = (int)pb.ydt;
+    prm.offsets = pb.offsets;
+    prm.n_experts = pb.n_experts;
+    prm.ksplit = 1;
+}
+
+cudaError_t device_pointers(Params& prm) {
+    static void* cache[64] = {nullptr};
+    void* a = nullptr;
+    cudaError_t e = symbol_address(g_device_error, cache, &a);
+    if (e != cudaSuccess) return e;
+    prm.err = static_cast<int*>(a);
+#if defined(AQ_TRACE) || defined(AQ_TIMELINE)
+    static void* cache_t[64] = {nullptr};
+    static void* cache_l[64] = {nullptr};
+    e = symbol_address(g_trace, cache_t, &a);
+    if (e != cudaSuccess) return e;
+    prm.trace = static_cast<unsigned long long*>(a);
+    e = symbol_address(g_timeline, cache_l, &a);
+    if (e != cudaSuccess) return e;
+    prm.tl = static_cast<long long*>(a);
+#endif
+    return cudaSuccess;
+}
+
+// Prefill: 128 W rows x 128 tokens per tile, one group per W stage (groups of 64 or 128)
+bool prefill_eligible(const MmaProblem& pb) {
+    return !pb.offsets && pb.M >= 64 && (pb.group == 64 || pb.group == 128);
+}
+
+cudaError_t launch_prefill_problem(const MmaProblem& pb, cudaStream_t stream) {
+    auto encode = get_encode();
+    if (!encode) return cudaErrorNotSupported;
+    using namespace pf;
+    Params prm;
+    memset(&prm, 0, sizeof prm);
+    const int sub = pb.group / KB;
+    const int rowb = pb.group * pb.bits / 8;
+    const size_t xstage = (size_t)sub * NTP * 128, wstage = (size_t)128 * rowb;
+    const int xst = sub == 1 ? 4 : 3;
+    const size_t fixed = (size_t)xst * xstage + p_fixed_bytes();
+    if (fixed + 4 * wstage > SMEM_LIMIT) return cudaErrorInvalidValue;
+    int stages = (int)((SMEM_LIMIT - fixed) / wstage);
+    if (stages > P_MAX_STAGES) stages = P_MAX_STAGES;
+    if (encode_x(encode, &prm.tx, pb, NTP) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    if (encode_w(encode, &prm.tw, pb, rowb) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    fill_common(prm, pb);
+    prm.n_ttiles = (int)((pb.M + NTP - 1) / NTP);
+    prm.n_wstages = (int)(pb.K / pb.group);
+    prm.stages = stages;
+    prm.xst = xst;
+    prm.tmem_cols = 512;   // [A block 0 | A block 1 | 2 accumulators of 128 columns]
+    prm.idesc = ptx::idesc_f16(NTP, pb.xdt == DT::BF16 ? 1 : 0);
+    cudaError_t e = device_pointers(prm);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = (int64_t)prm.n_wtiles * prm.n_ttiles * prm.nbatch;
+    const int sms = num_sms();
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    const size_t smem = fixed + (size_t)stages * wstage;
+    const bool bf = pb.xdt == DT::BF16;
+    switch (pb.bits) {
+        case 2: return launch_prefill<2>(bf, pb.group, prm, grid, smem, stream);
+        case 4: return launch_prefill<4>(bf, pb.group, prm, grid, smem, stream);
+        case 6: return launch_prefill<6>(bf, pb.group, prm, grid, smem, stream);
+        case 8: return launch_prefill<8>(bf, pb.group, prm, grid, smem, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
 cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
+    if (prefill_eligible(pb)) return launch_prefill_problem(pb, stream);
     auto encode = get_encode();
     if (!encode) return cudaErrorNotSupported;
     Params prm;
@@ -193,52 +321,10 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     const XPlan xp = pick_x(pb, kg, ms, split, geo);
     const int stages = xp.stages;
     if (stages < MIN_STAGES) return cudaErrorInvalidValue;
-    const int64_t rows_total = pb.M;
-    // ---- x tensor map: {K, rows, nb1, nb0}
-    {
-        cuuint64_t dims[4] = {(cuuint64_t)pb.K, (cuuint64_t)rows_total, (cuuint64_t)pb.nb[1], (cuuint64_t)pb.nb[0]};
-        const int64_t rowb = rows_total > 1 ? pb.x_row * 2 : (pb.K * 2 + 15) / 16 * 16;
-        const int64_t s1 = pb.nb[1] > 1 ? pb.xb[1] * 2 : rowb * rows_total;
-        const int64_t s2 = pb.nb[0] > 1 ? pb.xb[0] * 2 : s1 * (int64_t)pb.nb[1];
-        cuuint64_t strides[3] = {(cuuint64_t)rowb, (cuuint64_t)((s1 + 15) / 16 * 16), (cuuint64_t)((s2 + 15) / 16 * 16)};
-        cuuint32_t box[4] = {64, (cuuint32_t)NT, 1, 1};
-        cuuint32_t estr[4] = {1, 1, 1, 1};
-        CUresult r = encode(&prm.tx, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(pb.x), dims, strides, box,
-                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    }
-    // ---- W tensor map: {K*bits/32 words, rows}, box {rowb/4 words, 128 rows}
-    {
-        const int64_t wrows = pb.offsets ? pb.N * pb.n_experts : pb.N;
-        cuuint64_t dims[2] = {(cuuint64_t)(pb.K * bits / 32), (cuuint64_t)wrows};
-        cuuint64_t strides[1] = {(cuuint64_t)(pb.w_row * 4)};
-        cuuint32_t box[2] = {(cuuint32_t)(geo.rowb / 4), 128};
-        cuuint32_t estr[2] = {1, 1};
-        CUresult r = encode(&prm.tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(pb.wq), dims, strides,
-                            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, geo.tma_swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    }
-    prm.x = pb.x;
-    prm.y = pb.y;
-    prm.scales = (const uint16_t*)pb.scales;
-    prm.biases = (const uint16_t*)pb.biases;
-    prm.M = pb.M;
-    prm.N = pb.N;
-    prm.K = pb.K;
-    prm.x_row = pb.x_row;
-    prm.y_row = pb.y_row;
-    prm.xb[0] = pb.xb[0];
-    prm.xb[1] = pb.xb[1];
-    prm.yb[0] = pb.yb[0];
-    prm.yb[1] = pb.yb[1];
-    prm.nb1 = pb.nb[1];
-    prm.n_wtiles = (int)((pb.N + 127) / 128);
+    if (encode_x(encode, &prm.tx, pb, NT) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    if (encode_w(encode, &prm.tw, pb, geo.rowb) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    fill_common(prm, pb);
     prm.n_ttiles = (int)((pb.M + NT - 1) / NT);
-    prm.nbatch = (int)(pb.nb[0] * pb.nb[1]);
-    prm.kg = (int)kg;
-    prm.ydt = (int)pb.ydt;
     prm.n_wstages = nws;
     prm.ksplit = split;
     prm.stages = stages;
@@ -249,28 +335,10 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     while (pw < cols) pw <<= 1;
     prm.tmem_cols = pw;
     prm.idesc = ptx::idesc_f16(NT, pb.xdt == DT::BF16 ? 1 : 0);
-    prm.offsets = pb.offsets;
-    prm.n_experts = pb.n_experts;
     {
-        static void* cache[64] = {nullptr};
-        void* a = nullptr;
-        cudaError_t e = symbol_address(g_device_error, cache, &a);
+        cudaError_t e = device_pointers(prm);
         if (e != cudaSuccess) return e;
-        prm.err = static_cast<int*>(a);
     }
-#if defined(AQ_TRACE) || defined(AQ_TIMELINE)
-    {
-        static void* cache_t[64] = {nullptr};
-        static void* cache_l[64] = {nullptr};
-        void* a = nullptr;
-        cudaError_t e = symbol_address(g_trace, cache_t, &a);
-        if (e != cudaSuccess) return e;
-        prm.trace = static_cast<unsigned long long*>(a);
-        e = symbol_address(g_timeline, cache_l, &a);
-        if (e != cudaSuccess) return e;
-        prm.tl = static_cast<long long*>(a);
-    }
-#endif
 
     int grid;
     if (pb.offsets) grid = sms;

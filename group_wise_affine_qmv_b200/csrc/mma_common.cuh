@@ -100,7 +100,30 @@ __host__ __device__ constexpr size_t smem_fixed_bytes() {
            + 2 * 1024;                                           // alignment
 }
 
-// defined in mma_kernel.cuh, instantiated in kernels_mma_b<BITS>.cu
+// ---- prefill kernel (mma_prefill.cuh): tiles of 128 W rows x 128 tokens, one group per stage
+namespace pf {
+constexpr int NTP = 128;                                  // tokens per tile
+constexpr int P_EXP = 4;                                  // warps 2..5: code expanders
+constexpr int P_FOLD = 8;                                 // warps 6..13: folds
+constexpr int P_FOLD_THREADS = 32 * P_FOLD;
+constexpr int P_XPROD = 2 + P_EXP + P_FOLD;               // warp 14: x producer
+constexpr int P_THREADS = 32 * (P_XPROD + 1);             // 480
+constexpr int P_MAX_STAGES = 12;
+constexpr int P_MAX_XST = 4;
+// scale/bias slots, the two sums-of-x rows, mbarriers, TMEM base, abort flag, alignment
+__host__ __device__ constexpr size_t p_fixed_bytes() {
+    return 2 * 2 * 128 * SCP * 2 + 2 * NTP * 4 + (2 * P_MAX_STAGES + 2 * P_MAX_XST + 2 * 5 + 1) * 8 + 8 + 2 * 1024;
+}
+}  // namespace pf
+
+// defined in mma_kernel.cuh / mma_prefill.cuh, instantiated in kernels_mma_b<BITS>.cu
+template <int BITS>
+cudaError_t launch_prefill(bool bf16, int group, const Params& prm, int grid, size_t smem, cudaStream_t stream);
+extern template cudaError_t launch_prefill<2>(bool, int, const Params&, int, size_t, cudaStream_t);
+extern template cudaError_t launch_prefill<4>(bool, int, const Params&, int, size_t, cudaStream_t);
+extern template cudaError_t launch_prefill<6>(bool, int, const Params&, int, size_t, cudaStream_t);
+extern template cudaError_t launch_prefill<8>(bool, int, const Params&, int, size_t, cudaStream_t);
+
 template <int BITS>
 cudaError_t launch(bool bf16, int group, const Params& prm, int grid, size_t smem, cudaStream_t stream);
 extern template cudaError_t launch<2>(bool, int, const Params&, int, size_t, cudaStream_t);

@@ -1,0 +1,94 @@
+"""GPU parity of the prefill tensor-core kernel (rows per launch >= 64, groups 64/128:
+tiles of 128 W rows x 128 tokens) against the oracle.
+
+Several token tiles with a ragged tail, ragged W rows, K from one stage to two scale/bias
+chunks, every supported bit width, both activation dtypes, fp32 outputs, batched and strided
+views, and the prefill shapes of the decoder MLP at full size on sampled rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from group_wise_affine_qmv_b200 import aq, inputs
+from tests.parity import dtype_name, oracle_linear_view, row_errors, to_device_quant
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+DEV = "cuda"
+
+
+def _q(w, group, bits, sdtype="bf16"):
+    Q = oracle.quantize(w.float().numpy(), group, bits, sdtype)
+    tdt = torch.bfloat16 if sdtype == "bf16" else torch.float16
+    return Q, to_device_quant(Q, DEV, tdt)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 6, 8])
+@pytest.mark.parametrize("group", [64, 128])
+@pytest.mark.parametrize("M,N,K", [(64, 128, 256), (130, 300, 512), (257, 200, 4096)])
+def test_prefill_shapes(bits, group, M, N, K):
+    w = inputs.normal((N, K), 0.02, seed=M + N + K + bits + group)
+    Q, (wq, sc, bi) = _q(w, group, bits)
+    x = inputs.normal((M, K), 1.0, torch.bfloat16, seed=M * 3 + K)
+    xd = x.to(DEV)
+    y = aq.aq_qmm_t(xd, wq, sc, bi, group, bits)
+    err = row_errors(y, oracle_linear_view(x, Q.dequant()))
+    assert np.all(err <= 4e-3), (err.max(), int(err.argmax()))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("xdtype", [torch.bfloat16, torch.float16])
+def test_prefill_dtypes_fp32_out(bits, xdtype):
+    M, N, K, group = 200, 260, 2048, 64
+    sd = dtype_name(torch.empty(0, dtype=xdtype))
+    w = inputs.normal((N, K), 0.02, seed=bits + 7)
+    Q, (wq, sc, bi) = _q(w, group, bits, sd)
+    x = inputs.normal((M, K), 1.0, xdtype, seed=bits + 8)
+    xd = x.to(DEV)
+    ref = oracle_linear_view(x, Q.dequant())
+    y = aq.aq_qmm_t(xd, wq, sc, bi, group, bits)
+    assert np.all(row_errors(y, ref) <= 4e-3)
+    # fp32 output: only fp32 summation order remains
+    y32 = aq.aq_qmm_t(xd, wq, sc, bi, group, bits, out_dtype=torch.float32)
+    assert np.all(row_errors(y32, ref) <= 1e-4)
+
+
+def test_prefill_batched_views():
+    """Non-foldable batch dims with >= 64 rows each: every batch element matches the contiguous
+    copy bit for bit and the oracle to the bar."""
+    K, N, bits, group = 1024, 300, 4, 64
+    w = inputs.normal((N, K), 0.02, seed=51)
+    Q, (wq, sc, bi) = _q(w, group, bits)
+    base = inputs.normal((3, 2, 100, K), 1.0, torch.bfloat16, seed=52)
+    x = base.narrow(2, 10, 70)                     # [3, 2, 70, K]: rows do not fold across batches
+    xd = base.to(DEV).narrow(2, 10, 70)
+    y = aq.aq_qmm_t(xd, wq, sc, bi, group, bits)
+    yc = aq.aq_qmm_t(xd.contiguous(), wq, sc, bi, group, bits)
+    assert torch.equal(y, yc)
+    assert np.all(row_errors(y, oracle_linear_view(x, Q.dequant())) <= 4e-3)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("shape", ["up", "down"])
+def test_prefill_full_size_sampled(bits, shape):
+    """x [8, 2048, K] against the decoder MLP's W [14336, 4096] (up) or [4096, 14336] (down) at
+    full size, in one launch; the oracle checks sampled rows of x against every column."""
+    if shape == "up":
+        xs, (N, K) = inputs.PREFILL_X, inputs.PREFILL_W_UP
+    else:
+        xs, (N, K) = inputs.PREFILL_X_DOWN, inputs.PREFILL_W_DOWN
+    group = inputs.PREFILL_GROUP
+    w = inputs.normal((N, K), 0.02, seed=61 + bits)
+    Q, (wq, sc, bi) = _q(w, group, bits)
+    del w
+    xd = inputs.normal(xs, 1.0, torch.bfloat16, seed=62, device=DEV)
+    y = aq.aq_qmm_t(xd, wq, sc, bi, group, bits)
+    torch.cuda.synchronize()
+    rows = [(0, 0), (0, 2047), (3, 129), (5, 1000), (7, 2047), (7, 77)]
+    wd = Q.dequant()
+    xb = torch.stack([xd[b, t] for b, t in rows]).cpu()
+    ref = oracle.linear_contig(xb.view(torch.int16).numpy().view(np.uint16), "bf16", wd)
+    got = torch.stack([y[b, t] for b, t in rows])
+    assert np.all(row_errors(got, ref) <= 4e-3)
