@@ -59,6 +59,84 @@ def sweep_bytes(layers):
     return tot
 
 
+def bench_config(layers, world):
+    """The workload this benchmark's lines are quoted on (both arms)."""
+    return {"workload": "decode sweep: 28 layers x (q,k,v,o,gate,up,down) + lm_head, x [32,1,K] bf16, "
+                        "bits 4 and 8, G=64",
+            "tokens": inputs.DECODE_BATCH, "layers": layers, "bits": list(BITS_LIST), "group": GROUP,
+            "bytes_per_step": sweep_bytes(layers),
+            "l2": "inputs larger than L2 (weights streamed from HBM each step)",
+            "graph": "one CUDA graph per step", "parallelism": f"replicas x{world}"}
+
+
+def bf16_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (burst)"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def time_calls(fn, reps, stream):
+    """Average device time (ms) of `fn` over `reps` calls on `stream` (CUDA events)."""
+    with torch.cuda.stream(stream):
+        fn()
+        fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def prefill_and_moe(device, stream):
+    """Config 5: the decoder MLP's prefill shapes (x [8,2048,K] bf16, W 4- and 8-bit, G=64) and
+    the mixture-of-experts bank (128 experts [2816, 1408], 8-bit, G=32, 256 tokens routed top-8),
+    each call timed alone with CUDA events; inputs synthetic and generated on the device."""
+    from group_wise_affine_qmv_b200 import aq
+    peak, peak_kind = bf16_peak()
+    out = {"peak_tflops": peak, "peak_source": peak_kind}
+    for tag, xs, (N, K) in (("up", inputs.PREFILL_X, inputs.PREFILL_W_UP),
+                            ("down", inputs.PREFILL_X_DOWN, inputs.PREFILL_W_DOWN)):
+        x = inputs.normal(xs, 1.0, torch.bfloat16, seed=5, device=device)
+        M = xs[0] * xs[1]
+        for bits in BITS_LIST:
+            w = inputs.normal((N, K), inputs.W_STD, seed=6 + bits, device=device)
+            wq, sc, bi = aq.aq_quantize(w, inputs.PREFILL_GROUP, bits, scale_dtype=torch.bfloat16)
+            del w
+            y = torch.empty(xs[:-1] + (N,), dtype=torch.bfloat16, device=device)
+            ms = time_calls(lambda: aq.aq_qmm_t(x, wq, sc, bi, inputs.PREFILL_GROUP, bits, out=y), 5, stream)
+            tf = 2.0 * M * N * K / ms / 1e9
+            out[f"{tag}_w{bits}"] = {"x": list(xs), "W": [N, K], "ms": round(ms, 3), "TFLOPs": round(tf, 1),
+                                    "frac_of_peak": round(tf / peak, 4)}
+            del wq, sc, bi, y
+        del x
+    # expert bank
+    E, N, K, G, bits = inputs.MOE_EXPERTS, inputs.MOE_N, inputs.MOE_K, inputs.MOE_GROUP, inputs.MOE_BITS
+    wq = torch.empty(E, N, K * bits // 32, dtype=torch.int32, device=device)
+    sc = torch.empty(E, N, K // G, dtype=torch.bfloat16, device=device)
+    bi = torch.empty_like(sc)
+    for e in range(E):
+        w = inputs.normal((N, K), inputs.W_STD, seed=100 + e, device=device)
+        q = aq.aq_quantize(w, G, bits, scale_dtype=torch.bfloat16)
+        wq[e].copy_(q[0]); sc[e].copy_(q[1]); bi[e].copy_(q[2])
+    tok, offsets = inputs.moe_sort(inputs.moe_routing())
+    x_tok = inputs.normal((inputs.MOE_TOKENS, K), 1.0, torch.bfloat16, seed=9, device=device)
+    x_sorted = x_tok[tok.to(device)].contiguous()
+    off_d = offsets.to(device)
+    y = torch.empty(x_sorted.shape[0], N, dtype=torch.bfloat16, device=device)
+    ms = time_calls(lambda: aq.aq_qmm_t_grouped(x_sorted, off_d, wq, sc, bi, G, bits, out=y), 10, stream)
+    moe_bytes = E * N * (K * bits // 8 + 4 * (K // G)) + 2 * x_sorted.numel() + 2 * y.numel()
+    hbm, _ = hbm_peak()
+    out["moe_w8_g32"] = {"experts": E, "W": [N, K], "rows": int(x_sorted.shape[0]), "us": round(ms * 1e3, 2),
+                         "GBps": round(moe_bytes / ms / 1e6, 1), "frac_of_hbm_peak": round(moe_bytes / ms / 1e6 / hbm, 4)}
+    del wq, sc, bi, x_sorted, y
+    return out
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region (NVML, else nvidia-smi)
 # ---------------------------------------------------------------------------
@@ -381,11 +459,7 @@ def ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.02) weights quantized on the device, N(0,1) activations)",
-        "config": {"workload": "decode sweep: 28 layers x (q,k,v,o,gate,up,down) + lm_head, x [32,1,K] bf16, "
-                               "bits 4 and 8, G=64",
-                   "tokens": inputs.DECODE_BATCH, "layers": layers, "bits": list(BITS_LIST), "group": GROUP,
-                   "bytes_per_step": step_bytes, "l2": "inputs larger than L2 (weights streamed from HBM each step)",
-                   "graph": "one CUDA graph per step", "parallelism": f"replicas x{world}"},
+        "config": bench_config(layers, world),
         "detail": detail,
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -394,6 +468,8 @@ def ours(args):
                      "kernel": "aq_qmm_t (all launches of the step)", "peak_source": peak_kind},
         "clocks": clk.summary(),
     }
+    if not args.no_prefill:
+        result["detail"]["prefill"] = prefill_and_moe(device, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(layers)
     if rank == 0:
@@ -450,11 +526,43 @@ def reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": "decode sweep row sample (CPU oracle)", "layers": layers},
+        "data": "synthetic", "config": bench_config(layers, 1),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
+
+
+CASES = ("lm_head_w4", "lm_head_w8", "lm_head2x_w4", "prefill_w4", "prefill_w8")
+
+
+def single_case(name, reps):
+    """One shape alone, for profiling: `reps` timed calls after two warm-up calls (CUDA events).
+    lm_head*: x [32, 1, 1024] against W [151936, 1024] (2x: 303872 rows, > L2); prefill*: x
+    [2, 2048, 4096] against W [14336, 4096]; G = 64, weights quantized on the device."""
+    from group_wise_affine_qmv_b200 import aq
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    bits = int(name[-1])
+    if name.startswith("lm_head"):
+        K, N = 1024, inputs.LM_HEAD[2] * (2 if name.startswith("lm_head2x") else 1)
+        x = inputs.decode_x(K, device=device)
+        y = torch.empty(inputs.DECODE_BATCH, 1, N, dtype=torch.bfloat16, device=device)
+        M = inputs.DECODE_BATCH
+    else:
+        K, N = inputs.PREFILL_W_UP[1], inputs.PREFILL_W_UP[0]
+        x = inputs.normal((2, 2048, K), 1.0, torch.bfloat16, seed=5, device=device)
+        y = torch.empty(2, 2048, N, dtype=torch.bfloat16, device=device)
+        M = 2 * 2048
+    w = inputs.normal((N, K), inputs.W_STD, seed=6, device=device)
+    wq, sc, bi = aq.aq_quantize(w, GROUP, bits, scale_dtype=torch.bfloat16)
+    del w
+    ms = time_calls(lambda: aq.aq_qmm_t(x, wq, sc, bi, GROUP, bits, out=y), reps, torch.cuda.current_stream())
+    aq.aq_device_error()
+    nbytes = matrix_bytes(K, N, bits, M)
+    print(json.dumps({"case": name, "M": M, "N": N, "K": K, "bits": bits, "us": round(ms * 1e3, 2),
+                      "GBps": round(nbytes / ms / 1e6, 1), "TFLOPs": round(2.0 * M * N * K / ms / 1e9, 1)}),
+          flush=True)
 
 
 def main():
@@ -465,7 +573,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=inputs.DECODE_LAYERS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill / expert-bank detail")
+    ap.add_argument("--case", choices=CASES, help="time one shape alone (profiling) instead of the benchmark")
+    ap.add_argument("--reps", type=int, default=3, help="timed calls of --case")
     args = ap.parse_args()
+    if args.case:
+        single_case(args.case, args.reps)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -316,7 +316,10 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     const int gps = geo.wsc / pb.group;
     const int sms = num_sms();
     const int64_t tiles = pb.offsets ? 0 : ((pb.N + 127) / 128) * ((pb.M + NT - 1) / NT) * pb.nb[0] * pb.nb[1];
-    const int split = pb.offsets ? 1 : pick_split(tiles, nws, gps, sms);
+    // The split depends on the total rows, not on how they are grouped into launch batches, so
+    // that a strided view and its contiguous copy take the same split (and give the same bits).
+    const int64_t rows_all = pb.M * pb.nb[0] * pb.nb[1];
+    const int split = pb.offsets ? 1 : pick_split(((pb.N + 127) / 128) * ((rows_all + NT - 1) / NT), nws, gps, sms);
     const int ms = split > 1 ? split_max_stages(nws, gps, split) : nws;
     const XPlan xp = pick_x(pb, kg, ms, split, geo);
     const int stages = xp.stages;
