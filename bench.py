@@ -415,6 +415,28 @@ def ours(args):
                               "lm_head_us": round(lm_us, 2), "lm_head_GBps": round(lm_bytes / lm_us / 1e3, 1),
                               "lm_head_frac_of_peak": None}
         del g_layers, glm
+        # per projection: the 28 layers' calls of one projection in a graph, per call
+        per = {}
+        for proj in ("q", "k", "gate", "down"):
+            calls = [(m, y) for m, y in zip(mats[bits][:-1], ys[bits][:-1]) if m[0].split(".")[-1] == proj]
+            gp = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gp, stream=stream):
+                for (name, K, N, wq, sc, bi), y in calls:
+                    aq.aq_qmm_t(xs[K], wq, sc, bi, GROUP, bits, out=y)
+            with torch.cuda.stream(stream):
+                gp.replay()
+                p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                p0.record(stream)
+                for _ in range(10):
+                    gp.replay()
+                p1.record(stream)
+            p1.synchronize()
+            us = p0.elapsed_time(p1) / 10 / len(calls) * 1e3
+            K, N = calls[0][0][1], calls[0][0][2]
+            per[proj] = {"K": K, "N": N, "us": round(us, 2), "GBps": round(matrix_bytes(K, N, bits) / us / 1e3, 1)}
+            del gp
+        per["note"] = "28 calls of one projection per graph replay; their weights may stay in L2 between replays"
+        detail[f"w{bits}"]["per_projection"] = per
 
     # ---- end-to-end: activations H2D, graph, logits D2H, per step ----
     x_host = {K: xs[K].cpu().pin_memory() for K in xs}
