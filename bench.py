@@ -92,6 +92,51 @@ def time_calls(fn, reps, stream):
     return e0.elapsed_time(e1) / reps
 
 
+def time_graphed(fn, calls, stream):
+    """Average device time (ms) per call of `fn`, `calls` calls captured in one CUDA graph
+    (host launch overhead excluded), over 10 replays."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        fn()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(calls):
+            fn()
+    ms = time_calls(g.replay, 10, stream)
+    del g
+    return ms / calls
+
+
+def probe_and_ragged(device, stream):
+    """Configs 1 and 3, each shape in a CUDA graph of 20 calls (launch-bound shapes, so
+    microseconds are the figure; the same weights every call, so they may sit in L2): the probe
+    (K 2048, N 1024, 4-bit G64, x [2,K], [2,1,K], [2,4,K]) and the ragged GEMV (K 4096,
+    N 1001 / 4099, bits 2/3/5/6, G 32/128, x [1,K] and [4,1,K])."""
+    from group_wise_affine_qmv_b200 import aq
+    hbm, _ = hbm_peak()
+    out = {}
+    w, xs = inputs.probe_case()
+    K, N = w.shape[1], w.shape[0]
+    wq, sc, bi = aq.aq_quantize(w.to(device), 64, 4, scale_dtype=torch.bfloat16)
+    for x in xs:
+        xd = x.to(device)
+        us = time_graphed(lambda: aq.aq_qmm_t(xd, wq, sc, bi, 64, 4), 20, stream) * 1e3
+        out["probe_x" + "x".join(str(d) for d in x.shape)] = {"us": round(us, 2)}
+    for bits in (2, 3, 5, 6):
+        for group in (32, 128):
+            for N in (1001, 4099):
+                w, _ = inputs.ragged_case(bits, group, N, (1, inputs.RAGGED_K))
+                wq, sc, bi = aq.aq_quantize(w.to(device), group, bits, scale_dtype=torch.bfloat16)
+                for shape in ((1, inputs.RAGGED_K), (4, 1, inputs.RAGGED_K)):
+                    x = inputs.normal(shape, 1.0, torch.bfloat16, seed=3, device=device)
+                    us = time_graphed(lambda: aq.aq_qmv(x, wq, sc, bi, group, bits), 20, stream) * 1e3
+                    M = 1 if len(shape) == 2 else 4
+                    nbytes = N * (inputs.RAGGED_K * bits // 8 + 4 * (inputs.RAGGED_K // group)) + 2 * M * (inputs.RAGGED_K + N)
+                    out[f"qmv_b{bits}_g{group}_n{N}_m{M}"] = {"us": round(us, 2), "GBps": round(nbytes / us / 1e3, 1),
+                                                            "frac_of_hbm_peak": round(nbytes / us / 1e3 / hbm, 4)}
+    return out
+
+
 def prefill_and_moe(device, stream):
     """Config 5: the decoder MLP's prefill shapes (x [8,2048,K] bf16, W 4- and 8-bit, G=64) and
     the mixture-of-experts bank (128 experts [2816, 1408], 8-bit, G=32, 256 tokens routed top-8),
@@ -492,6 +537,7 @@ def ours(args):
     }
     if not args.no_prefill:
         result["detail"]["prefill"] = prefill_and_moe(device, stream)
+        result["detail"]["probe_and_ragged_qmv"] = probe_and_ragged(device, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(layers)
     if rank == 0:

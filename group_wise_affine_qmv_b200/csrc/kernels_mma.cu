@@ -138,12 +138,14 @@ XPlan pick_x(const MmaProblem& p, int64_t kg, int ms, int split, const Geom& g) 
 
 // CTAs per cluster splitting each tile's K: when the tiles alone would leave most SMs idle,
 // the largest power of two <= 8 that keeps the grid within the SMs and gives every rank
-// at least one W stage (two when a stage holds one group)
+// at least one W stage (two when a stage holds one group).  Clusters of 8 only while the grid
+// stays within 64 CTAs: more of them than that could not all be placed at once next to the
+// tail of the previous kernel (a cluster needs its SMs free in one GPC).
 int pick_split(int64_t tiles, int nws, int gps, int sms) {
     const int u = gps == 1 ? 2 : 1;
     const int nu = (nws + u - 1) / u;
     int cs = 1;
-    while (cs < 8 && tiles * cs * 2 <= sms && cs * 2 <= nu) cs *= 2;
+    while (cs < 8 && tiles * cs * 2 <= sms && cs * 2 <= nu && (cs < 4 || tiles * cs * 2 <= 64)) cs *= 2;
     return cs;
 }
 
