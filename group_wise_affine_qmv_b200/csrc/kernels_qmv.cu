@@ -7,7 +7,8 @@
 // sum, so the bias term b * sum(x) is exact whenever the exact sum is
 // representable in fp32.
 //
-// Layout of the work: a warp owns RPW = 4 consecutive rows of W; lane l walks
+// Layout of the work: a warp owns RPW (4, or 1 when N is so small that 4 would leave most SMs
+// idle) consecutive rows of W; lane l walks
 // the 32-code chunks l, l+32, l+64, ... of those rows (a chunk is `bits`
 // consecutive uint32 words, read with the widest aligned vector load: 16-byte
 // for 4/8-bit, 8-byte for 2/6-bit, 4-byte for 3/5-bit), reuses each x chunk
@@ -34,7 +35,6 @@ namespace {
 
 constexpr int QMV_THREADS = 256;
 constexpr int QMV_WARPS = QMV_THREADS / 32;
-constexpr int RPW = 4;  // W rows per warp
 
 // 128 + q  (bits <= 7) or 256 + q (bits == 8), as fp32 bit patterns
 template <int BITS> struct Magic {
@@ -94,7 +94,7 @@ __device__ __forceinline__ void load_x8(const XT* p, int vec, float* f) {
 }
 
 // P[r][t] += (BASE + q[r][I0+J]) * x[t][J] for the 8 codes I0..I0+7 of every row r
-template <int BITS, int TOK, int I0, int... J>
+template <int BITS, int TOK, int RPW, int I0, int... J>
 __device__ __forceinline__ void fma_codes(const uint32_t (&wv)[RPW][BITS + 1], const float (&xf)[TOK][8],
                                           float (&P)[RPW][TOK], std::integer_sequence<int, J...>) {
 #pragma unroll
@@ -109,7 +109,7 @@ __device__ __forceinline__ void fma_codes(const uint32_t (&wv)[RPW][BITS + 1], c
     }
 }
 
-template <int BITS, int TOK, typename XT, typename YT>
+template <int BITS, int TOK, int RPW, typename XT, typename YT>
 __global__ void __launch_bounds__(QMV_THREADS) qmv_kernel(const __grid_constant__ QmvArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t n0 = ((int64_t)blockIdx.x * QMV_WARPS + warp) * RPW;
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(QMV_THREADS) qmv_kernel(const __grid_constant_
 #pragma unroll
                     for (int j = 0; j < 8; ++j) X[t] += xf[t][j];  // widened before summing
                 }
-                fma_codes<BITS, TOK, SUB * 8>(wv, xf, P, std::make_integer_sequence<int, 8>{});
+                fma_codes<BITS, TOK, RPW, SUB * 8>(wv, xf, P, std::make_integer_sequence<int, 8>{});
             };
             do_sub(std::integral_constant<int, 0>{});
             do_sub(std::integral_constant<int, 1>{});
@@ -205,19 +205,27 @@ __global__ void __launch_bounds__(QMV_THREADS) qmv_kernel(const __grid_constant_
     }
 }
 
-template <int BITS, int TOK, typename XT, typename YT>
+template <int BITS, int TOK, int RPW, typename XT, typename YT>
 cudaError_t launch_t(const QmvArgs& a, int64_t nbatch, cudaStream_t s) {
     const int64_t rows_per_cta = QMV_WARPS * RPW;
     const dim3 grid((unsigned)((a.N + rows_per_cta - 1) / rows_per_cta), (unsigned)nbatch);
-    qmv_kernel<BITS, TOK, XT, YT><<<grid, QMV_THREADS, 0, s>>>(a);
+    qmv_kernel<BITS, TOK, RPW, XT, YT><<<grid, QMV_THREADS, 0, s>>>(a);
     return cudaGetLastError();
+}
+
+// one W row per warp while 4 per warp would leave most SMs idle (under 64 CTAs); above that
+// the four rows' reuse of each x chunk matters more than the extra warps
+template <int BITS, int TOK, typename XT, typename YT>
+cudaError_t launch_rpw(const QmvArgs& a, int64_t nbatch, cudaStream_t s) {
+    if ((a.N + QMV_WARPS * 4 - 1) / (QMV_WARPS * 4) * nbatch < 64) return launch_t<BITS, TOK, 1, XT, YT>(a, nbatch, s);
+    return launch_t<BITS, TOK, 4, XT, YT>(a, nbatch, s);
 }
 
 template <int BITS, typename XT, typename YT>
 cudaError_t launch_tok(const QmvArgs& a, int64_t nbatch, cudaStream_t s) {
-    if (a.M == 1) return launch_t<BITS, 1, XT, YT>(a, nbatch, s);
-    if (a.M == 2) return launch_t<BITS, 2, XT, YT>(a, nbatch, s);
-    return launch_t<BITS, 4, XT, YT>(a, nbatch, s);
+    if (a.M == 1) return launch_rpw<BITS, 1, XT, YT>(a, nbatch, s);
+    if (a.M == 2) return launch_rpw<BITS, 2, XT, YT>(a, nbatch, s);
+    return launch_rpw<BITS, 4, XT, YT>(a, nbatch, s);
 }
 
 template <typename XT, typename YT>
