@@ -79,20 +79,13 @@ constexpr size_t SMEM_LIMIT = 227 * 1024;
 constexpr int MIN_STAGES = 3;
 
 struct Geom {
-    int wsc, rowb, sub;
-    CUtensorMapSwizzle tma_swz;
+    int wsc, rowb, sub;   // codes, bytes per W row and 64-code sub-steps of one W stage
 };
 Geom geometry(int bits, int group) {
     Geom g;
     g.wsc = stage_codes(bits, group);
     g.rowb = stage_rowb(bits, group);
     g.sub = g.wsc / KB;
-    switch (g.rowb) {
-        case 128: g.tma_swz = CU_TENSOR_MAP_SWIZZLE_128B; break;
-        case 64: g.tma_swz = CU_TENSOR_MAP_SWIZZLE_64B; break;
-        case 32: g.tma_swz = CU_TENSOR_MAP_SWIZZLE_32B; break;
-        default: g.tma_swz = CU_TENSOR_MAP_SWIZZLE_NONE; break;
-    }
     return g;
 }
 

@@ -95,7 +95,7 @@ constexpr int RED_BYTES = FOLD_THREADS * (NT / 2) * 4;  // one CTA's partial y t
 // shared memory besides the x buffer, the W ring and the sum-of-x table
 __host__ __device__ constexpr size_t smem_fixed_bytes() {
     return 2 * 2 * 128 * SCP * 2                                  // scale/bias chunk slots
-           + (2 * MAX_STAGES + 2 * MAX_XST + 2 * 4 + 5) * 8 + 8  // mbarriers, TMEM base, abort flag
+           + (2 * MAX_STAGES + 2 * MAX_XST + 2 * 4 + 4) * 8 + 8  // mbarriers, TMEM base, abort flag
            + (MAX_EXPERTS + 1) * 4                               // grouped tile prefix sums
            + 2 * 1024;                                           // alignment
 }

@@ -96,7 +96,6 @@ struct Smem {
     uint64_t* xres_full; // resident x landed
     uint64_t* mdone;     // teardown: all MMAs retired
     uint64_t* red_full;  // split K: every rank's part of this CTA's rows has arrived (fold warps)
-    uint64_t* red_done;  // (unused)
     uint32_t* tmem_base;
     int* abort;
     int* prefix;         // grouped: tile prefix sums [n_experts + 1]
@@ -136,8 +135,7 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const Params& p, int ms) {
     s.xres_full = s.xbar + 1;
     s.mdone = s.xres_full + 1;
     s.red_full = s.mdone + 1;
-    s.red_done = s.red_full + 1;
-    s.tmem_base = reinterpret_cast<uint32_t*>(s.red_done + 1);
+    s.tmem_base = reinterpret_cast<uint32_t*>(s.red_full + 1);
     s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
     s.prefix = s.abort + 1;
     return s;

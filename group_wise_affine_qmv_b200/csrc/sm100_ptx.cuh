@@ -196,14 +196,6 @@ __device__ __forceinline__ void st_cluster_f4(uint32_t cluster_addr, float4 v) {
                  "f"(v.w)
                  : "memory");
 }
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t cluster_addr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(cluster_addr)
-                 : "memory");
-    return v;
-}
 
 // programmatic dependent launch: let the next grid in the stream be scheduled / wait until
 // every prerequisite grid has completed and its memory operations are visible

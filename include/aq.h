@@ -120,9 +120,17 @@ aq_status aq_dequantize(const aq_view* wq, const aq_view* scales, const aq_view*
  * scales, biases: [..., N, K/group], same dtype as x, same batch dims as wq.
  * y:      x.shape[:-1] + [N], dtype of x or AQ_F32, must not overlap inputs.
  * bits in {2,3,4,5,6,8}; group in {32,64,128}; K % group == 0.
- * Rows per launch decide the kernel: a CUDA-core GEMV for a handful of rows,
- * a tcgen05/TMEM tensor-core kernel above that.  Data pointers must be
- * 16-byte aligned.
+ * Rows per launch batch decide the kernel: up to 4 rows (or a batched W), a
+ * CUDA-core GEMV; 5..63 rows, a tcgen05/TMEM tensor-core kernel on tiles of
+ * 128 W rows x 32 tokens (K split over the CTAs of a thread-block cluster
+ * when the tiles alone would leave most SMs idle); 64 rows and more with
+ * groups of 64/128, a tensor-core kernel on 128 x 128 tiles.  3/5-bit codes,
+ * K not a multiple of 64, an odd or very large K/group, or unaligned rows
+ * take the GEMV.
+ * Every kernel keeps W exact (integer codes, scale and bias in fp32).  The
+ * tensor-core kernels are launched as programmatic dependents of the previous
+ * kernel in the stream: only their set-up overlaps it; stream order is kept.
+ * Data pointers must be 16-byte aligned.
  */
 aq_status aq_qmm_t(const aq_view* x, const aq_view* wq, const aq_view* scales,
                    const aq_view* biases, int group, int bits, const aq_view* y, void* stream);
