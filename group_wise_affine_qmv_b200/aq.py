@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_PKG, "libaq.so")
 
 AQ_F32, AQ_BF16, AQ_F16, AQ_U32 = 0, 1, 2, 3
 AQ_REGIME_QMV, AQ_REGIME_MMA = 0, 1
+KERNEL_NAMES = {0: "gemv", 1: "warp_mma", 2: "tc_small_m", 3: "tc_prefill"}
 
 _DT = {torch.float32: AQ_F32, torch.bfloat16: AQ_BF16, torch.float16: AQ_F16, torch.int32: AQ_U32,
        torch.uint32: AQ_U32}
@@ -42,7 +43,7 @@ class AqView(ctypes.Structure):
 class AqPlan(ctypes.Structure):
     _fields_ = [("regime", ctypes.c_int32), ("w_batched", ctypes.c_int32), ("M", ctypes.c_int64),
                 ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("nbatch_dims", ctypes.c_int32),
-                ("pad_", ctypes.c_int32), ("batch_shape", ctypes.c_int64 * 2),
+                ("kernel", ctypes.c_int32), ("batch_shape", ctypes.c_int64 * 2),
                 ("x_batch_stride", ctypes.c_int64 * 2), ("y_batch_stride", ctypes.c_int64 * 2),
                 ("w_batch_stride", ctypes.c_int64 * 2), ("s_batch_stride", ctypes.c_int64 * 2),
                 ("b_batch_stride", ctypes.c_int64 * 2), ("x_row_stride", ctypes.c_int64),
@@ -193,7 +194,8 @@ def aq_plan_linear(x, wq, scales, biases, group: int, bits: int, y, force_qmv: b
     _check(lib, lib.aq_plan_linear(view(x), view(wq), view(scales), view(biases), group, bits, view(y),
                                    1 if force_qmv else 0, ctypes.byref(p)))
     note = lib.aq_last_error_message().decode()
-    return dict(regime="mma" if p.regime == AQ_REGIME_MMA else "qmv", w_batched=bool(p.w_batched), M=p.M, N=p.N,
+    return dict(regime="mma" if p.regime == AQ_REGIME_MMA else "qmv", kernel=KERNEL_NAMES[p.kernel],
+                w_batched=bool(p.w_batched), M=p.M, N=p.N,
                 K=p.K, nbatch_dims=p.nbatch_dims, batch_shape=tuple(p.batch_shape),
                 x_batch_stride=tuple(p.x_batch_stride), y_batch_stride=tuple(p.y_batch_stride),
                 w_batch_stride=tuple(p.w_batch_stride), x_row_stride=p.x_row_stride, y_row_stride=p.y_row_stride,

@@ -303,6 +303,7 @@ aq_status resolve_linear(const aq_view* x, const aq_view* wq, const aq_view* sc,
         }
     }
     P.regime = R->mma_ok ? AQ_REGIME_MMA : AQ_REGIME_QMV;
+    P.kernel = R->mma_ok ? (int32_t)aq::mma_kernel_for(R->mp) : AQ_KERNEL_GEMV;
     return AQ_OK;
 }
 

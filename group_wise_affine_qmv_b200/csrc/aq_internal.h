@@ -75,6 +75,16 @@ struct MmaProblem {
 bool mma_supported(const MmaProblem& p, const char** why);
 cudaError_t launch_mma(const MmaProblem& p, cudaStream_t s);
 
+// Which tensor-core kernel launch_mma runs for a supported problem.
+enum class MmaKernel : int { WARP = AQ_KERNEL_WARP_MMA, SMALL_M = AQ_KERNEL_TC_SMALL_M, PREFILL = AQ_KERNEL_TC_PREFILL };
+MmaKernel mma_kernel_for(const MmaProblem& p);
+
+// Warp-level (mma.sync) kernel for up to 32 rows per launch batch: whether it takes the problem
+// (given that mma_supported accepted it) and its launch.
+bool warp_mma_supported(const MmaProblem& p);
+bool warp_mma_preferred(const MmaProblem& p);
+cudaError_t launch_warp_mma(const MmaProblem& p, cudaStream_t s);
+
 // Device-side error word (set by kernels whose bounded waits expire).
 cudaError_t read_and_clear_device_error(int* value, cudaStream_t s);
 

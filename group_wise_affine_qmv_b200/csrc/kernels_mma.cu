@@ -298,8 +298,16 @@ cudaError_t launch_prefill_problem(const MmaProblem& pb, cudaStream_t stream) {
 
 }  // namespace
 
+MmaKernel mma_kernel_for(const MmaProblem& pb) {
+    if (prefill_eligible(pb)) return MmaKernel::PREFILL;
+    if (warp_mma_supported(pb) && warp_mma_preferred(pb)) return MmaKernel::WARP;
+    return MmaKernel::SMALL_M;
+}
+
 cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
-    if (prefill_eligible(pb)) return launch_prefill_problem(pb, stream);
+    const MmaKernel kind = mma_kernel_for(pb);
+    if (kind == MmaKernel::PREFILL) return launch_prefill_problem(pb, stream);
+    if (kind == MmaKernel::WARP) return launch_warp_mma(pb, stream);
     auto encode = get_encode();
     if (!encode) return cudaErrorNotSupported;
     Params prm;

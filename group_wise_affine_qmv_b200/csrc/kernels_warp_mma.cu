@@ -1,0 +1,149 @@
+// kernels_warp_mma.cu -- host side of the warp-level tensor-core kernel (warp_mma_kernel.cuh):
+// which problems it takes and how a launch is shaped.
+#include <cuda_runtime.h>
+#include <string.h>
+
+#include "aq_internal.h"
+#include "warp_mma.cuh"
+
+namespace aq {
+
+namespace {
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+int tokens_per_tile(int64_t M) { return M <= 8 ? 8 : M <= 16 ? 16 : 32; }
+
+// scales and biases of a CTA's rows, staged in shared memory
+constexpr int64_t SB_MAX_BYTES = 64 * 1024;
+
+struct Shape {
+    int ntl, wr, wk, gpw;
+    int x_pitch;
+    bool xsm;
+    dim3 grid;
+    size_t smem;
+};
+
+// Warps of a CTA: wr blocks of 32 W rows while the CTAs still cover every SM, the rest slices
+// of K.  The split of K depends on N, K and the total rows only (not on how the rows are
+// grouped into launch batches), so a strided view and its contiguous copy sum in the same
+// order and give the same bits.
+Shape shape_for(const MmaProblem& p, int sms) {
+    Shape s;
+    const int nt = tokens_per_tile(p.M);
+    s.ntl = nt / 8;
+    const int64_t kg = p.K / p.group;
+    const int64_t nrt = (p.N + wm::ROWS - 1) / wm::ROWS;
+    const int64_t rows_all = p.M * p.nb[0] * p.nb[1];
+    const int64_t units = (rows_all + wm::MAX_TOKENS - 1) / wm::MAX_TOKENS;
+    int wr = 1;
+    while (wr < wm::MAX_WARPS && ((nrt + 2 * wr - 1) / (2 * wr)) * units >= sms &&
+           (int64_t)(2 * wr) * wm::ROWS * kg * 4 <= SB_MAX_BYTES)
+        wr *= 2;
+    int64_t wk = wm::MAX_WARPS / wr;
+    if (wk > kg) wk = kg;
+    const int64_t gpw = (kg + wk - 1) / wk;
+    wk = (kg + gpw - 1) / gpw;
+    s.wr = wr;
+    s.wk = (int)wk;
+    s.gpw = (int)gpw;
+    s.grid = dim3((unsigned)((nrt + wr - 1) / wr), (unsigned)((p.M + nt - 1) / nt), (unsigned)(p.nb[0] * p.nb[1]));
+    s.x_pitch = (int)(2 * p.K + 16);
+    const size_t base = wm::smem_bytes(s.wr * s.wk, s.wr, (int)kg, nt, s.x_pitch, false);
+    s.xsm = base + (size_t)nt * s.x_pitch <= wm::SMEM_LIMIT;
+    s.smem = wm::smem_bytes(s.wr * s.wk, s.wr, (int)kg, nt, s.x_pitch, s.xsm);
+    return s;
+}
+
+}  // namespace
+
+bool warp_mma_supported(const MmaProblem& p) {
+#if defined(AQ_WARP_MMA) && AQ_WARP_MMA == 0
+    return false;
+#endif
+    if (p.offsets) return false;
+    // by the total rows, so that a strided view and its contiguous copy run the same kernel
+    if (p.M < 1 || p.M * p.nb[0] * p.nb[1] > wm::MAX_TOKENS || p.N < 1) return false;
+    if (!(p.bits == 2 || p.bits == 4 || p.bits == 8)) return false;
+    if (!(p.group == 32 || p.group == 64 || p.group == 128)) return false;
+    if (p.bits * (p.group < 64 ? p.group : 64) < 128) return false;   // a lane's codes fill whole words
+    if (p.K % p.group != 0 || p.K < p.group) return false;
+    const int64_t kg = p.K / p.group;
+    if ((size_t)kg * wm::MAX_TOKENS * sizeof(float) > (size_t)wm::MAX_XTAB_BYTES) return false;
+    if ((int64_t)wm::ROWS * kg * 4 > SB_MAX_BYTES) return false;
+    if (p.nb[0] * p.nb[1] > 65535 || (p.N + wm::ROWS - 1) / wm::ROWS > 0x7fffffff) return false;
+    // 16-byte rows of x and W, as the tensor-core kernels require (checked by mma_supported)
+    return true;
+}
+
+// Whether the warp kernel is the faster choice for a problem it supports.  Measured on B200 at
+// 8/16/32 tokens against the tcgen05 small-M kernel (decode shapes, K 1024..3072, N 1024..151936):
+// the warp kernel wins every case of up to 16 tokens, and at 32 tokens when each warp of a
+// one-row-block CTA has at most two sub-blocks of K (the decode projections with K = 1024); with
+// more K per warp, or many row blocks per CTA (lm_head), its mma.sync work per SM outweighs the
+// tcgen05 kernel's fixed costs.  The choice depends on N, K and the total rows only.
+bool warp_mma_preferred(const MmaProblem& p) {
+#if defined(AQ_WARP_MMA) && AQ_WARP_MMA == 2
+    return true;
+#endif
+    const Shape s = shape_for(p, sm_count());
+    if (p.M * p.nb[0] * p.nb[1] <= 16) return true;
+    const int spg = p.group > 64 ? p.group / 64 : 1;
+    return s.wr == 1 && s.gpw * spg <= 2;
+}
+
+cudaError_t launch_warp_mma(const MmaProblem& pb, cudaStream_t stream) {
+    const Shape s = shape_for(pb, sm_count());
+    wm::WParams p;
+    memset(&p, 0, sizeof p);
+    p.x = static_cast<const uint16_t*>(pb.x);
+    p.y = pb.y;
+    p.wq = pb.wq;
+    p.scales = static_cast<const uint16_t*>(pb.scales);
+    p.biases = static_cast<const uint16_t*>(pb.biases);
+    p.M = pb.M;
+    p.N = pb.N;
+    p.K = pb.K;
+    p.x_row = pb.x_row;
+    p.y_row = pb.y_row;
+    for (int i = 0; i < 2; ++i) {
+        p.xb[i] = pb.nb[i] > 1 ? pb.xb[i] : 0;
+        p.yb[i] = pb.nb[i] > 1 ? pb.yb[i] : 0;
+    }
+    p.nb1 = pb.nb[1] > 0 ? pb.nb[1] : 1;
+    p.w_row = pb.w_row;
+    p.kg = (int)(pb.K / pb.group);
+    p.gpw = s.gpw;
+    p.wr = s.wr;
+    p.wk = s.wk;
+    p.ydt = (int)pb.ydt;
+    const size_t ysz = pb.ydt == DT::F32 ? 4 : 2;
+    bool yvec = ((uintptr_t)pb.y % (2 * ysz)) == 0 && (pb.M <= 1 || pb.y_row % 2 == 0);
+    for (int i = 0; i < 2; ++i)
+        if (pb.nb[i] > 1 && pb.yb[i] % 2 != 0) yvec = false;
+    p.yvec = yvec ? 1 : 0;
+    p.xsm = s.xsm ? 1 : 0;
+    p.x_pitch = s.x_pitch;
+    p.sb16 = (p.kg % 8 == 0 && ((uintptr_t)pb.scales & 15) == 0 && ((uintptr_t)pb.biases & 15) == 0) ? 1 : 0;
+    const bool bf = pb.xdt == DT::BF16;
+    const int warps = s.wr * s.wk;
+    switch (pb.bits) {
+        case 2: return wm::launch<2>(bf, pb.group, s.ntl, p, s.grid, warps, s.smem, stream);
+        case 4: return wm::launch<4>(bf, pb.group, s.ntl, p, s.grid, warps, s.smem, stream);
+        case 8: return wm::launch<8>(bf, pb.group, s.ntl, p, s.grid, warps, s.smem, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace aq

@@ -1,0 +1,59 @@
+// warp_mma.cuh -- definitions shared by the host side of the warp-level tensor-core kernel
+// (kernels_warp_mma.cu) and its device code (warp_mma_kernel.cuh, instantiated once per bit
+// width in kernels_warp_mma_b{2,4,8}.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace aq {
+namespace wm {
+
+constexpr int ROWS = 32;             // W rows per warp: two m16 tiles of mma.sync
+constexpr int MAX_WARPS = 8;         // warps per CTA
+constexpr int MAX_TOKENS = 32;       // x rows per token tile: up to four n8 tiles
+constexpr int RING_BYTES = 8192;     // per-warp ring of W sub-blocks in shared memory
+constexpr int RED_PITCH = ROWS + 4;  // floats per token of a warp's partial y tile (bank spread)
+constexpr int MAX_XTAB_BYTES = 48 * 1024;
+
+struct WParams {
+    const uint16_t* x;       // [nb0, nb1, M, K] through xb / x_row
+    void* y;                 // [nb0, nb1, M, N] through yb / y_row
+    const uint32_t* wq;      // [N, w_row] packed codes
+    const uint16_t* scales;  // [N, kg]
+    const uint16_t* biases;  // [N, kg]
+    int64_t M, N, K;
+    int64_t x_row, y_row;
+    int64_t xb[2], yb[2];
+    int64_t nb1;
+    int64_t w_row;           // words between W rows
+    int kg;                  // groups per row (K / group)
+    int gpw;                 // groups per warp
+    int wr, wk;              // warps of a CTA along W rows / along K
+    int ydt;                 // DT of y
+    int yvec;                // 1: pairs of adjacent y elements may be stored as one vector
+    int xsm;                 // 1: the CTA's x tile is staged in shared memory
+    int x_pitch;             // bytes per staged x row (2 K + 16: spreads the lanes over the banks)
+    int sb16;                // 1: scale/bias rows are copied in 16-byte pieces (else 4-byte)
+};
+
+constexpr size_t SMEM_LIMIT = 227 * 1024;
+
+// Dynamic shared memory of a launch: the warps' W rings, the sums of x per group and token, the
+// scales and biases of the CTA's rows and, when staged, the x tile.
+inline size_t smem_bytes(int warps, int wr, int kg, int nt, int x_pitch, bool xsm) {
+    return (size_t)warps * RING_BYTES + (size_t)kg * nt * sizeof(float) + (size_t)wr * ROWS * kg * 2 * 2 +
+           (xsm ? (size_t)nt * x_pitch : 0);
+}
+
+// defined in warp_mma_kernel.cuh, instantiated in kernels_warp_mma_b<BITS>.cu
+template <int BITS>
+cudaError_t launch(bool bf16, int group, int ntl, const WParams& p, dim3 grid, int warps, size_t smem,
+                   cudaStream_t stream);
+extern template cudaError_t launch<2>(bool, int, int, const WParams&, dim3, int, size_t, cudaStream_t);
+extern template cudaError_t launch<4>(bool, int, int, const WParams&, dim3, int, size_t, cudaStream_t);
+extern template cudaError_t launch<8>(bool, int, int, const WParams&, dim3, int, size_t, cudaStream_t);
+
+}  // namespace wm
+}  // namespace aq

@@ -1,0 +1,495 @@
+// warp_mma_kernel.cuh -- warp-level tensor-core kernel for decode batches (up to 32 rows of x
+// per launch batch).
+//
+// What it computes, like the other kernels of the library (the factored form of
+// x . (s*q + b)^T, "mlx PR #4516", load_vector fix):
+//     y[t, n] = sum_g  s[n,g] * D[n,g,t]  +  b[n,g] * X[g,t]
+//     D[n,g,t] = sum_{k in g} q[n,k] * x[t,k]   (tensor cores, exact integer codes, fp32 sums)
+//     X[g,t]   = sum_{k in g} x[t,k]            (x widened to fp32 before it is summed)
+//
+// Why a warp-level MMA here.  At a few dozen tokens the contraction has too few columns to keep
+// a tcgen05 tile busy: the time of the tensor-memory kernel goes into moving expanded codes
+// into tensor memory and each group's accumulator out of it, and its set-up (TMEM allocation,
+// barrier rings, a pipeline of specialised warps) dominates the small projections of a decode
+// step.  Here every step stays in the registers of one warp: the packed codes come from shared
+// memory, are expanded in place into mma.sync A fragments, and each group's accumulator is
+// folded into the running output with two FMAs per element.
+//
+// Layout of the work.  A warp owns 32 W rows (two m16 tiles) x NT = 8*NTL tokens (NTL n8 tiles)
+// and a contiguous range of groups; a CTA holds wr x wk warps, wr blocks of rows times wk slices
+// of K, whose partial tiles are summed in shared memory in slice order at the end (the result
+// does not depend on timing).  Within a sub-block of KS = min(G, 64) codes, lane (r = lane/4,
+// c = lane%4) owns codes c*KS/4 .. c*KS/4 + KS/4 - 1 of W rows r and r+8 of each m tile, and of
+// x row r of each n tile; k step s of the MMA takes codes 4s .. 4s+3 of every lane's span.  The
+// order of k inside an MMA is thus a permutation of the group's codes, the same for A (codes)
+// and B (x), which leaves every group sum unchanged and lets a lane load its x as plain 16-byte
+// vectors and its codes as one 4-, 8- or 16-byte word run.
+//
+// Memory.  W streams through a per-warp ring of RD sub-blocks in shared memory, filled with
+// 16-byte cp.async copies that the 32 lanes of the warp share; a lane reads its fragment words
+// back after the ring slot's copy group completed and the warp synchronised, so no other warp
+// is involved.  At the start the CTA stages, in one cp.async group issued before the ring's,
+// the scales and biases of its rows and (when it fits in shared memory) its x tile, so that no
+// group waits on a DRAM round trip of its own; the sums X of the tile are then built once per
+// CTA into shared memory by all threads.  An x tile too large to stage is read through L1.
+//
+// Partial rows and tokens: loads of rows past N and of tokens past M are clamped to the last
+// valid one; only the final stores check bounds, so the inner loop carries no bounds test.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <mutex>
+#include <type_traits>
+
+#include "aq_internal.h"
+#include "device_common.cuh"
+#include "sm100_ptx.cuh"
+#include "warp_mma.cuh"
+
+namespace aq {
+namespace wm {
+
+template <int BITS, int G>
+struct Geo {
+    static constexpr int KS = G < 64 ? G : 64;         // codes per sub-block
+    static constexpr int SPG = G / KS;                 // sub-blocks per group
+    static constexpr int STEPS = KS / 16;              // MMA k steps per sub-block
+    static constexpr int KSB = KS * BITS / 8;          // bytes of one W row per sub-block
+    static constexpr int LB = KSB / 4;                 // bytes of one W row per lane
+    static constexpr int WS = LB / 4;                  // words of one W row per lane
+    static constexpr int RD = RING_BYTES / (ROWS * KSB) < 16 ? RING_BYTES / (ROWS * KSB) : 16;  // ring depth
+    static constexpr int CPR = KSB / 16;               // 16-byte copies per W row
+    static constexpr int CPL = ROWS * CPR / 32;        // 16-byte copies per lane per sub-block
+    static constexpr int XV = KS / 32;                 // 16-byte x vectors per lane per n tile
+    static_assert(WS >= 1 && CPL >= 1 && RD >= 2 && RD * ROWS * KSB <= RING_BYTES, "sub-block geometry");
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// d += A (16 x 16, row) . B (16 x 8, col), fp32 accumulation
+template <bool BF>
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    if constexpr (BF)
+        asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    else
+        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// f16 pairs (1024 + q0, 1024 + q1) -> (q0, q1), exact
+__device__ __forceinline__ uint32_t f16_minus_1024(uint32_t v) {
+    const uint32_t off = 0x64006400u;
+    const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&v), *reinterpret_cast<const __half2*>(&off));
+    return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// The codes 4s .. 4s+3 of one W row of a lane's span, for every k step s, as two 16-bit pairs:
+// a[s][0] = (code 4s, code 4s+1), a[s][1] = (code 4s+2, code 4s+3).
+//   bf16, 2/4 bits: 128 + q (a code OR-ed into the mantissa of 128.0; the fold removes the 128)
+//   bf16, 8 bits:   q, formed exactly in fp32 (2^23 + q minus 2^23) and converted (q <= 255)
+//   f16, any:       q, from 1024 + q (OR-ed into the mantissa of 1024.0) minus 1024
+template <int BITS, bool BF, int STEPS>
+__device__ __forceinline__ void expand_row(const uint32_t* wv, uint32_t (*a)[2]) {
+    constexpr uint32_t MAGIC = BF ? 0x43004300u : 0x64006400u;
+    auto fin = [](uint32_t v) -> uint32_t {
+        if constexpr (BF) return v;
+        else return f16_minus_1024(v);
+    };
+    if constexpr (BITS == 4) {
+        // byte b of a word holds codes (2b, 2b+1); the word shifted right by 4 holds code 2b+1 in
+        // the low nibble of byte b.  PRMT puts byte b of each into the low byte of a half.
+#pragma unroll
+        for (int s = 0; s < STEPS; ++s) {
+            const uint32_t w = wv[s >> 1], sh = w >> 4;
+            const int b = 2 * (s & 1);
+            a[s][0] = fin((__byte_perm(w, sh, b | ((4 + b) << 8)) & 0x000F000Fu) | MAGIC);
+            a[s][1] = fin((__byte_perm(w, sh, (b + 1) | ((5 + b) << 8)) & 0x000F000Fu) | MAGIC);
+        }
+    } else if constexpr (BITS == 2) {
+        // byte b holds codes 4b .. 4b+3 in bit pairs 0-1, 2-3, 4-5, 6-7
+#pragma unroll
+        for (int s = 0; s < STEPS; ++s) {
+            const uint32_t w = wv[s >> 2];
+            const int b = s & 3;
+            a[s][0] = fin((__byte_perm(w, w >> 2, b | ((4 + b) << 8)) & 0x00030003u) | MAGIC);
+            a[s][1] = fin((__byte_perm(w >> 4, w >> 6, b | ((4 + b) << 8)) & 0x00030003u) | MAGIC);
+        }
+    } else {
+        static_assert(BITS == 8, "bits");
+#pragma unroll
+        for (int s = 0; s < STEPS; ++s) {
+            const uint32_t w = wv[s];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                if constexpr (BF) {
+                    const float m0 = __uint_as_float(__byte_perm(w, 0x4B000000u, (2 * j) | (4 << 4) | (5 << 8) | (7 << 12)));
+                    const float m1 = __uint_as_float(__byte_perm(w, 0x4B000000u, (2 * j + 1) | (4 << 4) | (5 << 8) | (7 << 12)));
+                    const __nv_bfloat162 q = __floats2bfloat162_rn(m0 - 8388608.0f, m1 - 8388608.0f);
+                    a[s][j] = *reinterpret_cast<const uint32_t*>(&q);
+                } else {
+                    a[s][j] = f16_minus_1024(__byte_perm(w, MAGIC, (2 * j) | (5 << 4) | ((2 * j + 1) << 8) | (7 << 12)));
+                }
+            }
+        }
+    }
+}
+
+template <int LB>
+__device__ __forceinline__ void load_lane_words(const uint8_t* p, uint32_t* w) {
+    if constexpr (LB == 16) {
+        const uint4 v = *reinterpret_cast<const uint4*>(p);
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    } else if constexpr (LB == 8) {
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
+        w[0] = v.x; w[1] = v.y;
+    } else {
+        w[0] = *reinterpret_cast<const uint32_t*>(p);
+    }
+}
+
+template <typename XT>
+__device__ __forceinline__ void store_pair(void* y, int64_t off, float v0, float v1, bool both, bool vec, int ydt) {
+    if (ydt == (int)DT::F32) {
+        float* p = reinterpret_cast<float*>(y) + off;
+        if (both && vec) *reinterpret_cast<float2*>(p) = make_float2(v0, v1);
+        else { p[0] = v0; if (both) p[1] = v1; }
+    } else if constexpr (std::is_same<XT, bf16_t>::value) {
+        __nv_bfloat16* p = reinterpret_cast<__nv_bfloat16*>(y) + off;
+        if (both && vec) *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v0, v1);
+        else { p[0] = __float2bfloat16_rn(v0); if (both) p[1] = __float2bfloat16_rn(v1); }
+    } else {
+        __half* p = reinterpret_cast<__half*>(y) + off;
+        if (both && vec) *reinterpret_cast<__half2*>(p) = __floats2half2_rn(v0, v1);
+        else { p[0] = __float2half_rn(v0); if (both) p[1] = __float2half_rn(v1); }
+    }
+}
+
+template <int BITS, typename XT, int G, int NTL>
+__global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __grid_constant__ WParams p) {
+    using Gm = Geo<BITS, G>;
+    constexpr bool BF = std::is_same<XT, bf16_t>::value;
+    constexpr int NT = 8 * NTL;
+    constexpr int KS = Gm::KS, SPG = Gm::SPG, STEPS = Gm::STEPS, KSB = Gm::KSB, LB = Gm::LB, WS = Gm::WS;
+    constexpr int RD = Gm::RD, CPR = Gm::CPR, CPL = Gm::CPL, XV = Gm::XV;
+    constexpr float OFF = (BF && BITS < 8) ? 128.0f : 0.0f;   // code offset of the expanded A values
+
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    const int rw = warp % p.wr, kw = warp / p.wr;
+    const int r = lane >> 2, c = lane & 3;
+    const int kg = p.kg;
+    const int rows_cta = p.wr * ROWS;
+    // [rings][sums of x: kg x NT fp32][scales, biases: rows_cta x kg each][x tile: NT x x_pitch]
+    uint8_t* ring = smem + (size_t)warp * RING_BYTES;
+    float* xs = reinterpret_cast<float*>(smem + (size_t)nwarps * RING_BYTES);
+    uint16_t* s_s = reinterpret_cast<uint16_t*>(xs + kg * NT);
+    uint16_t* s_b = s_s + rows_cta * kg;
+    uint8_t* xt = reinterpret_cast<uint8_t*>(s_b + rows_cta * kg);
+    const int xp = p.x_pitch;
+
+    const int64_t bz = blockIdx.z;
+    const int64_t bo = bz / p.nb1, bi = bz - bo * p.nb1;
+    const uint16_t* x = p.x + bo * p.xb[0] + bi * p.xb[1];
+    const int64_t tok0 = (int64_t)blockIdx.y * NT;
+    const int64_t rowc = (int64_t)blockIdx.x * rows_cta;        // first W row of the CTA
+    const int64_t roww = rowc + rw * ROWS;                       // first W row of this warp
+    const int g0 = kw * p.gpw;
+    const int g1 = min(g0 + p.gpw, kg);
+    const int nsub = (roww < p.N && g1 > g0) ? (g1 - g0) * SPG : 0;
+
+    // x may be the output of the previous kernel in the stream: read nothing before it completed
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
+
+    // ---- one copy group: the scales and biases of the CTA's rows, and the x tile when it fits ----
+    {
+        const uint32_t ss = ptx::smem_u32(s_s), sb = ptx::smem_u32(s_b);
+        const int step = p.sb16 ? 8 : 2;          // elements per copy (16 or 4 bytes)
+        const int cpr = kg / step;
+        const int total = rows_cta * cpr;
+        for (int i = threadIdx.x; i < total; i += blockDim.x) {
+            const int rl = i / cpr, col = i - rl * cpr;
+            const int64_t go = min(rowc + rl, p.N - 1) * kg + col * step;
+            const uint32_t so = (uint32_t)((rl * kg + col * step) * 2);
+            if (p.sb16) {
+                cp_async16(ss + so, p.scales + go);
+                cp_async16(sb + so, p.biases + go);
+            } else {
+                cp_async4(ss + so, p.scales + go);
+                cp_async4(sb + so, p.biases + go);
+            }
+        }
+        if (p.xsm) {
+            const uint32_t xb = ptx::smem_u32(xt);
+            const int xcpr = (int)(p.K / 8);
+            const int xtotal = NT * xcpr;
+            for (int i = threadIdx.x; i < xtotal; i += blockDim.x) {
+                const int t = i / xcpr, col = i - t * xcpr;
+                const int64_t tok = min(tok0 + t, p.M - 1);
+                cp_async16(xb + (uint32_t)(t * xp + col * 16), x + tok * p.x_row + col * 8);
+            }
+        }
+        cp_async_commit();
+    }
+
+    // ---- W ring: lane copies the 16-byte pieces lane + 32 i of each sub-block ----
+    const uint8_t* csrc[CPL];
+    uint32_t cdst[CPL];
+    {
+        const uint32_t ring_s = ptx::smem_u32(ring);
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int q = lane + 32 * i, rl = q / CPR, col = q % CPR;
+            const int64_t n = min(roww + rl, p.N - 1);
+            csrc[i] = reinterpret_cast<const uint8_t*>(p.wq + n * p.w_row) + (int64_t)g0 * SPG * KSB + col * 16;
+            cdst[i] = ring_s + (uint32_t)(rl * KSB + col * 16);
+        }
+    }
+    auto issue = [&](int j) {
+        const uint32_t so = (uint32_t)((j % RD) * ROWS * KSB);
+        const int64_t go = (int64_t)j * KSB;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) cp_async16(cdst[i] + so, csrc[i] + go);
+    };
+#pragma unroll
+    for (int j = 0; j < RD; ++j) {
+        if (j < nsub) issue(j);
+        cp_async_commit();   // one group per sub-block, empty past the end: wait counts stay uniform
+    }
+
+    cp_async_wait<RD>();     // this thread's part of the staging group has landed
+    __syncthreads();         // ... and every other thread's
+
+    // ---- sums of x per group and token of the tile: xs[g * NT + t] (consecutive threads take
+    // consecutive tokens of one group) ----
+    {
+        const int total = kg * NT;
+        for (int i = threadIdx.x; i < total; i += blockDim.x) {
+            const int g = i / NT, t = i - g * NT;
+            const uint4* src = p.xsm ? reinterpret_cast<const uint4*>(xt + t * xp + g * G * 2)
+                                     : reinterpret_cast<const uint4*>(x + min(tok0 + t, p.M - 1) * p.x_row + (int64_t)g * G);
+            uint4 v[G / 8];
+#pragma unroll
+            for (int u = 0; u < G / 8; ++u) v[u] = src[u];
+            float sum = 0.0f;
+#pragma unroll
+            for (int u = 0; u < G / 8; ++u) {
+                float f[8];
+                unpack8(v[u], f, XT{});
+#pragma unroll
+                for (int e = 0; e < 8; ++e) sum += f[e];
+            }
+            xs[i] = sum;
+        }
+    }
+    __syncthreads();
+
+    // ---- this lane's rows of the scale/bias tiles and x rows ----
+    int sb_row[4];   // (row - rowc) * kg for rows roww + 16 m + 8 h + r, index 2 m + h
+#pragma unroll
+    for (int mh = 0; mh < 4; ++mh) sb_row[mh] = (rw * ROWS + 16 * (mh >> 1) + 8 * (mh & 1) + r) * kg;
+    const uint8_t* xrow[NTL];   // this lane's span of x row 8 t + r (shared memory or global)
+#pragma unroll
+    for (int t = 0; t < NTL; ++t) {
+        if (p.xsm) {
+            xrow[t] = xt + (8 * t + r) * xp + c * (KS / 2);
+        } else {
+            const int64_t tok = min(tok0 + 8 * t + r, p.M - 1);
+            xrow[t] = reinterpret_cast<const uint8_t*>(x + tok * p.x_row + c * (KS / 4));
+        }
+    }
+    const uint8_t* rd_lane = ring + r * KSB + c * LB;
+
+    float acc[2][NTL][4];
+#pragma unroll
+    for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int t = 0; t < NTL; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[m][t][e] = 0.0f;
+    float d[2][NTL][4];
+
+#pragma unroll 1
+    for (int j = 0; j < nsub; ++j) {
+        const int g = g0 + j / SPG, sub = j % SPG;
+        if (sub == 0) {
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+#pragma unroll
+                for (int t = 0; t < NTL; ++t)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) d[m][t][e] = 0.0f;
+        }
+        // codes of this sub-block from the ring
+        cp_async_wait<RD - 1>();
+        __syncwarp();
+        uint32_t wv[4][WS];
+        {
+            const uint8_t* slot = rd_lane + (j % RD) * ROWS * KSB;
+#pragma unroll
+            for (int mh = 0; mh < 4; ++mh) load_lane_words<LB>(slot + (16 * (mh >> 1) + 8 * (mh & 1)) * KSB, wv[mh]);
+        }
+        __syncwarp();   // every lane has read the slot before it is refilled
+        if (j + RD < nsub) issue(j + RD);
+        cp_async_commit();
+
+        uint32_t a[4][STEPS][2];
+#pragma unroll
+        for (int mh = 0; mh < 4; ++mh) expand_row<BITS, BF, STEPS>(wv[mh], a[mh]);
+
+        const int kx2 = (g * G + sub * KS) * 2;   // byte offset of the sub-block in an x row
+#pragma unroll
+        for (int t = 0; t < NTL; ++t) {
+            uint4 xv[XV];
+#pragma unroll
+            for (int v = 0; v < XV; ++v) xv[v] = reinterpret_cast<const uint4*>(xrow[t] + kx2)[v];
+            const uint32_t* xw = reinterpret_cast<const uint32_t*>(xv);
+#pragma unroll
+            for (int s = 0; s < STEPS; ++s)
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
+                    mma16816<BF>(d[m][t], a[2 * m][s][0], a[2 * m + 1][s][0], a[2 * m][s][1], a[2 * m + 1][s][1],
+                                 xw[2 * s], xw[2 * s + 1]);
+        }
+
+        if (sub == SPG - 1) {   // fold the group: acc += s * D + (b - OFF * s) * X
+            float sv[4], bv[4];
+#pragma unroll
+            for (int mh = 0; mh < 4; ++mh) {
+                sv[mh] = half_bits_to_float(s_s[sb_row[mh] + g], XT{});
+                bv[mh] = half_bits_to_float(s_b[sb_row[mh] + g], XT{});
+                if (OFF != 0.0f) bv[mh] = fmaf(-OFF, sv[mh], bv[mh]);
+            }
+            const float* xg = xs + g * NT + 2 * c;
+#pragma unroll
+            for (int t = 0; t < NTL; ++t) {
+                const float2 X = *reinterpret_cast<const float2*>(xg + 8 * t);
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float s = sv[2 * m + h], b = bv[2 * m + h];
+                        acc[m][t][2 * h] = fmaf(s, d[m][t][2 * h], fmaf(b, X.x, acc[m][t][2 * h]));
+                        acc[m][t][2 * h + 1] = fmaf(s, d[m][t][2 * h + 1], fmaf(b, X.y, acc[m][t][2 * h + 1]));
+                    }
+            }
+        }
+    }
+
+    // ---- partial tile of this warp into its own ring (no copy is in flight any more) ----
+    cp_async_wait<0>();
+    __syncwarp();
+    {
+        float* red = reinterpret_cast<float*>(ring);
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int t = 0; t < NTL; ++t)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+                        red[(8 * t + 2 * c + e) * RED_PITCH + 16 * m + 8 * h + r] = acc[m][t][2 * h + e];
+    }
+    __syncthreads();
+
+    // ---- sum the K slices in slice order and store pairs of adjacent outputs ----
+    const int rpairs = p.wr * (ROWS / 2);
+    const int total = NT * rpairs;
+    const int64_t ybase = bo * p.yb[0] + bi * p.yb[1];
+    for (int i = threadIdx.x; i < total; i += blockDim.x) {
+        const int tt = i / rpairs, rp = i - tt * rpairs;
+        const int wrr = rp / (ROWS / 2), rl = 2 * (rp % (ROWS / 2));
+        const int64_t tok = tok0 + tt, n = rowc + wrr * ROWS + rl;
+        if (tok >= p.M || n >= p.N) continue;
+        float v0 = 0.0f, v1 = 0.0f;
+        for (int k = 0; k < p.wk; ++k) {
+            const float* part = reinterpret_cast<const float*>(smem + (size_t)(k * p.wr + wrr) * RING_BYTES);
+            const float2 u = *reinterpret_cast<const float2*>(part + tt * RED_PITCH + rl);
+            v0 += u.x;
+            v1 += u.y;
+        }
+        store_pair<XT>(p.y, ybase + tok * p.y_row + n, v0, v1, n + 1 < p.N, p.yvec != 0, p.ydt);
+    }
+}
+
+template <int BITS, typename XT, int G, int NTL>
+cudaError_t launch_t(const WParams& p, dim3 grid, int warps, size_t smem, cudaStream_t s) {
+    static std::mutex mu;
+    static bool done[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!done[dev]) {
+            e = cudaFuncSetAttribute(qmm_warp_kernel<BITS, XT, G, NTL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)SMEM_LIMIT);
+            if (e != cudaSuccess) return e;
+            done[dev] = true;
+        }
+    }
+    // a programmatic dependent of the previous kernel in the stream: it may be scheduled early,
+    // but reads nothing before that kernel completed (griddepcontrol.wait at its start)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(32 * warps);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, qmm_warp_kernel<BITS, XT, G, NTL>, p);
+}
+
+template <int BITS, typename XT, int G>
+cudaError_t launch_n(int ntl, const WParams& p, dim3 grid, int warps, size_t smem, cudaStream_t s) {
+    switch (ntl) {
+        case 1: return launch_t<BITS, XT, G, 1>(p, grid, warps, smem, s);
+        case 2: return launch_t<BITS, XT, G, 2>(p, grid, warps, smem, s);
+        case 4: return launch_t<BITS, XT, G, 4>(p, grid, warps, smem, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <int BITS, typename XT>
+cudaError_t launch_g(int group, int ntl, const WParams& p, dim3 grid, int warps, size_t smem, cudaStream_t s) {
+    switch (group) {
+        case 32:
+            if constexpr (BITS * 32 >= 128) return launch_n<BITS, XT, 32>(ntl, p, grid, warps, smem, s);
+            else return cudaErrorInvalidValue;
+        case 64: return launch_n<BITS, XT, 64>(ntl, p, grid, warps, smem, s);
+        case 128: return launch_n<BITS, XT, 128>(ntl, p, grid, warps, smem, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <int BITS>
+cudaError_t launch(bool bf16, int group, int ntl, const WParams& p, dim3 grid, int warps, size_t smem,
+                   cudaStream_t stream) {
+    return bf16 ? launch_g<BITS, bf16_t>(group, ntl, p, grid, warps, smem, stream)
+                : launch_g<BITS, f16_t>(group, ntl, p, grid, warps, smem, stream);
+}
+
+}  // namespace wm
+}  // namespace aq

@@ -120,13 +120,15 @@ aq_status aq_dequantize(const aq_view* wq, const aq_view* scales, const aq_view*
  * scales, biases: [..., N, K/group], same dtype as x, same batch dims as wq.
  * y:      x.shape[:-1] + [N], dtype of x or AQ_F32, must not overlap inputs.
  * bits in {2,3,4,5,6,8}; group in {32,64,128}; K % group == 0.
- * Rows per launch batch decide the kernel: up to 4 rows (or a batched W), a
- * CUDA-core GEMV; 5..63 rows, a tcgen05/TMEM tensor-core kernel on tiles of
- * 128 W rows x 32 tokens (K split over the CTAs of a thread-block cluster
+ * Rows per launch batch decide the kernel (aq_plan_linear reports it): up to 4
+ * rows (or a batched W), a CUDA-core GEMV; 5..32 rows with 2/4/8-bit codes, a
+ * warp-level mma.sync kernel that expands W in registers (2-bit codes need
+ * groups of 64/128); other cases below 64 rows, a tcgen05/TMEM kernel on tiles
+ * of 128 W rows x 32 tokens (K split over the CTAs of a thread-block cluster
  * when the tiles alone would leave most SMs idle); 64 rows and more with
- * groups of 64/128, a tensor-core kernel on 128 x 128 tiles.  3/5-bit codes,
- * K not a multiple of 64, an odd or very large K/group, or unaligned rows
- * take the GEMV.
+ * groups of 64/128, a tcgen05 kernel on 128 x 128 tiles.  3/5-bit codes, K
+ * not a multiple of 64, an odd or very large K/group, or unaligned rows take
+ * the GEMV.
  * Every kernel keeps W exact (integer codes, scale and bias in fp32).  The
  * tensor-core kernels are launched as programmatic dependents of the previous
  * kernel in the stream: only their set-up overlaps it; stream order is kept.
@@ -166,8 +168,16 @@ aq_status aq_qmm_t_grouped(const aq_view* x_sorted, const int64_t* offsets, int 
 
 typedef enum aq_regime {
     AQ_REGIME_QMV = 0,   /* CUDA-core GEMV                      */
-    AQ_REGIME_MMA = 1    /* tcgen05 tensor-core kernel (TMEM)   */
+    AQ_REGIME_MMA = 1    /* a tensor-core kernel (aq_kernel)    */
 } aq_regime;
+
+/* The kernel a call runs (aq_plan.kernel). */
+typedef enum aq_kernel {
+    AQ_KERNEL_GEMV = 0,        /* CUDA-core GEMV, 128-bit loads, warp-shuffle sums        */
+    AQ_KERNEL_WARP_MMA = 1,    /* mma.sync, W expanded in registers, up to 32 rows        */
+    AQ_KERNEL_TC_SMALL_M = 2,  /* tcgen05/TMEM, 128 W rows x 32 tokens, split-K clusters  */
+    AQ_KERNEL_TC_PREFILL = 3   /* tcgen05/TMEM, 128 x 128 tiles, >= 64 rows, groups 64/128 */
+} aq_kernel;
 
 /* How a call will be executed: the result of view resolution and batch folding. */
 typedef struct aq_plan {
@@ -176,7 +186,7 @@ typedef struct aq_plan {
     int64_t M;                 /* rows per launch batch after folding                  */
     int64_t N, K;
     int32_t nbatch_dims;       /* launch batch dims left after folding (0..2)         */
-    int32_t pad_;
+    int32_t kernel;            /* aq_kernel                                            */
     int64_t batch_shape[2];    /* outer first                                          */
     int64_t x_batch_stride[2];
     int64_t y_batch_stride[2];
