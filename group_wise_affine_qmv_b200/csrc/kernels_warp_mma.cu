@@ -28,7 +28,7 @@ int tokens_per_tile(int64_t M) { return M <= 8 ? 8 : M <= 16 ? 16 : 32; }
 constexpr int64_t SB_MAX_BYTES = 64 * 1024;
 
 struct Shape {
-    int ntl, wr, wk, gpw;
+    int ntl, wr, wk, gpw, cs, kgc;
     int x_pitch;
     bool xsm;
     dim3 grid;
@@ -51,18 +51,26 @@ Shape shape_for(const MmaProblem& p, int sms) {
     while (wr < wm::MAX_WARPS && ((nrt + 2 * wr - 1) / (2 * wr)) * units >= sms &&
            (int64_t)(2 * wr) * wm::ROWS * kg * 4 <= SB_MAX_BYTES)
         wr *= 2;
+    // one row block per CTA and still few CTAs: a cluster of cs CTAs splits K of each row block
+    int cs = 1;
+    if (wr == 1)
+        while (cs < wm::MAX_CLUSTER && nrt * units * cs * 2 <= sms && kg >= 4 * cs) cs *= 2;
+    const int64_t kgc = (kg + cs - 1) / cs;
     int64_t wk = wm::MAX_WARPS / wr;
-    if (wk > kg) wk = kg;
-    const int64_t gpw = (kg + wk - 1) / wk;
-    wk = (kg + gpw - 1) / gpw;
+    if (wk > kgc) wk = kgc;
+    const int64_t gpw = (kgc + wk - 1) / wk;
+    wk = (kgc + gpw - 1) / gpw;
     s.wr = wr;
     s.wk = (int)wk;
     s.gpw = (int)gpw;
-    s.grid = dim3((unsigned)((nrt + wr - 1) / wr), (unsigned)((p.M + nt - 1) / nt), (unsigned)(p.nb[0] * p.nb[1]));
-    s.x_pitch = (int)(2 * p.K + 16);
-    const size_t base = wm::smem_bytes(s.wr * s.wk, s.wr, (int)kg, nt, s.x_pitch, false);
+    s.cs = cs;
+    s.kgc = (int)kgc;
+    s.grid = dim3((unsigned)(((nrt + wr - 1) / wr) * cs), (unsigned)((p.M + nt - 1) / nt),
+                  (unsigned)(p.nb[0] * p.nb[1]));
+    s.x_pitch = (int)(2 * kgc * p.group + 16);
+    const size_t base = wm::smem_bytes(s.wr * s.wk, s.wr, (int)kg, s.kgc, cs, nt, s.x_pitch, false);
     s.xsm = base + (size_t)nt * s.x_pitch <= wm::SMEM_LIMIT;
-    s.smem = wm::smem_bytes(s.wr * s.wk, s.wr, (int)kg, nt, s.x_pitch, s.xsm);
+    s.smem = wm::smem_bytes(s.wr * s.wk, s.wr, (int)kg, s.kgc, cs, nt, s.x_pitch, s.xsm);
     return s;
 }
 
@@ -90,9 +98,9 @@ bool warp_mma_supported(const MmaProblem& p) {
 // Whether the warp kernel is the faster choice for a problem it supports.  Measured on B200 at
 // 8/16/32 tokens against the tcgen05 small-M kernel (decode shapes, K 1024..3072, N 1024..151936):
 // the warp kernel wins every case of up to 16 tokens, and at 32 tokens when each warp of a
-// one-row-block CTA has at most two sub-blocks of K (the decode projections with K = 1024); with
-// more K per warp, or many row blocks per CTA (lm_head), its mma.sync work per SM outweighs the
-// tcgen05 kernel's fixed costs.  The choice depends on N, K and the total rows only.
+// one-row-block CTA has at most two sub-blocks of K (after a cluster split of K); with more K
+// per warp, or many row blocks per CTA (lm_head), its serial per-warp work outweighs the tcgen05
+// kernel's fixed costs.  The choice depends on N, K and the total rows only.
 bool warp_mma_preferred(const MmaProblem& p) {
 #if defined(AQ_WARP_MMA) && AQ_WARP_MMA == 2
     return true;
@@ -124,6 +132,8 @@ cudaError_t launch_warp_mma(const MmaProblem& pb, cudaStream_t stream) {
     p.nb1 = pb.nb[1] > 0 ? pb.nb[1] : 1;
     p.w_row = pb.w_row;
     p.kg = (int)(pb.K / pb.group);
+    p.cs = s.cs;
+    p.kgc = s.kgc;
     p.gpw = s.gpw;
     p.wr = s.wr;
     p.wk = s.wk;

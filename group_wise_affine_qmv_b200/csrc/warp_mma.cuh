@@ -12,6 +12,7 @@ namespace wm {
 
 constexpr int ROWS = 32;             // W rows per warp: two m16 tiles of mma.sync
 constexpr int MAX_WARPS = 8;         // warps per CTA
+constexpr int MAX_CLUSTER = 4;       // CTAs of a cluster splitting K
 constexpr int MAX_TOKENS = 32;       // x rows per token tile: up to four n8 tiles
 constexpr int RING_BYTES = 8192;     // per-warp ring of W sub-blocks in shared memory
 constexpr int RED_PITCH = ROWS + 4;  // floats per token of a warp's partial y tile (bank spread)
@@ -29,6 +30,8 @@ struct WParams {
     int64_t nb1;
     int64_t w_row;           // words between W rows
     int kg;                  // groups per row (K / group)
+    int cs;                  // CTAs of a cluster splitting K (1: no split)
+    int kgc;                 // groups per CTA of a cluster (kg when cs == 1)
     int gpw;                 // groups per warp
     int wr, wk;              // warps of a CTA along W rows / along K
     int ydt;                 // DT of y
@@ -40,11 +43,12 @@ struct WParams {
 
 constexpr size_t SMEM_LIMIT = 227 * 1024;
 
-// Dynamic shared memory of a launch: the warps' W rings, the sums of x per group and token, the
-// scales and biases of the CTA's rows and, when staged, the x tile.
-inline size_t smem_bytes(int warps, int wr, int kg, int nt, int x_pitch, bool xsm) {
-    return (size_t)warps * RING_BYTES + (size_t)kg * nt * sizeof(float) + (size_t)wr * ROWS * kg * 2 * 2 +
-           (xsm ? (size_t)nt * x_pitch : 0);
+// Dynamic shared memory of a launch: the warps' W rings, the sums of x per group and token of the
+// CTA's groups, the scales and biases of the CTA's rows, the CTA's partial tile when a cluster
+// splits K, and, when staged, the x tile.
+inline size_t smem_bytes(int warps, int wr, int kg, int kgc, int cs, int nt, int x_pitch, bool xsm) {
+    return (size_t)warps * RING_BYTES + (size_t)kgc * nt * sizeof(float) + (size_t)wr * ROWS * kg * 2 * 2 +
+           (cs > 1 ? (size_t)nt * wr * ROWS * sizeof(float) : 0) + (xsm ? (size_t)nt * x_pitch : 0);
 }
 
 // defined in warp_mma_kernel.cuh, instantiated in kernels_warp_mma_b<BITS>.cu

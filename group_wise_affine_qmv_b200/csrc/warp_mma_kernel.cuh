@@ -17,8 +17,10 @@
 //
 // Layout of the work.  A warp owns 32 W rows (two m16 tiles) x NT = 8*NTL tokens (NTL n8 tiles)
 // and a contiguous range of groups; a CTA holds wr x wk warps, wr blocks of rows times wk slices
-// of K, whose partial tiles are summed in shared memory in slice order at the end (the result
-// does not depend on timing).  Within a sub-block of KS = min(G, 64) codes, lane (r = lane/4,
+// of K, whose partial tiles are summed in shared memory in slice order at the end.  When one row
+// block per CTA would still leave most SMs idle, a thread-block cluster of cs CTAs splits the K
+// of each row block; after a cluster barrier every CTA adds the CTAs' partial tiles, in rank
+// order, for its share of the outputs over distributed shared memory.  No sum depends on timing.  Within a sub-block of KS = min(G, 64) codes, lane (r = lane/4,
 // c = lane%4) owns codes c*KS/4 .. c*KS/4 + KS/4 - 1 of W rows r and r+8 of each m tile, and of
 // x row r of each n tile; k step s of the MMA takes codes 4s .. 4s+3 of every lane's span.  The
 // order of k inside an MMA is thus a permutation of the group's codes, the same for A (codes)
@@ -196,22 +198,28 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
     const int r = lane >> 2, c = lane & 3;
     const int kg = p.kg;
     const int rows_cta = p.wr * ROWS;
-    // [rings][sums of x: kg x NT fp32][scales, biases: rows_cta x kg each][x tile: NT x x_pitch]
+    const int cs = p.cs;
+    const int rank = cs > 1 ? (int)ptx::cluster_ctarank() : 0;   // K slice of this CTA in its cluster
+    // [rings][sums of x: kgc x NT fp32][scales, biases: rows_cta x kg each]
+    // [partial tile: NT x rows_cta fp32, clusters only][x tile: NT x x_pitch]
     uint8_t* ring = smem + (size_t)warp * RING_BYTES;
     float* xs = reinterpret_cast<float*>(smem + (size_t)nwarps * RING_BYTES);
-    uint16_t* s_s = reinterpret_cast<uint16_t*>(xs + kg * NT);
+    uint16_t* s_s = reinterpret_cast<uint16_t*>(xs + p.kgc * NT);
     uint16_t* s_b = s_s + rows_cta * kg;
-    uint8_t* xt = reinterpret_cast<uint8_t*>(s_b + rows_cta * kg);
+    float* cpart = reinterpret_cast<float*>(s_b + rows_cta * kg);
+    uint8_t* xt = reinterpret_cast<uint8_t*>(cpart + (cs > 1 ? NT * rows_cta : 0));
     const int xp = p.x_pitch;
 
     const int64_t bz = blockIdx.z;
     const int64_t bo = bz / p.nb1, bi = bz - bo * p.nb1;
     const uint16_t* x = p.x + bo * p.xb[0] + bi * p.xb[1];
     const int64_t tok0 = (int64_t)blockIdx.y * NT;
-    const int64_t rowc = (int64_t)blockIdx.x * rows_cta;        // first W row of the CTA
+    const int64_t rowc = (int64_t)(blockIdx.x / cs) * rows_cta; // first W row of the CTA
     const int64_t roww = rowc + rw * ROWS;                       // first W row of this warp
-    const int g0 = kw * p.gpw;
-    const int g1 = min(g0 + p.gpw, kg);
+    const int cg0 = rank * p.kgc, cg1 = min(cg0 + p.kgc, kg);   // groups of this CTA
+    const int ckg = cg1 > cg0 ? cg1 - cg0 : 0;
+    const int g0 = cg0 + kw * p.gpw;                             // groups of this warp
+    const int g1 = min(g0 + p.gpw, cg1);
     const int nsub = (roww < p.N && g1 > g0) ? (g1 - g0) * SPG : 0;
 
     // x may be the output of the previous kernel in the stream: read nothing before it completed
@@ -236,14 +244,14 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
                 cp_async4(sb + so, p.biases + go);
             }
         }
-        if (p.xsm) {
+        if (p.xsm) {   // codes [cg0 G, cg1 G) of every token row
             const uint32_t xb = ptx::smem_u32(xt);
-            const int xcpr = (int)(p.K / 8);
+            const int xcpr = ckg * G / 8;
             const int xtotal = NT * xcpr;
             for (int i = threadIdx.x; i < xtotal; i += blockDim.x) {
                 const int t = i / xcpr, col = i - t * xcpr;
                 const int64_t tok = min(tok0 + t, p.M - 1);
-                cp_async16(xb + (uint32_t)(t * xp + col * 16), x + tok * p.x_row + col * 8);
+                cp_async16(xb + (uint32_t)(t * xp + col * 16), x + tok * p.x_row + (int64_t)cg0 * G + col * 8);
             }
         }
         cp_async_commit();
@@ -277,14 +285,15 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
     cp_async_wait<RD>();     // this thread's part of the staging group has landed
     __syncthreads();         // ... and every other thread's
 
-    // ---- sums of x per group and token of the tile: xs[g * NT + t] (consecutive threads take
-    // consecutive tokens of one group) ----
+    // ---- sums of x per group and token of the tile: xs[(g - cg0) * NT + t] (consecutive threads
+    // take consecutive tokens of one group) ----
     {
-        const int total = kg * NT;
+        const int total = ckg * NT;
         for (int i = threadIdx.x; i < total; i += blockDim.x) {
-            const int g = i / NT, t = i - g * NT;
-            const uint4* src = p.xsm ? reinterpret_cast<const uint4*>(xt + t * xp + g * G * 2)
-                                     : reinterpret_cast<const uint4*>(x + min(tok0 + t, p.M - 1) * p.x_row + (int64_t)g * G);
+            const int gl = i / NT, t = i - gl * NT;
+            const uint4* src = p.xsm ? reinterpret_cast<const uint4*>(xt + t * xp + gl * G * 2)
+                                     : reinterpret_cast<const uint4*>(x + min(tok0 + t, p.M - 1) * p.x_row +
+                                                                      (int64_t)(cg0 + gl) * G);
             uint4 v[G / 8];
 #pragma unroll
             for (int u = 0; u < G / 8; ++u) v[u] = src[u];
@@ -354,7 +363,7 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
 #pragma unroll
         for (int mh = 0; mh < 4; ++mh) expand_row<BITS, BF, STEPS>(wv[mh], a[mh]);
 
-        const int kx2 = (g * G + sub * KS) * 2;   // byte offset of the sub-block in an x row
+        const int kx2 = ((g - (p.xsm ? cg0 : 0)) * G + sub * KS) * 2;   // sub-block's byte offset in an x row
 #pragma unroll
         for (int t = 0; t < NTL; ++t) {
             uint4 xv[XV];
@@ -377,7 +386,7 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
                 bv[mh] = half_bits_to_float(s_b[sb_row[mh] + g], XT{});
                 if (OFF != 0.0f) bv[mh] = fmaf(-OFF, sv[mh], bv[mh]);
             }
-            const float* xg = xs + g * NT + 2 * c;
+            const float* xg = xs + (g - cg0) * NT + 2 * c;
 #pragma unroll
             for (int t = 0; t < NTL; ++t) {
                 const float2 X = *reinterpret_cast<const float2*>(xg + 8 * t);
@@ -410,7 +419,8 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
     }
     __syncthreads();
 
-    // ---- sum the K slices in slice order and store pairs of adjacent outputs ----
+    // ---- sum the warps' K slices in slice order; without a cluster, store pairs of adjacent
+    // outputs; with one, keep the CTA's partial tile for the cluster-wide sum ----
     const int rpairs = p.wr * (ROWS / 2);
     const int total = NT * rpairs;
     const int64_t ybase = bo * p.yb[0] + bi * p.yb[1];
@@ -418,7 +428,7 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
         const int tt = i / rpairs, rp = i - tt * rpairs;
         const int wrr = rp / (ROWS / 2), rl = 2 * (rp % (ROWS / 2));
         const int64_t tok = tok0 + tt, n = rowc + wrr * ROWS + rl;
-        if (tok >= p.M || n >= p.N) continue;
+        if (cs == 1 && (tok >= p.M || n >= p.N)) continue;
         float v0 = 0.0f, v1 = 0.0f;
         for (int k = 0; k < p.wk; ++k) {
             const float* part = reinterpret_cast<const float*>(smem + (size_t)(k * p.wr + wrr) * RING_BYTES);
@@ -426,7 +436,33 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
             v0 += u.x;
             v1 += u.y;
         }
-        store_pair<XT>(p.y, ybase + tok * p.y_row + n, v0, v1, n + 1 < p.N, p.yvec != 0, p.ydt);
+        if (cs == 1) store_pair<XT>(p.y, ybase + tok * p.y_row + n, v0, v1, n + 1 < p.N, p.yvec != 0, p.ydt);
+        else *reinterpret_cast<float2*>(cpart + tt * rows_cta + wrr * ROWS + rl) = make_float2(v0, v1);
+    }
+    if (cs > 1) {
+        // every CTA's partial tile is complete and visible cluster-wide (hardware barrier)
+        asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+        // this CTA's share of the tile: the CTAs' partials added in rank order over distributed
+        // shared memory
+        const int per = (total + cs - 1) / cs;
+        const int i0 = rank * per, i1 = min(i0 + per, total);
+        const uint32_t cp_s = ptx::smem_u32(cpart);
+        for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
+            const int tt = i / rpairs, rp = i - tt * rpairs;
+            const int wrr = rp / (ROWS / 2), rl = 2 * (rp % (ROWS / 2));
+            const int64_t tok = tok0 + tt, n = rowc + wrr * ROWS + rl;
+            if (tok >= p.M || n >= p.N) continue;
+            const uint32_t off = (uint32_t)((tt * rows_cta + wrr * ROWS + rl) * 4);
+            float v0 = 0.0f, v1 = 0.0f;
+            for (int q = 0; q < cs; ++q) {
+                const float2 u = ptx::ld_cluster_f2(ptx::mapa(cp_s + off, (uint32_t)q));
+                v0 += u.x;
+                v1 += u.y;
+            }
+            store_pair<XT>(p.y, ybase + tok * p.y_row + n, v0, v1, n + 1 < p.N, p.yvec != 0, p.ydt);
+        }
+        // no CTA leaves while another may still read its partial tile
+        asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
     }
 }
 
@@ -454,11 +490,15 @@ cudaError_t launch_t(const WParams& p, dim3 grid, int warps, size_t smem, cudaSt
     cfg.blockDim = dim3(32 * warps);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;   // CTAs splitting K of one row block
+    attr[1].val.clusterDim.x = (unsigned)p.cs;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, qmm_warp_kernel<BITS, XT, G, NTL>, p);
 }
 

@@ -35,7 +35,7 @@ def _kernel(x, wq, sc, bi, group, bits):
 @pytest.mark.parametrize("bits", [2, 4, 8])
 @pytest.mark.parametrize("M,N,K", [(5, 129, 128), (8, 40, 256), (9, 1, 256), (13, 300, 384), (16, 1000, 1024),
                                    (17, 33, 512), (24, 4099, 1024), (32, 300, 1024), (16, 257, 3072),
-                                   (8, 5000, 4096)])
+                                   (8, 5000, 4096), (13, 300, 640), (32, 1000, 3072)])
 def test_warp_shapes(bits, M, N, K):
     group = 64
     w = inputs.normal((N, K), 0.02, seed=M * 5 + N + K + bits)
@@ -108,7 +108,8 @@ def test_warp_matches_other_kernels():
 
 def test_warp_kernel_choice():
     """Up to 16 rows always take the warp kernel; 32 rows take it while each warp has at most two
-    64-code sub-blocks of K (K = 1024 projections), the tcgen05 kernel otherwise."""
+    64-code sub-blocks of K once a cluster splits K (every decode projection), the tcgen05 kernel
+    otherwise (lm_head: many row blocks per CTA; large K with many row blocks)."""
     def kern(M, K, N):
         x = torch.empty((M, 1, K), dtype=torch.bfloat16, device=DEV)
         wq = torch.empty((N, K // 8), dtype=torch.int32, device=DEV)
@@ -116,7 +117,9 @@ def test_warp_kernel_choice():
         return _kernel(x, wq, s, s, 64, 4)
     assert kern(32, 1024, 2048) == "warp_mma"
     assert kern(32, 1024, 3072) == "warp_mma"
-    assert kern(32, 3072, 1024) == "tc_small_m"
+    assert kern(32, 3072, 1024) == "warp_mma"
+    assert kern(32, 2048, 1024) == "warp_mma"
+    assert kern(32, 8192, 4096) == "tc_small_m"
     assert kern(32, 1024, 151936) == "tc_small_m"
     assert kern(16, 3072, 1024) == "warp_mma"
     assert kern(8, 1024, 151936) == "warp_mma"
