@@ -121,9 +121,12 @@ aq_status aq_dequantize(const aq_view* wq, const aq_view* scales, const aq_view*
  * y:      x.shape[:-1] + [N], dtype of x or AQ_F32, must not overlap inputs.
  * bits in {2,3,4,5,6,8}; group in {32,64,128}; K % group == 0.
  * Rows per launch batch decide the kernel (aq_plan_linear reports it): up to 4
- * rows (or a batched W), a CUDA-core GEMV; 5..32 rows with 2/4/8-bit codes, a
- * warp-level mma.sync kernel that expands W in registers (2-bit codes need
- * groups of 64/128); other cases below 64 rows, a tcgen05/TMEM kernel on tiles
+ * rows (or a batched W), a CUDA-core GEMV; 5..32 rows in total with 2/4/8-bit
+ * codes (2-bit codes need groups of 64/128), where measured faster (always up
+ * to 16 rows; at 32 rows unless N is so large that a CTA holds many row
+ * blocks, or K per warp is long), a warp-level mma.sync kernel that expands W
+ * in registers, K split over a thread-block cluster when row blocks are few;
+ * other cases below 64 rows, a tcgen05/TMEM kernel on tiles
  * of 128 W rows x 32 tokens (K split over the CTAs of a thread-block cluster
  * when the tiles alone would leave most SMs idle); 64 rows and more with
  * groups of 64/128, a tcgen05 kernel on 128 x 128 tiles.  3/5-bit codes, K
