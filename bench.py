@@ -601,19 +601,24 @@ def reference(args):
     }), flush=True)
 
 
-CASES = ("lm_head_w4", "lm_head_w8", "lm_head2x_w4", "prefill_w4", "prefill_w8")
+CASES = ("lm_head_w4", "lm_head_w8", "lm_head2x_w4", "prefill_w4", "prefill_w8", "k_w4", "k_w8", "down_w4",
+         "down_w8")
 
 
 def single_case(name, reps):
     """One shape alone, for profiling: `reps` timed calls after two warm-up calls (CUDA events).
-    lm_head*: x [32, 1, 1024] against W [151936, 1024] (2x: 303872 rows, > L2); prefill*: x
-    [2, 2048, 4096] against W [14336, 4096]; G = 64, weights quantized on the device."""
+    lm_head*: x [32, 1, 1024] against W [151936, 1024] (2x: 303872 rows, > L2); k*, down*: x
+    [32, 1, K] against the decode step's k (W [1024, 1024]) or down (W [1024, 3072]) projection;
+    prefill*: x [2, 2048, 4096] against W [14336, 4096]; G = 64, weights quantized on the device."""
     from group_wise_affine_qmv_b200 import aq
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     bits = int(name[-1])
-    if name.startswith("lm_head"):
-        K, N = 1024, inputs.LM_HEAD[2] * (2 if name.startswith("lm_head2x") else 1)
+    if name.startswith(("lm_head", "k_", "down_")):
+        if name.startswith("lm_head"):
+            K, N = 1024, inputs.LM_HEAD[2] * (2 if name.startswith("lm_head2x") else 1)
+        else:
+            _, K, N = {p[0]: p for p in inputs.DECODE_PROJ}[name.split("_")[0]]
         x = inputs.decode_x(K, device=device)
         y = torch.empty(inputs.DECODE_BATCH, 1, N, dtype=torch.bfloat16, device=device)
         M = inputs.DECODE_BATCH
