@@ -35,7 +35,8 @@ def _kernel(x, wq, sc, bi, group, bits):
 @pytest.mark.parametrize("bits", [2, 4, 8])
 @pytest.mark.parametrize("M,N,K", [(5, 129, 128), (8, 40, 256), (9, 1, 256), (13, 300, 384), (16, 1000, 1024),
                                    (17, 33, 512), (24, 4099, 1024), (32, 300, 1024), (16, 257, 3072),
-                                   (8, 5000, 4096), (13, 300, 640), (32, 1000, 3072)])
+                                   (8, 5000, 4096), (13, 300, 640), (32, 1000, 3072),
+                                   (16, 4096, 8192)])   # x tile too large for shared memory: read through L1
 def test_warp_shapes(bits, M, N, K):
     group = 64
     w = inputs.normal((N, K), 0.02, seed=M * 5 + N + K + bits)
