@@ -122,10 +122,44 @@ def test_strided_rows_kept(lib):
 
 def test_regime_by_rows(lib):
     w = _weights(1024, 1024, 4, 64)
-    assert plan(torch.zeros(1, 1024, dtype=torch.bfloat16), *w, 64, 4)["regime"] == "qmv"
-    assert plan(torch.zeros(4, 1, 1024, dtype=torch.bfloat16), *w, 64, 4)["regime"] == "qmv"
+    for x in (torch.zeros(1, 1024, dtype=torch.bfloat16), torch.zeros(4, 1, 1024, dtype=torch.bfloat16)):
+        p = plan(x, *w, 64, 4)
+        assert p["regime"] == "qmv" and p["kernel"] == "gemv"
     # forced GEMV whatever the size
-    assert plan(torch.zeros(32, 1, 1024, dtype=torch.bfloat16), *w, 64, 4, force_qmv=True)["regime"] == "qmv"
+    p = plan(torch.zeros(32, 1, 1024, dtype=torch.bfloat16), *w, 64, 4, force_qmv=True)
+    assert p["regime"] == "qmv" and p["kernel"] == "gemv"
+
+
+def test_plan_struct_layout(lib, tmp_path):
+    """The ctypes mirrors of aq_plan and aq_view match the C declarations in include/aq.h field by
+    field (sizes and offsets printed by a C program compiled against the header)."""
+    import ctypes
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    structs = [("aq_plan", aq.AqPlan), ("aq_view", aq.AqView)]
+    body = ""
+    for cname, cls in structs:
+        body += f'  printf("%zu\\n", sizeof({cname}));\n'
+        body += "".join(f'  printf("%zu\\n", offsetof({cname}, {f[0]}));\n' for f in cls._fields_)
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"aq.h\"\nint main(void) {\n" + body +
+                   "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = [int(v) for v in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
+    expect = []
+    for _, cls in structs:
+        expect += [ctypes.sizeof(cls)] + [getattr(cls, f[0]).offset for f in cls._fields_]
+    assert out == expect
+    assert aq.AqPlan.kernel.offset == aq.AqPlan.nbatch_dims.offset + 4
+    assert set(aq.KERNEL_NAMES.values()) == {"gemv", "warp_mma", "tc_small_m", "tc_prefill"}
+    hdr = open(os.path.join(ROOT, "include", "aq.h")).read()
+    for name, value in (("AQ_KERNEL_GEMV", 0), ("AQ_KERNEL_WARP_MMA", 1), ("AQ_KERNEL_TC_SMALL_M", 2),
+                        ("AQ_KERNEL_TC_PREFILL", 3)):
+        assert f"{name} = {value}" in hdr
 
 
 @pytest.mark.parametrize("case,status", [
