@@ -87,16 +87,9 @@ def main(argv=None):
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-v", action="store_true", help="print register/smem usage per kernel")
-    ap.add_argument("--trace", metavar="OUT",
-                    help="build a tracing variant (-DAQ_TRACE: per-wait-site time counters, aq_trace_read) into OUT")
     args = ap.parse_args(argv)
     extra = ["-Xptxas", "-v"] if args.ptxas_v else []
-    if args.trace:
-        out = os.path.abspath(args.trace)
-        path = build(force=args.force, verbose=args.verbose, extra_flags=extra + ["-DAQ_TRACE"], out=out,
-                     build_dir=os.path.join(BUILD, "trace"))
-    else:
-        path = build(force=args.force or args.ptxas_v, verbose=args.verbose or args.ptxas_v, extra_flags=extra)
+    path = build(force=args.force or args.ptxas_v, verbose=args.verbose or args.ptxas_v, extra_flags=extra)
     print(path)
 
 

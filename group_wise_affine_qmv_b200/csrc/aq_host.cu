@@ -84,6 +84,31 @@ bool overlaps(const aq_view* a, const aq_view* b) {
     return alo < bhi && blo < ahi;
 }
 
+// Whether two different indices of an output view reach the same element (a zero stride on a
+// dimension of extent > 1, as an expand()ed tensor has, or strides too small for the extents
+// inside them): several threads would then race on one element.  Dimensions are visited from the
+// smallest stride up; each stride must exceed the largest offset the dimensions below it reach.
+bool self_overlapping(const aq_view* v) {
+    int idx[4];
+    int n = 0;
+    for (int i = 0; i < v->rank; ++i)
+        if (v->shape[i] > 1) idx[n++] = i;
+    std::sort(idx, idx + n, [&](int a, int b) { return v->stride[a] < v->stride[b]; });
+    int64_t reach = 0;
+    for (int j = 0; j < n; ++j) {
+        const int i = idx[j];
+        if (v->stride[i] <= reach) return true;
+        reach += (v->shape[i] - 1) * v->stride[i];
+    }
+    return false;
+}
+
+aq_status check_output(const aq_view* v, const char* name) {
+    if (numel(v) > 0 && self_overlapping(v))
+        return fail(AQ_ERR_OVERLAP, "%s: elements overlap (zero or too small stride)", name);
+    return AQ_OK;
+}
+
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 aq_status check_bits_group(int bits, int group) {
@@ -141,6 +166,7 @@ aq_status resolve_linear(const aq_view* x, const aq_view* wq, const aq_view* sc,
     if ((st = check_view(sc, "scales", 2, 4)) != AQ_OK) return st;
     if ((st = check_view(bi, "biases", 2, 4)) != AQ_OK) return st;
     if ((st = check_view(y, "y", 1, 4)) != AQ_OK) return st;
+    if ((st = check_output(y, "y")) != AQ_OK) return st;
     if ((st = check_bits_group(bits, group)) != AQ_OK) return st;
     if (!is_half(x->dtype)) return fail(AQ_ERR_DTYPE, "x must be bf16 or f16");
     if (wq->dtype != AQ_U32) return fail(AQ_ERR_DTYPE, "wq must be u32");
@@ -375,6 +401,13 @@ aq_status check_quant_views(const aq_view* w, int group, int bits, const aq_view
     const aq_view* out = w_is_output ? w : wq;
     const aq_view* ins[3] = {w_is_output ? wq : w, sc, bi};
     if (w_is_output) {
+        if ((st = check_output(w, "w_out")) != AQ_OK) return st;
+    } else {
+        if ((st = check_output(wq, "wq")) != AQ_OK) return st;
+        if ((st = check_output(sc, "scales")) != AQ_OK) return st;
+        if ((st = check_output(bi, "biases")) != AQ_OK) return st;
+    }
+    if (w_is_output) {
         for (const aq_view* v : ins)
             if (overlaps(out, v)) return fail(AQ_ERR_OVERLAP, "w_out overlaps an input");
     } else {
@@ -500,6 +533,7 @@ AQ_API aq_status aq_qmm_t_grouped(const aq_view* x_sorted, const int64_t* offset
     if ((st = check_view(s_bank, "s_bank", 3, 3)) != AQ_OK) return st;
     if ((st = check_view(b_bank, "b_bank", 3, 3)) != AQ_OK) return st;
     if ((st = check_view(y_sorted, "y_sorted", 2, 2)) != AQ_OK) return st;
+    if ((st = check_output(y_sorted, "y_sorted")) != AQ_OK) return st;
     if ((st = check_bits_group(bits, group)) != AQ_OK) return st;
     if (!offsets) return fail(AQ_ERR_NULL, "offsets is NULL");
     if (n_experts <= 0 || wq_bank->shape[0] != n_experts || s_bank->shape[0] != n_experts ||

@@ -18,12 +18,6 @@ namespace aq {
 // aq_device_error().  Kernels receive its address in their parameters.
 __device__ int g_device_error = 0;
 
-#if defined(AQ_TRACE) || defined(AQ_TIMELINE)
-// instrumented builds: per-site counters and the CTA-0 event timeline
-__device__ unsigned long long g_trace[64];
-__device__ long long g_timeline[16 * 512];
-#endif
-
 namespace {
 
 using namespace mma;
@@ -71,11 +65,7 @@ cudaError_t symbol_address(const T& sym, void** cache, void** out) {
     return cudaSuccess;
 }
 
-#ifdef AQ_TRACE
-constexpr size_t SMEM_LIMIT = 226 * 1024;  // the trace counters take static shared memory
-#else
 constexpr size_t SMEM_LIMIT = 227 * 1024;
-#endif
 constexpr int MIN_STAGES = 3;
 
 struct Geom {
@@ -239,16 +229,6 @@ cudaError_t device_pointers(Params& prm) {
     cudaError_t e = symbol_address(g_device_error, cache, &a);
     if (e != cudaSuccess) return e;
     prm.err = static_cast<int*>(a);
-#if defined(AQ_TRACE) || defined(AQ_TIMELINE)
-    static void* cache_t[64] = {nullptr};
-    static void* cache_l[64] = {nullptr};
-    e = symbol_address(g_trace, cache_t, &a);
-    if (e != cudaSuccess) return e;
-    prm.trace = static_cast<unsigned long long*>(a);
-    e = symbol_address(g_timeline, cache_l, &a);
-    if (e != cudaSuccess) return e;
-    prm.tl = static_cast<long long*>(a);
-#endif
     return cudaSuccess;
 }
 
@@ -360,24 +340,6 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     }
     return cudaErrorInvalidValue;
 }
-
-#ifdef AQ_TRACE
-extern "C" __attribute__((visibility("default"))) int aq_trace_read(unsigned long long* out, int reset) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-    if (cudaMemcpyFromSymbol(out, g_trace, sizeof(unsigned long long) * 64) != cudaSuccess) return -1;
-    if (reset) {
-        unsigned long long z[64] = {0};
-        if (cudaMemcpyToSymbol(g_trace, z, sizeof z) != cudaSuccess) return -1;
-    }
-    return 0;
-}
-#endif
-#ifdef AQ_TIMELINE
-extern "C" __attribute__((visibility("default"))) int aq_tl_read(long long* out) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-    return cudaMemcpyFromSymbol(out, g_timeline, sizeof(long long) * 16 * 512) == cudaSuccess ? 0 : -1;
-}
-#endif
 
 cudaError_t read_and_clear_device_error(int* value, cudaStream_t s) {
     cudaError_t e = cudaStreamSynchronize(s);

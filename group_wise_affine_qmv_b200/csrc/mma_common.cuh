@@ -69,8 +69,6 @@ struct Params {
     int n_experts;
     int ksplit;                  // CTAs per cluster splitting each tile's K (1: no split)
     int* err;                    // device error word (set on a timed-out wait)
-    unsigned long long* trace;   // instrumented builds only: per-site counters [64]
-    long long* tl;               // instrumented builds only: event timeline [16][512]
 };
 
 // W stages [w0, w1) of the tile handled by rank `rank` of `cs` CTAs splitting K.  Ranges

@@ -53,26 +53,18 @@
 namespace aq {
 namespace mma {
 
-#ifdef AQ_TRACE
-// trace builds: clock cycles of a section, per warp, into the per-site counters
-#define AQ_TSTART(v) const long long v = clock64()
-#define AQ_TSTOP(site, v) AQ_TRACE_ADD(site, clock64() - (v))
-#else
-#define AQ_TSTART(v)
-#define AQ_TSTOP(site, v)
-#endif
-#ifdef AQ_TIMELINE
-// timeline builds: clock64 of events in CTAs 0 and 1, relative to each CTA's start
-#define AQ_TL(ev, idx, cond)                                                                         \
-    do {                                                                                             \
-        if (blockIdx.x < 2 && (cond) && (idx) >= 0 && (idx) < 256)                                   \
-            p.tl[(ev) * 512 + 256 * blockIdx.x + (idx)] = clock64() - tl0;                             \
-    } while (0)
-#else
-#define AQ_TL(ev, idx, cond)
-#endif
-
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+// Grouped mode: rows [*off, *off + *cnt) of x_sorted / y_sorted belong to expert e.  The device
+// offsets are clamped into [0, M] and each end to at least its start, so no offsets array, however
+// malformed, makes a CTA read or write a row outside the M rows of the call.
+__device__ __forceinline__ void expert_rows(const Params& p, int e, int64_t* off, int64_t* cnt) {
+    const int64_t lo = min64(max64(p.offsets[e], 0), p.M);
+    const int64_t hi = min64(max64(p.offsets[e + 1], lo), p.M);
+    *off = lo;
+    *cnt = hi - lo;
+}
 
 struct TileInfo {
     int64_t wrow0;   // first W row of the tile in the W tensor (expert offset included)
@@ -162,7 +154,8 @@ __device__ __forceinline__ TileInfo tile_info(const Params& p, const Smem& s, in
         const int e = lo;
         const int local = t - s.prefix[e];
         const int wt = local % p.n_wtiles, tt = local / p.n_wtiles;
-        const int64_t off = p.offsets[e], cnt = p.offsets[e + 1] - off;
+        int64_t off, cnt;
+        expert_rows(p, e, &off, &cnt);
         ti.n0 = (int64_t)wt * 128;
         ti.wrow0 = (int64_t)e * p.N + ti.n0;
         ti.nvalid = (int)min64(128, p.N - ti.n0);
@@ -405,17 +398,10 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
     const int cs = p.ksplit;   // CTAs of a cluster splitting each tile's K (1: none)
     const Smem s = carve<SUB, ROWB, GPS>(base, p, cs > 1 ? split_max_stages(NWS, GPS, cs) : NWS);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    AQ_TSTART(t_kernel);
-#ifdef AQ_TIMELINE
-    const long long tl0 = clock64();
-#endif
     const int S = p.stages;
     const int KBLK = (int)(p.K / KB);
     const int NG = p.kg;
 
-#ifdef AQ_TRACE
-    if (threadIdx.x < 64) aq_trace_smem[threadIdx.x] = 0;
-#endif
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
             ptx::mbar_init(&s.wfull[i], 1);
@@ -462,7 +448,8 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
             const int e = e0 + lane;
             int v = 0;
             if (e < p.n_experts) {
-                const int64_t cnt = p.offsets[e + 1] - p.offsets[e];
+                int64_t off, cnt;
+                expert_rows(p, e, &off, &cnt);
                 v = (int)((cnt + NT - 1) / NT) * p.n_wtiles;
             }
 #pragma unroll
@@ -493,8 +480,6 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
     if (cs > 1) split_range(NWS, GPS, cs, rank, &w0, &w1);
     const int g_lo = w0 * GPS, g_hi = min(w1 * GPS, NG);
     const bool has_tiles = tile0 < ntiles;
-    if (warp == 1) AQ_TSTOP(15, t_kernel);
-    AQ_TL(10, 1, threadIdx.x == 32);
 
     if (warp == 0) {
         // ======================= W producer =======================
@@ -506,7 +491,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
             const TileInfo ti = tile_info(p, s, t);
             for (int w = w0; w < w1; ++w) {
                 const int st = wg % S;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfree[st], ((wg / S) & 1) ^ 1, s.abort, WAIT_NS, 0));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfree[st], ((wg / S) & 1) ^ 1, s.abort, WAIT_NS));
                 if (!ok) break;
                 if (leader) {
                     // columns past K (a partial last stage) read as zero fill
@@ -514,7 +499,6 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                     ptx::tma_load_2d(s.ws + (size_t)st * 128 * ROWB, &p.tw, &s.wfull[st], w * (ROWB / 4),
                                      (int32_t)ti.wrow0);
                 }
-                AQ_TL(0, wg, leader);
                 ++wg;
             }
         }
@@ -533,7 +517,6 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         uint32_t wg = 0;
         if (p.xres) {
             if (has_tiles && leader) {
-                // the CTA's only token tile: all of K, once
                 // the CTA's only token tile: its K range, once
                 const TileInfo t0 = tile_info(p, s, tile0);
                 const int kb0 = w0 * SUB, kb1 = min(w1 * SUB, KBLK);
@@ -551,7 +534,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 for (int w = w0; w < w1; ++w) {
                     const int xs = wg % XS;
                     ok = __all_sync(0xffffffffu,
-                                    ptx::mbar_wait(&s.xfree[xs], ((wg / XS) & 1) ^ 1, s.abort, WAIT_NS, 9));
+                                    ptx::mbar_wait(&s.xfree[xs], ((wg / XS) & 1) ^ 1, s.abort, WAIT_NS));
                     if (!ok) break;
                     if (leader) {
                         const int nsub = min(SUB, KBLK - w * SUB);
@@ -578,7 +561,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         const bool leader = lane == 0;
         uint32_t wg = 0;
         bool ok = true;
-        if (p.xres && has_tiles) ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xres_full, 0, s.abort, WAIT_NS, 1));
+        if (p.xres && has_tiles) ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xres_full, 0, s.abort, WAIT_NS));
         for (int t = tile0; t < ntiles && ok; t += tstep) {
             for (int w = w0; w < w1; ++w, ++wg) {
                 const int slot = wg & 1;
@@ -586,18 +569,15 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 const int xs = p.xres ? 0 : (int)(wg % (uint32_t)p.xst);
                 if (!p.xres) {
                     ok = __all_sync(0xffffffffu,
-                                    ptx::mbar_wait(&s.xfull[xs], (wg / p.xst) & 1, s.abort, WAIT_NS, 1));
+                                    ptx::mbar_wait(&s.xfull[xs], (wg / p.xst) & 1, s.abort, WAIT_NS));
                     if (!ok) break;
                 }
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.afull[slot], ph, s.abort, WAIT_NS, 2));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.afull[slot], ph, s.abort, WAIT_NS));
                 if (!ok) break;
-                AQ_TL(4, wg, leader);
                 // the folds have read this slot's accumulators (stage wg - 2)
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.dfree[slot], ph ^ 1, s.abort, WAIT_NS, 3));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.dfree[slot], ph ^ 1, s.abort, WAIT_NS));
                 if (!ok) break;
-                AQ_TL(13, wg, leader);
                 ptx::tc_fence_after();
-                AQ_TSTART(t_issue);
                 if (leader) {
                     const uint32_t a_blk = tbase + (uint32_t)(slot * ACOLS);
                     const uint32_t d_blk = d_tmem + (uint32_t)(slot * GPS * NT);
@@ -624,8 +604,6 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                     if (!p.xres) ptx::mma_commit(&s.xfree[xs]);
                 }
                 __syncwarp();
-                AQ_TSTOP(12, t_issue);
-                AQ_TL(5, wg, leader);
             }
         }
         if (!ok && leader) raise_abort(p, s.abort);
@@ -649,10 +627,8 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         for (int t = tile0; t < ntiles && ok; t += tstep) {
             for (int w = w0; w < w1; ++w, ++wg) {
                 const int st = wg % S;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfull[st], (wg / S) & 1, s.abort, WAIT_NS, 4));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfull[st], (wg / S) & 1, s.abort, WAIT_NS));
                 if (!ok) break;
-                AQ_TSTART(t_exp);
-                AQ_TL(1, wg, threadIdx.x == 64);
                 // expand the whole stage into registers while the MMAs of stage wg - 2 may still
                 // be reading A block wg % 2
                 const uint8_t* wstage = s.ws + (size_t)st * 128 * ROWB;
@@ -668,11 +644,10 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 }
                 if (wg >= 2) {
                     ok = __all_sync(0xffffffffu,
-                                    ptx::mbar_wait(&s.sdone[wg & 1], ((wg >> 1) & 1) ^ 1, s.abort, WAIT_NS, 5));
+                                    ptx::mbar_wait(&s.sdone[wg & 1], ((wg >> 1) & 1) ^ 1, s.abort, WAIT_NS));
                     if (!ok) break;
                     ptx::tc_fence_after();
                 }
-                AQ_TL(11, wg, threadIdx.x == 64);
                 const uint32_t a_blk = tbase + lane_base + (uint32_t)((wg & 1) * ACOLS);
 #pragma unroll
                 for (int j = 0; j < SUB; ++j)
@@ -684,9 +659,6 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                     ptx::mbar_arrive(&s.wfree[st]);
                     ptx::mbar_arrive(&s.afull[wg & 1]);
                 }
-                AQ_TSTOP(10, t_exp);
-                AQ_TL(2, wg, threadIdx.x == 64);
-                AQ_TL(3, wg, threadIdx.x == 192);
             }
         }
         if (!ok) raise_abort(p, s.abort);
@@ -716,22 +688,21 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
 
         for (int t = tile0; t < ntiles && ok; t += tstep) {
             const TileInfo ti = tile_info(p, s, t);
-            AQ_TL(8, (t - (int)blockIdx.x) / (int)gridDim.x, threadIdx.x == 320);
             if (ti.xrow0 != cur_x0 || ti.b0 != cur_b0 || ti.b1 != cur_b1 || ti.tvalid != cur_tv) {
                 // sums of x for this token tile
                 ptx::mbar_arrive(s.xbar);  // everyone is done reading the previous table
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_NS, 8));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_NS));
                 ++xph;
                 if (!ok) break;
                 if (p.xres) {
-                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xres_full, 0, s.abort, WAIT_NS, 8));
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xres_full, 0, s.abort, WAIT_NS));
                     if (!ok) break;
                     build_xtab_smem<XT, G>(g_hi - g_lo, s.xs, s.xtab, tid);
                 } else {
                     build_xtab<XT, G>(p, ti, g_lo, g_hi, s.xtab, tid);
                 }
                 ptx::mbar_arrive(s.xbar);
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_NS, 8));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_NS));
                 ++xph;
                 if (!ok) break;
                 cur_x0 = ti.xrow0;
@@ -748,7 +719,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                     ptx::cp_async_wait_all();
                     ptx::mbar_arrive(&s.sbar[unit & 1]);
                     ok = __all_sync(0xffffffffu,
-                                    ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS, 7));
+                                    ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS));
                     if (!ok) break;
                     sbslot = s.sb + (unit & 1) * 2 * 128 * SCP;
                     g_chunk0 = g_lo + ((w - w0) / CS_W) * SCW;
@@ -763,11 +734,9 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                     ++unit;
                 }
                 const int slot = wg & 1;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.sdone[slot], (wg >> 1) & 1, s.abort, WAIT_NS, 6));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.sdone[slot], (wg >> 1) & 1, s.abort, WAIT_NS));
                 if (!ok) break;
                 ptx::tc_fence_after();
-                AQ_TL(6, wg, threadIdx.x == 320);
-                AQ_TSTART(t_epi);
 #pragma unroll
                 for (int lg = 0; lg < GPS; ++lg) {
                     const int g = w * GPS + lg;
@@ -796,8 +765,6 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&s.dfree[slot]);
-                AQ_TSTOP(11, t_epi);
-                AQ_TL(7, wg, threadIdx.x == 320);
             }
             if (!ok) break;
             if (cs > 1) {
@@ -835,7 +802,6 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 break;   // one tile per cluster
             }
             // ---- this thread's row of y for its half of the tokens ----
-            AQ_TSTART(t_store);
             if (row < ti.nvalid) {
                 const int64_t n = ti.n0 + row;
                 int64_t off = ti.xrow0 * p.y_row + n;
@@ -847,14 +813,10 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                     if (tok + 1 < ti.tvalid) store_y(p.y, off + (int64_t)(tok + 1) * p.y_row, acc[i].y, p.ydt, XT{});
                 }
             }
-            AQ_TSTOP(13, t_store);
-            AQ_TL(9, (t - (int)blockIdx.x) / (int)gridDim.x, threadIdx.x == 320);
         }
         ptx::cp_async_wait_all();
         if (!ok) raise_abort(p, s.abort);
     }
-    if (warp == 1) AQ_TSTOP(14, t_kernel);
-    if (warp == 2) AQ_TSTOP(16, t_kernel);
 
     ptx::tc_fence_before();
     __syncthreads();
@@ -862,19 +824,12 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tbase, p.tmem_cols);
     }
-#ifdef AQ_TRACE
-    if (threadIdx.x < 64) atomicAdd(&p.trace[threadIdx.x], aq_trace_smem[threadIdx.x]);
-#endif
 }
 
 // ---------------------------------------------------------------------------
 // launch (per device: raise the dynamic shared memory limit once)
 // ---------------------------------------------------------------------------
-#ifdef AQ_TRACE
-constexpr size_t SMEM_LIMIT = 226 * 1024;  // the trace counters take static shared memory
-#else
 constexpr size_t SMEM_LIMIT = 227 * 1024;
-#endif
 
 template <int BITS, typename XT, int G>
 cudaError_t launch_t(const Params& prm, int grid, size_t smem, cudaStream_t s) {

@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
             const PTile ti = p_tile(p, t);
             for (int w = 0; w < NWS; ++w, ++wg) {
                 const int st = wg % S;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfree[st], ((wg / S) & 1) ^ 1, s.abort, WAIT_NS, 0));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfree[st], ((wg / S) & 1) ^ 1, s.abort, WAIT_NS));
                 if (!ok) break;
                 if (leader) {
                     ptx::mbar_arrive_expect_tx(&s.wfull[st], 128u * ROWB);
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
             const PTile ti = p_tile(p, t);
             for (int w = 0; w < NWS; ++w, ++wg) {
                 const int xs = wg % XS;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.xfree[xs], ((wg / XS) & 1) ^ 1, s.abort, WAIT_NS, 9));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.xfree[xs], ((wg / XS) & 1) ^ 1, s.abort, WAIT_NS));
                 if (!ok) break;
                 if (leader) {
                     ptx::mbar_arrive_expect_tx(&s.xfull[xs], (uint32_t)SUB * NTP * 128);
@@ -227,11 +227,11 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
                 const int slot = wg & 1;
                 const uint32_t ph = (wg >> 1) & 1;
                 const int xs = wg % XS;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.xfull[xs], (wg / XS) & 1, s.abort, WAIT_NS, 1));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.xfull[xs], (wg / XS) & 1, s.abort, WAIT_NS));
                 if (!ok) break;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.afull[slot], ph, s.abort, WAIT_NS, 2));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.afull[slot], ph, s.abort, WAIT_NS));
                 if (!ok) break;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.dfree[slot], ph ^ 1, s.abort, WAIT_NS, 3));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.dfree[slot], ph ^ 1, s.abort, WAIT_NS));
                 if (!ok) break;
                 ptx::tc_fence_after();
                 if (leader) {
@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             for (int w = 0; w < NWS; ++w, ++wg) {
                 const int st = wg % S;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfull[st], (wg / S) & 1, s.abort, WAIT_NS, 4));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfull[st], (wg / S) & 1, s.abort, WAIT_NS));
                 if (!ok) break;
                 const uint8_t* wstage = s.ws + (size_t)st * 128 * ROWB;
                 uint32_t out[2 * SUB][16];
@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
                 }
                 if (wg >= 2) {
                     ok = __all_sync(0xffffffffu,
-                                    ptx::mbar_wait(&s.sdone[wg & 1], ((wg >> 1) & 1) ^ 1, s.abort, WAIT_NS, 5));
+                                    ptx::mbar_wait(&s.sdone[wg & 1], ((wg >> 1) & 1) ^ 1, s.abort, WAIT_NS));
                     if (!ok) break;
                     ptx::tc_fence_after();
                 }
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
                     ptx::cp_async_wait_all();
                     ptx::mbar_arrive(&s.sbar[unit & 1]);
                     ok = __all_sync(0xffffffffu,
-                                    ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS, 7));
+                                    ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS));
                     if (!ok) break;
                     sbslot = s.sb + (unit & 1) * 2 * 128 * SCP;
                     g_chunk0 = w;
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
                 const int slot = wg & 1;
                 const int xs = wg % XS;
                 // the MMAs of this stage are complete: its x block and accumulator are final
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.sdone[slot], (wg >> 1) & 1, s.abort, WAIT_NS, 6));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.sdone[slot], (wg >> 1) & 1, s.abort, WAIT_NS));
                 if (!ok) break;
                 ptx::tc_fence_after();
                 // ---- X_g of the stage's 128 tokens: thread pair (2t, 2t+1) sums token t's codes,
@@ -364,7 +364,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
                     if (half == 0) s.xg[slot * NTP + tok] = sum + other;
                 }
                 ptx::mbar_arrive(&s.xgbar[slot]);
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.xgbar[slot], (wg >> 1) & 1, s.abort, WAIT_NS, 8));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.xgbar[slot], (wg >> 1) & 1, s.abort, WAIT_NS));
                 if (!ok) break;
                 if (lane == 0) ptx::mbar_arrive(&s.xfree[xs]);   // x block read by this warp
                 // ---- y += s * D' + (b - OFF*s) * X_g ----

@@ -8,10 +8,6 @@
 #include <cuda.h>
 #include <stdint.h>
 
-#ifdef AQ_TRACE
-static __shared__ unsigned long long aq_trace_smem[64];   // per-CTA accumulation, flushed at exit
-#endif
-
 namespace aq {
 namespace ptx {
 
@@ -70,28 +66,13 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_
     return ok != 0;
 }
 
-#ifdef AQ_TRACE
-// Trace builds only: nanoseconds spent (lane 0 of each waiting warp) and number of
-// waits per wait site, accumulated over all CTAs; read back with aq_trace_read().
-#define AQ_TRACE_ADD(site, ns)                                         \
-    do {                                                               \
-        if ((threadIdx.x & 31) == 0) {                                 \
-            atomicAdd(&::aq_trace_smem[(site)], (unsigned long long)(ns)); \
-            atomicAdd(&::aq_trace_smem[32 + (site)], 1ull);              \
-        }                                                              \
-    } while (0)
-#endif
-
 // Wait for the phase of parity `parity` to complete.  Returns false if the
 // budget ran out or *abort became non-zero (another warp gave up).  The budget is
 // counted in SM clock cycles (clock64, cheap to read; at most ~2 GHz, so
 // 2 cycles per nanosecond of budget never undercounts the wall time).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint64_t budget_ns, int site = -1) {
+                                          uint64_t budget_ns) {
     const uint32_t a = smem_u32(bar);
-#ifdef AQ_TRACE
-    const uint64_t tt0 = globaltimer_ns();
-#endif
     bool done = mbar_try_wait(a, parity);
     if (!done) {
         const long long c0 = clock64();
@@ -101,11 +82,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
             if ((i & 63u) == 0 && (*abort || clock64() - c0 > limit)) break;
         }
     }
-#ifdef AQ_TRACE
-    if (site >= 0) AQ_TRACE_ADD(site, globaltimer_ns() - tt0);
-#else
-    (void)site;
-#endif
     return done;
 }
 
@@ -211,7 +187,6 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
 
 // D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16 (bf16/f16 inputs, fp32 accumulate); the accumulate
 // flag is an immediate (ACC = 0: D = A.B, 1: D += A.B)

@@ -59,7 +59,7 @@ typedef enum aq_status {
     AQ_ERR_GROUP = 7,        /* group not in {32, 64, 128}, or K % group != 0        */
     AQ_ERR_ALIGN = 8,        /* a data pointer is not 16-byte aligned                */
     AQ_ERR_UNSUPPORTED = 9,  /* valid request the library does not implement         */
-    AQ_ERR_OVERLAP = 10,     /* the output overlaps an input                         */
+    AQ_ERR_OVERLAP = 10,     /* the output overlaps an input or itself               */
     AQ_ERR_CUDA = 11,        /* a CUDA runtime/driver call or a launch failed        */
     AQ_ERR_DEVICE = 12,      /* current device is not an sm_100 (B200-class) GPU     */
     AQ_ERR_TIMEOUT = 13      /* a kernel's bounded pipeline wait expired (device)    */
@@ -94,6 +94,7 @@ typedef struct aq_view {
  * w:      [N, K] AQ_F32, AQ_BF16 or AQ_F16 (rank 2; rows may be strided).
  * wq:     [N, K*bits/32] AQ_U32 out, packed as described at the top.
  * scales: [N, K/group] AQ_BF16 or AQ_F16 out; biases: same shape and dtype.
+ * The outputs must not overlap the input, each other, or themselves.
  * W must be finite; NaN/Inf inputs give unspecified codes.
  */
 aq_status aq_quantize(const aq_view* w, int group, int bits, const aq_view* wq,
@@ -118,7 +119,9 @@ aq_status aq_dequantize(const aq_view* wq, const aq_view* scales, const aq_view*
  *         (shared weight) or equal to x's corresponding batch dims
  *         (right-aligned, as in broadcasting).
  * scales, biases: [..., N, K/group], same dtype as x, same batch dims as wq.
- * y:      x.shape[:-1] + [N], dtype of x or AQ_F32, must not overlap inputs.
+ * y:      x.shape[:-1] + [N], dtype of x or AQ_F32, must not overlap inputs, and no two
+ *         of its elements may share an address (a zero stride on a dimension of extent
+ *         > 1 is AQ_ERR_OVERLAP).
  * bits in {2,3,4,5,6,8}; group in {32,64,128}; K % group == 0.
  * Rows per launch batch decide the kernel (aq_plan_linear reports it): up to 4
  * rows (or a batched W), a CUDA-core GEMV; 5..32 rows in total with 2/4/8-bit
@@ -155,7 +158,10 @@ aq_status aq_qmv(const aq_view* x, const aq_view* wq, const aq_view* scales,
  *   y_sorted[t] = x_sorted[t] . dequant(W_e)^T  for offsets[e] <= t < offsets[e+1].
  * x_sorted: [T, K] AQ_BF16|AQ_F16 (rows grouped by expert, row stride free).
  * offsets:  DEVICE pointer to n_experts+1 int64, non-decreasing, offsets[0] = 0,
- *           offsets[n_experts] = T (not checked on the host: it lives on the device).
+ *           offsets[n_experts] = T.  The host cannot check it (it lives on the device);
+ *           the kernel clamps every expert's range into [0, T) (an end below its start is
+ *           an empty expert), so a malformed array gives wrong rows but never an access
+ *           outside x_sorted / y_sorted.
  * wq_bank [E, N, K*bits/32] AQ_U32; s_bank, b_bank [E, N, K/group].
  * y_sorted: [T, N], dtype of x or AQ_F32.
  * (Prior art: the gathered QMV of "mlx PR #4516"; expert shapes from "Metal

@@ -166,7 +166,8 @@ def test_plan_struct_layout(lib, tmp_path):
     ("bits", "AQ_ERR_BITS"), ("group", "AQ_ERR_GROUP"), ("kmod", "AQ_ERR_GROUP"), ("wshape", "AQ_ERR_SHAPE"),
     ("sshape", "AQ_ERR_SHAPE"), ("ydtype", "AQ_ERR_DTYPE"), ("sdtype", "AQ_ERR_DTYPE"), ("xdtype", "AQ_ERR_DTYPE"),
     ("stride", "AQ_ERR_STRIDE"), ("yshape", "AQ_ERR_SHAPE"), ("overlap", "AQ_ERR_OVERLAP"), ("rank", "AQ_ERR_RANK"),
-    ("wbatch", "AQ_ERR_SHAPE"), ("align", "AQ_ERR_ALIGN"),
+    ("wbatch", "AQ_ERR_SHAPE"), ("align", "AQ_ERR_ALIGN"), ("yexpand", "AQ_ERR_OVERLAP"),
+    ("yrows", "AQ_ERR_OVERLAP"), ("ybatch0", "AQ_ERR_OVERLAP"),
 ])
 def test_validation_errors(lib, case, status):
     K, N, G, B = 256, 64, 64, 4
@@ -210,6 +211,13 @@ def test_validation_errors(lib, case, status):
         wq, sc, bi = _weights(N, K, B, G, batch=(3,))
     elif case == "align":
         wq = torch.zeros(N * (K * B // 32) + 1, dtype=torch.int32)[1:].view(N, K * B // 32)
+    elif case == "yexpand":     # an expand()ed y: both rows are the same memory
+        y = torch.empty(1, N, dtype=torch.bfloat16).expand(2, N)
+    elif case == "yrows":       # row stride smaller than the row: rows overlap
+        y = torch.empty(2 * N, dtype=torch.bfloat16).as_strided((2, N), (N // 2, 1))
+    elif case == "ybatch0":     # a batch dim of stride 0 on a 3D y
+        x = torch.zeros(3, 2, K, dtype=torch.bfloat16)
+        y = torch.empty(1, 2, N, dtype=torch.bfloat16).expand(3, 2, N)
     with pytest.raises(aq.AQError) as ei:
         aq.aq_plan_linear(x, wq, sc, bi, group, bits, y)
     assert ei.value.name == status, (case, str(ei.value))
@@ -220,3 +228,28 @@ def test_empty_inputs_plan(lib):
     w = _weights(64, 256, 4, 64)
     p = plan(x, *w, 64, 4)
     assert p["total_rows"] == 0
+
+
+def test_output_self_overlap_rejected_everywhere(lib):
+    """No output view may alias itself: quantize's outputs, dequantize's output and the grouped
+    entry's y_sorted are checked like aq_qmm_t's y (before anything would launch)."""
+    K, N, G, B = 256, 64, 64, 4
+    w = torch.zeros(N, K, dtype=torch.float32)
+    wq, sc, bi = _weights(N, K, B, G)
+    lib_ = aq.load_library()
+    bad_sc = torch.zeros(1, K // G, dtype=torch.bfloat16).expand(N, K // G)
+    st = lib_.aq_quantize(aq.view(w), G, B, aq.view(wq), aq.view(bad_sc), aq.view(bi), None)
+    assert lib_.aq_status_string(st) == b"AQ_ERR_OVERLAP"
+    bad_w = torch.zeros(1, K, dtype=torch.float32).expand(N, K)
+    st = lib_.aq_dequantize(aq.view(wq), aq.view(sc), aq.view(bi), G, B, aq.view(bad_w), None)
+    assert lib_.aq_status_string(st) == b"AQ_ERR_OVERLAP"
+    E, T = 2, 6
+    xs = torch.zeros(T, K, dtype=torch.bfloat16)
+    wqb, scb, bib = _weights(N, K, B, G, batch=(E,))
+    ys = torch.zeros(1, N, dtype=torch.bfloat16).expand(T, N)
+    st = lib_.aq_qmm_t_grouped(aq.view(xs), 8, E, aq.view(wqb), aq.view(scb), aq.view(bib), G, B, aq.view(ys),
+                               None)
+    assert lib_.aq_status_string(st) == b"AQ_ERR_OVERLAP"
+    # a y whose zero stride sits on a dimension of extent 1 is fine
+    y1 = torch.empty(1, N, dtype=torch.bfloat16).as_strided((1, N), (0, 1))
+    assert aq.aq_plan_linear(torch.zeros(1, K, dtype=torch.bfloat16), wq, sc, bi, G, B, y1)["total_rows"] == 1

@@ -147,6 +147,56 @@ def test_grouped_moe_bank_shape():
             assert np.all(row_errors(y[r:r + 1], ref) <= 4e-3), (e, r)
 
 
+def test_grouped_moe_bank_config_size():
+    """The full expert bank of the benchmark: 128 experts of [2816 out, 1408 in], 8-bit, G = 32
+    ("Metal Kernel Bits=8 Final Report" shapes), 256 tokens routed to 8 distinct experts each
+    (2048 rows), one launch; every row against every column of the fp64 oracle."""
+    E, N, K, group, bits = inputs.MOE_EXPERTS, inputs.MOE_N, inputs.MOE_K, inputs.MOE_GROUP, inputs.MOE_BITS
+    tok, offsets = inputs.moe_sort(inputs.moe_routing())
+    T = tok.numel()
+    x_tok = inputs.normal((inputs.MOE_TOKENS, K), 1.0, torch.bfloat16, seed=9)
+    x_sorted = x_tok[tok].contiguous()
+    xb = x_sorted.view(torch.int16).numpy().view(np.uint16)
+    wq = torch.empty(E, N, K * bits // 32, dtype=torch.int32, device=DEV)
+    sc = torch.empty(E, N, K // group, dtype=torch.bfloat16, device=DEV)
+    bi = torch.empty_like(sc)
+    ref = np.empty((T, N), np.float64)
+    for e in range(E):
+        Q = oracle.quantize(inputs.normal((N, K), inputs.W_STD, seed=100 + e).numpy(), group, bits, "bf16")
+        qd = to_device_quant(Q, DEV, torch.bfloat16)
+        wq[e].copy_(qd[0]); sc[e].copy_(qd[1]); bi[e].copy_(qd[2])
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi > lo:
+            ref[lo:hi] = oracle.linear_contig(xb[lo:hi], "bf16", Q.dequant())
+    y = aq.aq_qmm_t_grouped(x_sorted.to(DEV), offsets.to(DEV), wq, sc, bi, group, bits)
+    err = row_errors(y, ref)
+    assert err.size == T == 2048 and np.all(err <= 4e-3), (err.max(), int(err.argmax()))
+
+
+def test_grouped_offsets_clamped_on_device():
+    """Offsets the host cannot check (they live on the device) that start below 0 and end past T:
+    the kernel clamps each expert's rows into [0, T), writes nothing outside y_sorted (canary rows
+    and columns around it keep their value) and the rows it owns match the oracle."""
+    E, N, K, group, bits = 4, 200, 256, 32, 8
+    T = 40
+    bad = np.array([-7, 10, 25, 25, 60], np.int64)
+    clamped = np.array([0, 10, 25, 25, 40], np.int64)
+    w = inputs.normal((E, N, K), 0.02, seed=71)
+    Q = oracle.quantize(w.numpy(), group, bits, "bf16")
+    wq, sc, bi = to_device_quant(Q, DEV, torch.bfloat16)
+    x = inputs.normal((T, K), 1.0, torch.bfloat16, seed=72)
+    buf = torch.full((T + 4, N + 8), 3072.0, dtype=torch.bfloat16, device=DEV)
+    y = buf[2:T + 2, 4:4 + N]
+    aq.aq_qmm_t_grouped(x.to(DEV), torch.from_numpy(bad).to(DEV), wq, sc, bi, group, bits, out=y)
+    aq.aq_device_error()
+    b = buf.float().cpu()
+    assert torch.all(b[:2] == 3072.0) and torch.all(b[T + 2:] == 3072.0)
+    assert torch.all(b[:, :4] == 3072.0) and torch.all(b[:, 4 + N:] == 3072.0)
+    xb = x.contiguous().view(torch.int16).numpy().view(np.uint16)
+    ref = oracle.linear_grouped(xb, "bf16", clamped, Q.dequant())
+    assert np.all(row_errors(y, ref) <= 4e-3)
+
+
 def test_odd_group_count_takes_gemv():
     """K/group odd (K=192, G=64) is served by the GEMV kernel, still to the same bar."""
     w = inputs.normal((100, 192), 0.02, seed=41)

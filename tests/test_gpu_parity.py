@@ -49,6 +49,24 @@ def test_quantize_bit_exact(bits, group, sdtype):
     assert np.array_equal(bi.float().cpu().numpy(), oracle.half_to_double(Q.bias_bits, sdtype).astype(np.float32))
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("group", [32, 64, 128])
+def test_quantize_ties_bit_exact(bits, group):
+    """Values exactly halfway between two codes (scale a power of two, (w - bias)/scale = k + 1/2
+    with no rounding) take the oracle's codes, which a CPU pin fixes to the even neighbour."""
+    maxq = (1 << bits) - 1
+    rows = []
+    for r, (s, b) in enumerate([(1.0, 0.0), (0.5, -3.0), (2.0, 5.25), (0.125, -0.5)]):
+        ks = [(r * 7 + j) % maxq for j in range(group - 2)]
+        g = [b, b + s * maxq] + [b + s * (k + 0.5) for k in ks]
+        rows.append(g * 4)
+    w = torch.tensor(rows, dtype=torch.float32)
+    Q = oracle.quantize(w.numpy(), group, bits, "bf16")
+    wq, sc, bi = aq.aq_quantize(w.to(DEV), group, bits, scale_dtype=torch.bfloat16)
+    assert np.array_equal(wq.cpu().numpy().view(np.uint32), Q.packed)
+    assert np.array_equal(sc.float().cpu().numpy(), oracle.half_to_double(Q.scale_bits, "bf16").astype(np.float32))
+
+
 @pytest.mark.parametrize("wdtype", [torch.bfloat16, torch.float16])
 def test_quantize_half_input(wdtype):
     w = inputs.normal((40, 256), 0.02, dtype=wdtype, seed=9)
@@ -132,6 +150,41 @@ def test_running_sum_stress_exact(xdtype, bits, group, rows):
         assert np.all(np.abs(got - exact) <= 1e-6 * exact), (N, got.ravel()[:4], exact)
 
 
+# The same exact-sum case through every kernel of aq_qmm_t, with the kernel asserted: the
+# warp-level kernel (8 and 32 rows), the tcgen05 small-M kernel (40 rows) and the tcgen05 prefill
+# kernel (128 rows).  Each forms sum(x) per group with its own code; each must give the exact
+# bias * sum(x) ("mlx PR #4516": exact result for inputs whose running sum is not representable in
+# half types).  Every bits x group the kernel takes; N over the ragged set.
+_WARP_BG = [(2, 64), (2, 128), (4, 32), (4, 64), (4, 128), (8, 32), (8, 64), (8, 128)]
+_STRESS_KERNELS = {
+    "warp_m8": (8, 4096, "warp_mma", _WARP_BG, (1, 4, 7, 1001, 4099)),
+    "warp_m32": (32, 1024, "warp_mma", _WARP_BG, (1, 4, 7, 1001, 1024)),
+    "tc_small_m": (40, 4096, "tc_small_m", [(b, g) for b in (2, 4, 6, 8) for g in (32, 64, 128)],
+                   (1, 7, 1001, 4099)),
+    "tc_prefill": (128, 4096, "tc_prefill", [(b, g) for b in (2, 4, 6, 8) for g in (64, 128)],
+                   (1, 7, 1001, 4099)),
+}
+
+
+@pytest.mark.parametrize("xdtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("case", list(_STRESS_KERNELS))
+def test_running_sum_stress_every_kernel(xdtype, case):
+    rows, K, kernel, bgs, Ns = _STRESS_KERNELS[case]
+    sd = dtype_name(torch.empty(0, dtype=xdtype))
+    small = 2.0 ** -9 if xdtype == torch.bfloat16 else 2.0 ** -12
+    exact = (K // 2) * (1.0 + small)
+    x = inputs.stress_x(K, rows, xdtype).to(DEV).view(rows, 1, K)
+    for bits, group in bgs:
+        for N in Ns:
+            Q, (wq, sc, bi) = _q(inputs.stress_w(N, K), group, bits, sd)
+            assert np.all(Q.codes == 0)
+            y = torch.empty(rows, 1, N, dtype=torch.float32, device=DEV)
+            assert aq.aq_plan_linear(x, wq, sc, bi, group, bits, y)["kernel"] == kernel, (bits, group, N)
+            aq.aq_qmm_t(x, wq, sc, bi, group, bits, out=y)
+            got = y.double().cpu().numpy()
+            assert np.all(np.abs(got - exact) <= 1e-6 * exact), (bits, group, N, got.ravel()[:4], exact)
+
+
 # ---------------------------------------------------------------------------
 # strided batched views (candle pitfall page)
 # ---------------------------------------------------------------------------
@@ -205,15 +258,39 @@ def test_output_canaries_untouched(bits):
     assert np.all(row_errors(y, ref) <= 4e-3)
 
 
-def test_minimal_k_and_single_row():
-    w = inputs.normal((1, 32), 1.0, seed=77)
-    Q, (wq, sc, bi) = _q(w, 32, 4)
-    x = inputs.normal((1, 32), 1.0, torch.bfloat16, seed=78)
-    y = aq.aq_qmm_t(x.to(DEV), wq, sc, bi, 32, 4, out_dtype=torch.float32)
+def _gemv_fp32_bound(Q, x: torch.Tensor, bits: int) -> np.ndarray:
+    """Worst-case fp32 error of the GEMV's fp32 output, per element (forward error analysis).
+
+    Per 32-code chunk the GEMV adds 32 exact products (BASE + q) * x (BASE = 128, or 256 for
+    8-bit codes) and the 32 widened x values, then folds s * P + (b - BASE*s) * X into the row
+    sum; the chunk sums of all lanes meet in a 5-level shuffle tree.  With u = 2^-24 every
+    rounded sum of n terms is off by at most n*u times the sum of their magnitudes, so
+        |y - ref| <= (32 + C + 8) * u * sum_k (|s_k| (BASE + q_k) + |b_k| + BASE |s_k|) |x_k|
+    with C the number of chunks.  This is an absolute bound: the offset BASE makes it scale with
+    BASE * |s| * sum|x|, not with |y|.
+    """
+    base = 256.0 if bits == 8 else 128.0
+    G = Q.group
+    s = np.repeat(oracle.half_to_double(Q.scale_bits, "bf16"), G, axis=-1)
+    b = np.repeat(oracle.half_to_double(Q.bias_bits, "bf16"), G, axis=-1)
+    mag = np.abs(s) * (base + Q.codes) + np.abs(b) + base * np.abs(s)          # [N, K]
+    xa = np.abs(x.float().double().numpy().reshape(-1, x.shape[-1]))          # [M, K]
+    C = x.shape[-1] // 32
+    return (32 + C + 8) * 2.0 ** -24 * (xa @ mag.T)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("K", [32, 4096])
+def test_gemv_fp32_output_bound(bits, K):
+    """fp32 outputs of the GEMV stay inside their derived rounding bound (single row, K from one
+    chunk to 128 chunks)."""
+    w = inputs.normal((3, K), 1.0, seed=77 + K)
+    Q, (wq, sc, bi) = _q(w, 32, bits)
+    x = inputs.normal((1, K), 1.0, torch.bfloat16, seed=78 + K)
+    y = aq.aq_qmv(x.to(DEV), wq, sc, bi, 32, bits, out_dtype=torch.float32)
     ref = oracle_linear_view(x, Q.dequant())
-    # fp32 output: the GEMV forms (128 + q) * x products exactly and removes the offset once per
-    # 32-code chunk, which leaves a few fp32 ulps of 128 * sum(x) in the result
-    assert abs(float(y.item()) - ref.item()) <= 1e-4 * max(1.0, abs(ref.item()))
+    bound = _gemv_fp32_bound(Q, x, bits)
+    assert np.all(np.abs(y.double().cpu().numpy() - ref) <= bound), (y, ref, bound)
 
 
 def test_f16_activations():

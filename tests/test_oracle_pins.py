@@ -157,6 +157,46 @@ def test_quantize_exact_grid(orc, bits, group, sdtype):
 
 
 @pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("group", [32, 64, 128])
+def test_quantize_ties_round_to_even(orc, bits, group):
+    """(w - bias) / scale exactly halfway between two codes goes to the even code.
+
+    Each group holds its minimum b and maximum b + s*(2^bits - 1) (so the quantizer's scale is s
+    exactly, s a power of two) and values b + s*(k + 1/2): the quotient is k + 1/2 with no
+    rounding anywhere, and the expected code is whichever of k, k + 1 is even.  Rounding half away
+    from zero (roundf), half up (floor(v + 1/2)) or half down would each miss every odd or every
+    even k.
+    """
+    maxq = (1 << bits) - 1
+    rows = []
+    expect = []
+    for r, (s, b) in enumerate([(1.0, 0.0), (0.5, -3.0), (2.0, 5.25), (0.125, -0.5)]):
+        ks = [(r * 7 + j) % maxq for j in range(group - 2)] if maxq > 1 else [0] * (group - 2)
+        row_w = [b, b + s * maxq] + [b + s * (k + 0.5) for k in ks]
+        row_q = [0, maxq] + [k if k % 2 == 0 else k + 1 for k in ks]
+        # four groups per row: the same values in rotated positions
+        w_row, q_row = [], []
+        for g in range(4):
+            rot = (5 * g) % group
+            w_row += row_w[rot:] + row_w[:rot]
+            q_row += row_q[rot:] + row_q[:rot]
+        rows.append(w_row)
+        expect.append(q_row)
+    w = np.array(rows, np.float32)
+    # every value is exact in fp32 and every quotient is an exact half-integer
+    assert np.array_equal(w.astype(np.float64), np.array(rows, np.float64))
+    Q = orc.quantize(w, group, bits, "bf16")
+    assert np.array_equal(Q.scale32, np.repeat(np.array([[1.0], [0.5], [2.0], [0.125]], np.float32), 4, axis=1))
+    assert np.array_equal(Q.codes, np.array(expect, np.uint8))
+    # and the packed words decode (bit by bit, Python integers) to the same codes
+    packed = Q.packed.astype(np.uint64)
+    for r in range(len(rows)):
+        stream = sum(int(v) << (32 * i) for i, v in enumerate(packed[r]))
+        got = [(stream >> (i * bits)) & maxq for i in range(w.shape[1])]
+        assert got == expect[r]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
 @pytest.mark.parametrize("group", [32, 128])
 def test_quantize_error_bound(orc, bits, group):
     """|w - w'| <= scale/2 + q*|scale - s_stored| + |bias - b_stored| (+ fp32 slack)."""
