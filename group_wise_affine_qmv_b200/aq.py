@@ -50,8 +50,9 @@ class AqPlan(ctypes.Structure):
                 ("y_row_stride", ctypes.c_int64), ("total_rows", ctypes.c_int64)]
 
 
-EXPORTED = ("aq_quantize", "aq_dequantize", "aq_qmv", "aq_qmm_t", "aq_qmm_t_grouped", "aq_plan_linear",
-            "aq_status_string", "aq_last_error_message", "aq_device_error", "aq_version")
+EXPORTED = ("aq_quantize", "aq_dequantize", "aq_qmv", "aq_qmm_t", "aq_qmm_t_grouped", "aq_qmm_t_multi",
+            "aq_qmm_t_swiglu", "aq_qmm_t_residual", "aq_plan_linear", "aq_status_string", "aq_last_error_message",
+            "aq_device_error", "aq_version")
 
 _lib = None
 _lock = threading.Lock()
@@ -78,6 +79,13 @@ def load_library(path: str = LIB_PATH):
         lib.aq_dequantize.restype = ci
         lib.aq_qmm_t_grouped.argtypes = [V, vp, ci, V, V, V, ci, ci, V, vp]
         lib.aq_qmm_t_grouped.restype = ci
+        VA = ctypes.POINTER(V)
+        lib.aq_qmm_t_multi.argtypes = [V, ci, VA, VA, VA, ci, ci, VA, vp]
+        lib.aq_qmm_t_multi.restype = ci
+        lib.aq_qmm_t_swiglu.argtypes = [V, V, V, V, V, V, V, ci, ci, V, vp]
+        lib.aq_qmm_t_swiglu.restype = ci
+        lib.aq_qmm_t_residual.argtypes = [V, V, V, V, ci, ci, V, V, vp]
+        lib.aq_qmm_t_residual.restype = ci
         lib.aq_plan_linear.argtypes = [V, V, V, V, ci, ci, V, ci, ctypes.POINTER(AqPlan)]
         lib.aq_plan_linear.restype = ci
         lib.aq_status_string.argtypes = [ci]
@@ -184,6 +192,44 @@ def aq_qmm_t_grouped(x_sorted, offsets, wq_bank, s_bank, b_bank, group: int, bit
         _check(lib, lib.aq_qmm_t_grouped(view(x_sorted), ctypes.c_void_p(offsets.data_ptr()), wq_bank.shape[0],
                                          view(wq_bank), view(s_bank), view(b_bank), group, bits, view(out),
                                          _stream(x_sorted)))
+    return out
+
+
+def aq_qmm_t_multi(x, weights, group: int, bits: int, outs=None, out_dtype=None):
+    """y[j] = x . dequant(W_j)^T for up to three (wq, scales, biases) sharing x, in one launch
+    where the warp-level kernel takes them.  Returns the list of outputs."""
+    lib = load_library()
+    n = len(weights)
+    if outs is None:
+        outs = [torch.empty(tuple(x.shape[:-1]) + (w[0].shape[-2],), dtype=out_dtype or x.dtype, device=x.device)
+                for w in weights]
+    V = ctypes.POINTER(AqView)
+    keep = [[view(w[i]) for w in weights] for i in range(3)] + [[view(o) for o in outs]]
+    arrs = [(V * n)(*[ctypes.pointer(v) for v in vs]) for vs in keep]
+    with torch.cuda.device(x.device):
+        _check(lib, lib.aq_qmm_t_multi(view(x), n, arrs[0], arrs[1], arrs[2], group, bits, arrs[3], _stream(x)))
+    return outs
+
+
+def aq_qmm_t_swiglu(x, gate, up, group: int, bits: int, out=None, out_dtype=None):
+    """y = silu(x . dequant(W_gate)^T) * (x . dequant(W_up)^T); gate, up = (wq, scales, biases)."""
+    lib = load_library()
+    if out is None:
+        out = torch.empty(tuple(x.shape[:-1]) + (gate[0].shape[-2],), dtype=out_dtype or x.dtype, device=x.device)
+    with torch.cuda.device(x.device):
+        _check(lib, lib.aq_qmm_t_swiglu(view(x), view(gate[0]), view(gate[1]), view(gate[2]), view(up[0]),
+                                        view(up[1]), view(up[2]), group, bits, view(out), _stream(x)))
+    return out
+
+
+def aq_qmm_t_residual(x, wq, scales, biases, group: int, bits: int, r, out=None):
+    """y = r + x . dequant(W)^T (out may be r itself: an in-place residual update)."""
+    lib = load_library()
+    if out is None:
+        out = torch.empty_like(r)
+    with torch.cuda.device(x.device):
+        _check(lib, lib.aq_qmm_t_residual(view(x), view(wq), view(scales), view(biases), group, bits, view(r),
+                                          view(out), _stream(x)))
     return out
 
 

@@ -158,6 +158,9 @@ struct Resolved {
     aq::MmaProblem mp;
 };
 
+void fill_mma_problem(const aq_view* x, const aq_view* wq, const aq_view* sc, const aq_view* bi, int group,
+                      int bits, const aq_view* y, Resolved* R);
+
 aq_status resolve_linear(const aq_view* x, const aq_view* wq, const aq_view* sc, const aq_view* bi,
                          int group, int bits, const aq_view* y, int force_qmv, Resolved* R) {
     aq_status st;
@@ -302,27 +305,8 @@ aq_status resolve_linear(const aq_view* x, const aq_view* wq, const aq_view* sc,
         else if (M <= 4) R->mma_why = "few rows per launch: GEMV";
         else if (K == 0 || N == 0) R->mma_why = "empty contraction";
         else {
+            fill_mma_problem(x, wq, sc, bi, group, bits, y, R);
             aq::MmaProblem& mp = R->mp;
-            memset(&mp, 0, sizeof mp);
-            mp.x = x->data;
-            mp.y = y->data;
-            mp.wq = (const uint32_t*)wq->data;
-            mp.scales = sc->data;
-            mp.biases = bi->data;
-            mp.M = M;
-            mp.N = N;
-            mp.K = K;
-            mp.x_row = xrow;
-            mp.y_row = yrow;
-            mp.nb[0] = P.batch_shape[0];
-            mp.nb[1] = P.batch_shape[1];
-            for (int s = 0; s < 2; ++s) { mp.xb[s] = P.x_batch_stride[s]; mp.yb[s] = P.y_batch_stride[s]; }
-            mp.w_row = R->w_row;
-            mp.group = group;
-            mp.bits = bits;
-            mp.xdt = (aq::DT)x->dtype;
-            mp.ydt = (aq::DT)y->dtype;
-            mp.offsets = nullptr;
             // scales/biases rows must be contiguous for the tile loads
             if (R->s_row != K / group || R->b_row != K / group) R->mma_why = "scales/biases rows not contiguous";
             else R->mma_ok = aq::mma_supported(mp, &R->mma_why);
@@ -331,6 +315,33 @@ aq_status resolve_linear(const aq_view* x, const aq_view* wq, const aq_view* sc,
     P.regime = R->mma_ok ? AQ_REGIME_MMA : AQ_REGIME_QMV;
     P.kernel = R->mma_ok ? (int32_t)aq::mma_kernel_for(R->mp) : AQ_KERNEL_GEMV;
     return AQ_OK;
+}
+
+// The tensor-core problem of a resolved call (its plan already filled in).
+void fill_mma_problem(const aq_view* x, const aq_view* wq, const aq_view* sc, const aq_view* bi, int group,
+                      int bits, const aq_view* y, Resolved* R) {
+    const aq_plan& P = R->plan;
+    aq::MmaProblem& mp = R->mp;
+    memset(&mp, 0, sizeof mp);
+    mp.x = x->data;
+    mp.y = y->data;
+    mp.wq = (const uint32_t*)wq->data;
+    mp.scales = sc->data;
+    mp.biases = bi->data;
+    mp.M = P.M;
+    mp.N = P.N;
+    mp.K = P.K;
+    mp.x_row = P.x_row_stride;
+    mp.y_row = P.y_row_stride;
+    mp.nb[0] = P.batch_shape[0];
+    mp.nb[1] = P.batch_shape[1];
+    for (int s = 0; s < 2; ++s) { mp.xb[s] = P.x_batch_stride[s]; mp.yb[s] = P.y_batch_stride[s]; }
+    mp.w_row = R->w_row;
+    mp.group = group;
+    mp.bits = bits;
+    mp.xdt = (aq::DT)x->dtype;
+    mp.ydt = (aq::DT)y->dtype;
+    mp.offsets = nullptr;
 }
 
 aq_status run_linear(const aq_view* x, const aq_view* wq, const aq_view* sc, const aq_view* bi, int group,
@@ -377,6 +388,33 @@ aq_status run_linear(const aq_view* x, const aq_view* wq, const aq_view* sc, con
     if (nbatch > 65535) return fail(AQ_ERR_UNSUPPORTED, "more than 65535 launch batches");
     e = aq::launch_qmv(a, bits, (aq::DT)x->dtype, (aq::DT)y->dtype, nbatch, s);
     if (e != cudaSuccess) return cuda_fail(e, "GEMV kernel launch");
+    return AQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// fused calls on the warp-level kernel: several W sharing x, gate/up with silu, a residual
+// ---------------------------------------------------------------------------
+
+// Resolves matrix j of a fused call as a plain call and checks that it folds to one 2D problem
+// (no launch batch dims, unbatched W) the warp-level kernel can take.
+aq_status resolve_fused_part(const aq_view* x, const aq_view* wq, const aq_view* sc, const aq_view* bi, int group,
+                             int bits, const aq_view* y, const char* what, Resolved* R, bool* warp_ok) {
+    aq_status st = resolve_linear(x, wq, sc, bi, group, bits, y, 0, R);
+    if (st != AQ_OK) return st;
+    if (R->plan.nbatch_dims != 0 || R->plan.w_batched)
+        return fail(AQ_ERR_UNSUPPORTED, "%s: x and y must fold into one 2D problem, with an unbatched W", what);
+    fill_mma_problem(x, wq, sc, bi, group, bits, y, R);
+    const char* why = nullptr;
+    *warp_ok = R->plan.total_rows > 0 && R->plan.N > 0 && R->s_row == R->plan.K / group &&
+               R->b_row == R->plan.K / group && aq::mma_supported(R->mp, &why) && aq::warp_mma_supported(R->mp);
+    return AQ_OK;
+}
+
+aq_status launch_fused(aq::MmaProblem& mp, void* stream) {
+    aq_status st = check_device();
+    if (st != AQ_OK) return st;
+    cudaError_t e = aq::launch_warp_mma(mp, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "fused warp-level kernel launch");
     return AQ_OK;
 }
 
@@ -597,4 +635,121 @@ AQ_API aq_status aq_device_error(void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
     if (v != 0) return fail(AQ_ERR_TIMEOUT, "a kernel's bounded wait expired (code %d)", v);
     return AQ_OK;
+}
+
+AQ_API aq_status aq_qmm_t_multi(const aq_view* x, int n, const aq_view* const* wq, const aq_view* const* scales,
+                                const aq_view* const* biases, int group, int bits, const aq_view* const* y,
+                                void* stream) {
+    g_msg[0] = 0;
+    if (n < 1 || n > 3) return fail(AQ_ERR_UNSUPPORTED, "n=%d matrices (1..3 supported)", n);
+    if (!wq || !scales || !biases || !y) return fail(AQ_ERR_NULL, "NULL array of views");
+    Resolved R[3];
+    bool all_warp = true;
+    for (int j = 0; j < n; ++j) {
+        aq_status st = resolve_linear(x, wq[j], scales[j], biases[j], group, bits, y[j], 0, &R[j]);
+        if (st != AQ_OK) return st;
+    }
+    // no output may overlap another output or another matrix's inputs
+    for (int j = 0; j < n; ++j)
+        for (int k = 0; k < n; ++k) {
+            if (j == k) continue;
+            if (overlaps(y[j], y[k]) || overlaps(y[j], wq[k]) || overlaps(y[j], scales[k]) || overlaps(y[j], biases[k]))
+                return fail(AQ_ERR_OVERLAP, "y[%d] overlaps an input or output of matrix %d", j, k);
+        }
+    if (R[0].plan.total_rows == 0) return AQ_OK;
+    for (int j = 0; j < n && all_warp; ++j) {
+        bool ok = false;
+        aq_status st = resolve_fused_part(x, wq[j], scales[j], biases[j], group, bits, y[j], "aq_qmm_t_multi", &R[j],
+                                          &ok);
+        if (st != AQ_OK) ok = false;
+        all_warp = ok && R[j].plan.M == R[0].plan.M && R[j].plan.x_row_stride == R[0].plan.x_row_stride;
+    }
+    if (!all_warp || n == 1) {
+        // one plain call per matrix, in order, on the same stream
+        for (int j = 0; j < n; ++j) {
+            aq_status st = run_linear(x, wq[j], scales[j], biases[j], group, bits, y[j], stream, 0);
+            if (st != AQ_OK) return st;
+        }
+        return AQ_OK;
+    }
+    aq::MmaProblem mp = R[0].mp;
+    mp.nseg = n;
+    for (int j = 0; j < n; ++j) {
+        mp.seg_wq[j] = R[j].mp.wq;
+        mp.seg_scales[j] = R[j].mp.scales;
+        mp.seg_biases[j] = R[j].mp.biases;
+        mp.seg_y[j] = R[j].mp.y;
+        mp.seg_N[j] = R[j].mp.N;
+        mp.seg_w_row[j] = R[j].mp.w_row;
+        mp.seg_y_row[j] = R[j].mp.y_row;
+    }
+    if (!aq::warp_mma_supported(mp)) return fail(AQ_ERR_UNSUPPORTED, "fused projections: too many row blocks");
+    return launch_fused(mp, stream);
+}
+
+AQ_API aq_status aq_qmm_t_swiglu(const aq_view* x, const aq_view* wq_gate, const aq_view* s_gate,
+                                 const aq_view* b_gate, const aq_view* wq_up, const aq_view* s_up,
+                                 const aq_view* b_up, int group, int bits, const aq_view* y, void* stream) {
+    g_msg[0] = 0;
+    Resolved Rg, Ru;
+    bool okg = false, oku = false;
+    aq_status st = resolve_fused_part(x, wq_gate, s_gate, b_gate, group, bits, y, "aq_qmm_t_swiglu", &Rg, &okg);
+    if (st != AQ_OK) return st;
+    st = resolve_fused_part(x, wq_up, s_up, b_up, group, bits, y, "aq_qmm_t_swiglu", &Ru, &oku);
+    if (st != AQ_OK) return st;
+    if (Ru.plan.N != Rg.plan.N) return fail(AQ_ERR_SHAPE, "gate and up matrices must have the same N");
+    if (Rg.plan.total_rows == 0 || Rg.plan.N == 0) return AQ_OK;
+    if (!okg || !oku)
+        return fail(AQ_ERR_UNSUPPORTED,
+                    "aq_qmm_t_swiglu runs on the warp-level kernel only (up to 32 rows, 2/4/8-bit codes, "
+                    "16-byte aligned rows)");
+    aq::MmaProblem mp = Rg.mp;
+    mp.nseg = 2;
+    mp.glu = 1;
+    const Resolved* parts[2] = {&Rg, &Ru};
+    for (int j = 0; j < 2; ++j) {
+        mp.seg_wq[j] = parts[j]->mp.wq;
+        mp.seg_scales[j] = parts[j]->mp.scales;
+        mp.seg_biases[j] = parts[j]->mp.biases;
+        mp.seg_y[j] = Rg.mp.y;
+        mp.seg_N[j] = parts[j]->mp.N;
+        mp.seg_w_row[j] = parts[j]->mp.w_row;
+        mp.seg_y_row[j] = Rg.mp.y_row;
+    }
+    if (!aq::warp_mma_supported(mp)) return fail(AQ_ERR_UNSUPPORTED, "gate/up: too many row blocks");
+    return launch_fused(mp, stream);
+}
+
+AQ_API aq_status aq_qmm_t_residual(const aq_view* x, const aq_view* wq, const aq_view* scales,
+                                   const aq_view* biases, int group, int bits, const aq_view* r, const aq_view* y,
+                                   void* stream) {
+    g_msg[0] = 0;
+    Resolved R, Rr;
+    bool ok = false, okr = false;
+    aq_status st = resolve_fused_part(x, wq, scales, biases, group, bits, y, "aq_qmm_t_residual", &R, &ok);
+    if (st != AQ_OK) return st;
+    if ((st = check_view(r, "r", 1, 4)) != AQ_OK) return st;
+    if (r->dtype != y->dtype) return fail(AQ_ERR_DTYPE, "r must have y's dtype");
+    // r has y's shape and folds the same way; it is read as an input, so it may be y itself
+    // (the same view: each element is read and then written by the same thread) but must not
+    // overlap y otherwise, nor the other inputs
+    const bool same = r->data == y->data && r->rank == y->rank &&
+                      memcmp(r->shape, y->shape, sizeof(int64_t) * y->rank) == 0 &&
+                      memcmp(r->stride, y->stride, sizeof(int64_t) * y->rank) == 0;
+    if (!same) {
+        st = resolve_fused_part(x, wq, scales, biases, group, bits, r, "aq_qmm_t_residual (r)", &Rr, &okr);
+        if (st != AQ_OK) return st;
+        if (overlaps(r, y)) return fail(AQ_ERR_OVERLAP, "r overlaps y (other than being the same view)");
+    } else {
+        Rr = R;
+    }
+    if (R.plan.total_rows == 0 || R.plan.N == 0) return AQ_OK;
+    if (!ok)
+        return fail(AQ_ERR_UNSUPPORTED,
+                    "aq_qmm_t_residual runs on the warp-level kernel only (up to 32 rows, 2/4/8-bit codes, "
+                    "16-byte aligned rows)");
+    aq::MmaProblem mp = R.mp;
+    mp.r = r->data;
+    mp.r_row = Rr.plan.y_row_stride;
+    return launch_fused(mp, stream);
 }

@@ -69,6 +69,19 @@ struct MmaProblem {
     const int64_t* offsets;     // device, n_experts + 1
     int n_experts;
     int64_t w_expert, s_expert, b_expert;  // per-expert strides (words / elements)
+    // fused calls (warp-level kernel only): nseg > 1 W matrices share x in one launch; entry 0
+    // repeats wq/scales/biases/y/N/w_row/y_row above.  glu: two segments (gate, up) whose
+    // output is silu(gate) * up, written to seg_y[0].
+    int nseg;
+    int glu;
+    const uint32_t* seg_wq[3];
+    const void* seg_scales[3];
+    const void* seg_biases[3];
+    void* seg_y[3];
+    int64_t seg_N[3], seg_w_row[3], seg_y_row[3];
+    // optional residual of the plain call (warp-level kernel only): y = r + x . W^T
+    const void* r;
+    int64_t r_row;
 };
 
 // Whether the tensor-core kernel can run this problem (alignment, bits, K), and why not.

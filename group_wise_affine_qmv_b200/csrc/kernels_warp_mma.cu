@@ -39,12 +39,22 @@ struct Shape {
 // of K.  The split of K depends on N, K and the total rows only (not on how the rows are
 // grouped into launch batches), so a strided view and its contiguous copy sum in the same
 // order and give the same bits.
+// Row blocks (of wm::ROWS W rows, one per warp) of a launch: the plain W; the fused matrices one
+// after another; or, for gate/up, 16 rows of each matrix per block.
+int64_t row_blocks(const MmaProblem& p) {
+    if (p.nseg <= 1) return (p.N + wm::ROWS - 1) / wm::ROWS;
+    if (p.glu) return (p.seg_N[0] + wm::ROWS / 2 - 1) / (wm::ROWS / 2);
+    int64_t n = 0;
+    for (int s = 0; s < p.nseg; ++s) n += (p.seg_N[s] + wm::ROWS - 1) / wm::ROWS;
+    return n;
+}
+
 Shape shape_for(const MmaProblem& p, int sms) {
     Shape s;
     const int nt = tokens_per_tile(p.M);
     s.ntl = nt / 8;
     const int64_t kg = p.K / p.group;
-    const int64_t nrt = (p.N + wm::ROWS - 1) / wm::ROWS;
+    const int64_t nrt = row_blocks(p);
     const int64_t rows_all = p.M * p.nb[0] * p.nb[1];
     const int64_t units = (rows_all + wm::MAX_TOKENS - 1) / wm::MAX_TOKENS;
     int wr = 1;
@@ -90,7 +100,7 @@ bool warp_mma_supported(const MmaProblem& p) {
     const int64_t kg = p.K / p.group;
     if ((size_t)kg * wm::MAX_TOKENS * sizeof(float) > (size_t)wm::MAX_XTAB_BYTES) return false;
     if ((int64_t)wm::ROWS * kg * 4 > SB_MAX_BYTES) return false;
-    if (p.nb[0] * p.nb[1] > 65535 || (p.N + wm::ROWS - 1) / wm::ROWS > 0x7fffffff) return false;
+    if (p.nb[0] * p.nb[1] > 65535 || row_blocks(p) > 0x7fffffff) return false;
     // 16-byte rows of x and W, as the tensor-core kernels require (checked by mma_supported)
     return true;
 }
@@ -116,21 +126,33 @@ cudaError_t launch_warp_mma(const MmaProblem& pb, cudaStream_t stream) {
     wm::WParams p;
     memset(&p, 0, sizeof p);
     p.x = static_cast<const uint16_t*>(pb.x);
-    p.y = pb.y;
-    p.wq = pb.wq;
-    p.scales = static_cast<const uint16_t*>(pb.scales);
-    p.biases = static_cast<const uint16_t*>(pb.biases);
+    const bool fused = pb.nseg > 1;
+    p.nseg = fused ? pb.nseg : 1;
+    p.glu = fused && pb.glu ? 1 : 0;
+    int64_t rb = 0;
+    for (int i = 0; i < p.nseg; ++i) {
+        wm::WSeg& g = p.seg[i];
+        g.wq = fused ? pb.seg_wq[i] : pb.wq;
+        g.scales = static_cast<const uint16_t*>(fused ? pb.seg_scales[i] : pb.scales);
+        g.biases = static_cast<const uint16_t*>(fused ? pb.seg_biases[i] : pb.biases);
+        g.y = fused ? pb.seg_y[i] : pb.y;
+        g.N = fused ? pb.seg_N[i] : pb.N;
+        g.w_row = fused ? pb.seg_w_row[i] : pb.w_row;
+        g.y_row = fused ? pb.seg_y_row[i] : pb.y_row;
+        g.rb0 = p.glu ? 0 : rb;
+        g.r = fused ? nullptr : pb.r;
+        g.r_row = pb.r_row;
+        rb += (g.N + wm::ROWS - 1) / wm::ROWS;
+    }
+    p.nrb = row_blocks(pb);
     p.M = pb.M;
-    p.N = pb.N;
     p.K = pb.K;
     p.x_row = pb.x_row;
-    p.y_row = pb.y_row;
     for (int i = 0; i < 2; ++i) {
         p.xb[i] = pb.nb[i] > 1 ? pb.xb[i] : 0;
         p.yb[i] = pb.nb[i] > 1 ? pb.yb[i] : 0;
     }
     p.nb1 = pb.nb[1] > 0 ? pb.nb[1] : 1;
-    p.w_row = pb.w_row;
     p.kg = (int)(pb.K / pb.group);
     p.cs = s.cs;
     p.kgc = s.kgc;
@@ -139,13 +161,17 @@ cudaError_t launch_warp_mma(const MmaProblem& pb, cudaStream_t stream) {
     p.wk = s.wk;
     p.ydt = (int)pb.ydt;
     const size_t ysz = pb.ydt == DT::F32 ? 4 : 2;
-    bool yvec = ((uintptr_t)pb.y % (2 * ysz)) == 0 && (pb.M <= 1 || pb.y_row % 2 == 0);
+    bool yvec = true, sb16 = p.kg % 8 == 0;
+    for (int i = 0; i < p.nseg; ++i) {
+        if (((uintptr_t)p.seg[i].y % (2 * ysz)) != 0 || (pb.M > 1 && p.seg[i].y_row % 2 != 0)) yvec = false;
+        if (((uintptr_t)p.seg[i].scales & 15) || ((uintptr_t)p.seg[i].biases & 15)) sb16 = false;
+    }
     for (int i = 0; i < 2; ++i)
         if (pb.nb[i] > 1 && pb.yb[i] % 2 != 0) yvec = false;
     p.yvec = yvec ? 1 : 0;
     p.xsm = s.xsm ? 1 : 0;
     p.x_pitch = s.x_pitch;
-    p.sb16 = (p.kg % 8 == 0 && ((uintptr_t)pb.scales & 15) == 0 && ((uintptr_t)pb.biases & 15) == 0) ? 1 : 0;
+    p.sb16 = sb16 ? 1 : 0;
     const bool bf = pb.xdt == DT::BF16;
     const int warps = s.wr * s.wk;
     switch (pb.bits) {

@@ -438,6 +438,27 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
     // now; this grid reads nothing an earlier kernel may write (x, W, scales, biases, offsets)
     // and writes no y before the earlier grids have completed.
     ptx::pdl_launch_dependents();
+    if (!p.offsets && warp == 0) {
+        // The W stages, scales and biases of the CTA's first two tiles go to L2 while the previous
+        // kernel in the stream may still run: prefetches change no value that any load sees, so
+        // they are safe before the wait.  (Grouped tiles depend on the device offsets: none.)
+        const int cs0 = p.ksplit;
+        const int rk = cs0 > 1 ? (int)(blockIdx.x % cs0) : 0;
+        const int t0 = cs0 > 1 ? (int)(blockIdx.x / cs0) : (int)blockIdx.x;
+        const int nt_all = p.n_wtiles * p.n_ttiles * p.nbatch;
+        int pw0 = 0, pw1 = NWS;
+        if (cs0 > 1) split_range(NWS, GPS, cs0, rk, &pw0, &pw1);
+        for (int k = 0; k < (cs0 > 1 ? 1 : 2); ++k) {
+            const int t = t0 + k * (int)gridDim.x;
+            if (t >= nt_all) break;
+            const int64_t n0 = (int64_t)(t % p.n_wtiles) * 128;
+            if (lane == 0)
+                for (int w = pw0; w < pw1; ++w) ptx::tma_prefetch_2d(&p.tw, w * (ROWB / 4), (int32_t)n0);
+            const int64_t nr = min64(128, p.N - n0);
+            ptx::prefetch_l2_range(p.scales + n0 * p.kg, (size_t)nr * p.kg * 2, lane, 32);
+            ptx::prefetch_l2_range(p.biases + n0 * p.kg, (size_t)nr * p.kg * 2, lane, 32);
+        }
+    }
     ptx::pdl_wait();
     if (p.offsets && warp == 2) {
         // tiles per expert: ceil(count / NT) * n_wtiles, prefix-summed

@@ -105,6 +105,13 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
+// one box of a 2D tensor map into L2 (no shared-memory destination, no completion)
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* m, int32_t c0, int32_t c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+                 ::"l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t c0,
                                             int32_t c1) {
     asm volatile(
@@ -182,6 +189,24 @@ __device__ __forceinline__ void st_cluster_f4(uint32_t cluster_addr, float4 v) {
 // every prerequisite grid has completed and its memory operations are visible
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// L2 prefetches.  A prefetch only moves lines into L2, which every SM reads coherently: no load
+// sees a different value because of it, so a kernel may issue it for its weights before its
+// programmatic-dependent-launch wait, while the previous grid in the stream still runs.
+// Bulk form: [p, p + bytes), 16-byte aligned address and size.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+// one line
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
+// every 128-byte line of [p, p + bytes), spread over `nthr` threads (this one is `tid`)
+__device__ __forceinline__ void prefetch_l2_range(const void* p, size_t bytes, int tid, int nthr) {
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(p) & ~uintptr_t(127);
+    const uintptr_t hi = reinterpret_cast<uintptr_t>(p) + bytes;
+    for (uintptr_t a = lo + (uintptr_t)tid * 128; a < hi; a += (uintptr_t)nthr * 128)
+        prefetch_l2(reinterpret_cast<const void*>(a));
+}
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }

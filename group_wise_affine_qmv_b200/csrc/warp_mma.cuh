@@ -18,17 +18,35 @@ constexpr int RING_BYTES = 8192;     // per-warp ring of W sub-blocks in shared 
 constexpr int RED_PITCH = ROWS + 4;  // floats per token of a warp's partial y tile (bank spread)
 constexpr int MAX_XTAB_BYTES = 48 * 1024;
 
-struct WParams {
-    const uint16_t* x;       // [nb0, nb1, M, K] through xb / x_row
-    void* y;                 // [nb0, nb1, M, N] through yb / y_row
+constexpr int MAX_SEGS = 3;          // W matrices sharing one x in one launch
+
+// One W matrix of a launch, with its scales, biases and output.  A launch's W rows form one
+// "logical" row space cut into blocks of ROWS rows (one block per warp): segment s owns blocks
+// [rb0, rb0 + ceil(N / ROWS)) in the plain and fused-projection layouts.
+struct WSeg {
     const uint32_t* wq;      // [N, w_row] packed codes
     const uint16_t* scales;  // [N, kg]
     const uint16_t* biases;  // [N, kg]
-    int64_t M, N, K;
-    int64_t x_row, y_row;
+    void* y;                 // [nb0, nb1, M, N] through the launch's yb and this y_row
+    int64_t N;
+    int64_t w_row;           // words between W rows
+    int64_t y_row;           // elements between rows of y
+    int64_t rb0;             // first row block of the segment
+    const void* r;           // optional residual, y's dtype and layout: y = r + x . W^T (null: none)
+    int64_t r_row;           // elements between rows of r
+};
+
+struct WParams {
+    const uint16_t* x;       // [nb0, nb1, M, K] through xb / x_row
+    WSeg seg[MAX_SEGS];
+    int nseg;                // segments (1: a plain call)
+    int glu;                 // 1: segments 0 (gate) and 1 (up) share every row block, 16 rows
+                             //    each; the output is silu(gate) * up into segment 0's y
+    int64_t nrb;             // row blocks of the launch
+    int64_t M, K;
+    int64_t x_row;
     int64_t xb[2], yb[2];
     int64_t nb1;
-    int64_t w_row;           // words between W rows
     int kg;                  // groups per row (K / group)
     int cs;                  // CTAs of a cluster splitting K (1: no split)
     int kgc;                 // groups per CTA of a cluster (kg when cs == 1)

@@ -165,6 +165,13 @@ __device__ __forceinline__ void load_lane_words(const uint8_t* p, uint32_t* w) {
     }
 }
 
+// element `off` of a tensor of y's dtype (fp32, or the activation dtype XT), as fp32
+template <typename XT>
+__device__ __forceinline__ float load_out(const void* r, int64_t off, int ydt) {
+    if (ydt == (int)DT::F32) return reinterpret_cast<const float*>(r)[off];
+    return half_bits_to_float(reinterpret_cast<const uint16_t*>(r)[off], XT{});
+}
+
 template <typename XT>
 __device__ __forceinline__ void store_pair(void* y, int64_t off, float v0, float v1, bool both, bool vec, int ydt) {
     if (ydt == (int)DT::F32) {
@@ -181,6 +188,37 @@ __device__ __forceinline__ void store_pair(void* y, int64_t off, float v0, float
         else { p[0] = __float2half_rn(v0); if (both) p[1] = __float2half_rn(v1); }
     }
 }
+
+// Where logical row r of a launch lives: segment, row of that segment's W (clamped to its last
+// row for loads) and whether it exists.  Plain and fused-projection layouts: row block r / ROWS
+// belongs to the segment whose blocks contain it.  Gate/up layout: block b holds rows
+// 16 b .. 16 b + 15 of the gate matrix (logical rows 0..15 of the block) and the same rows of the
+// up matrix (logical rows 16..31), so both halves of every output sit in one warp's m tiles.
+struct RowRef {
+    int seg;
+    int64_t n;
+    bool valid;
+};
+__device__ __forceinline__ RowRef row_ref(const WParams& p, int64_t r) {
+    RowRef o;
+    const int64_t blk = r / ROWS;
+    const int j = (int)(r - blk * ROWS);
+    if (p.glu) {
+        o.seg = j >= ROWS / 2 ? 1 : 0;
+        o.n = blk * (ROWS / 2) + (j & (ROWS / 2 - 1));
+    } else {
+        int s = 0;
+        while (s + 1 < p.nseg && blk >= p.seg[s + 1].rb0) ++s;
+        o.seg = s;
+        o.n = (blk - p.seg[s].rb0) * ROWS + j;
+    }
+    const int64_t N = p.seg[o.seg].N;
+    o.valid = o.n < N;
+    if (!o.valid) o.n = N - 1;
+    return o;
+}
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
 
 template <int BITS, typename XT, int G, int NTL>
 __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __grid_constant__ WParams p) {
@@ -214,16 +252,32 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
     const int64_t bo = bz / p.nb1, bi = bz - bo * p.nb1;
     const uint16_t* x = p.x + bo * p.xb[0] + bi * p.xb[1];
     const int64_t tok0 = (int64_t)blockIdx.y * NT;
-    const int64_t rowc = (int64_t)(blockIdx.x / cs) * rows_cta; // first W row of the CTA
-    const int64_t roww = rowc + rw * ROWS;                       // first W row of this warp
+    const int64_t rowc = (int64_t)(blockIdx.x / cs) * rows_cta; // first logical row of the CTA
+    const int64_t roww = rowc + rw * ROWS;                       // first logical row of this warp
     const int cg0 = rank * p.kgc, cg1 = min(cg0 + p.kgc, kg);   // groups of this CTA
     const int ckg = cg1 > cg0 ? cg1 - cg0 : 0;
     const int g0 = cg0 + kw * p.gpw;                             // groups of this warp
     const int g1 = min(g0 + p.gpw, cg1);
-    const int nsub = (roww < p.N && g1 > g0) ? (g1 - g0) * SPG : 0;
+    const int nsub = (roww / ROWS < p.nrb && g1 > g0) ? (g1 - g0) * SPG : 0;
 
-    // x may be the output of the previous kernel in the stream: read nothing before it completed
     ptx::pdl_launch_dependents();
+    // The CTA's weights (its rows' K range of W, and their scales and biases) go to L2 while the
+    // previous kernel in the stream may still run: prefetches change no value that any load sees,
+    // so they are safe before the wait; the copies below then hit L2.
+    if (ckg > 0) {
+        const uint32_t seg = (uint32_t)ckg * (G * BITS / 8);   // a multiple of 16 bytes
+        for (int rl = threadIdx.x; rl < rows_cta; rl += blockDim.x) {
+            if ((rowc + rl) / ROWS >= p.nrb) break;
+            const RowRef rr = row_ref(p, rowc + rl);
+            if (!rr.valid) continue;
+            const WSeg& sg = p.seg[rr.seg];
+            ptx::prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(sg.wq + rr.n * sg.w_row) +
+                                      (size_t)cg0 * (G * BITS / 8), seg);
+            ptx::prefetch_l2_range(sg.scales + rr.n * kg + cg0, (size_t)ckg * 2, 0, 1);
+            ptx::prefetch_l2_range(sg.biases + rr.n * kg + cg0, (size_t)ckg * 2, 0, 1);
+        }
+    }
+    // x may be the output of the previous kernel in the stream: read nothing before it completed
     ptx::pdl_wait();
 
     // ---- one copy group: the scales and biases of the CTA's rows, and the x tile when it fits ----
@@ -234,14 +288,16 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
         const int total = rows_cta * cpr;
         for (int i = threadIdx.x; i < total; i += blockDim.x) {
             const int rl = i / cpr, col = i - rl * cpr;
-            const int64_t go = min(rowc + rl, p.N - 1) * kg + col * step;
+            const RowRef rr = row_ref(p, min(rowc + rl, p.nrb * ROWS - 1));
+            const WSeg& sg = p.seg[rr.seg];
+            const int64_t go = rr.n * kg + col * step;
             const uint32_t so = (uint32_t)((rl * kg + col * step) * 2);
             if (p.sb16) {
-                cp_async16(ss + so, p.scales + go);
-                cp_async16(sb + so, p.biases + go);
+                cp_async16(ss + so, sg.scales + go);
+                cp_async16(sb + so, sg.biases + go);
             } else {
-                cp_async4(ss + so, p.scales + go);
-                cp_async4(sb + so, p.biases + go);
+                cp_async4(ss + so, sg.scales + go);
+                cp_async4(sb + so, sg.biases + go);
             }
         }
         if (p.xsm) {   // codes [cg0 G, cg1 G) of every token row
@@ -265,8 +321,9 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
 #pragma unroll
         for (int i = 0; i < CPL; ++i) {
             const int q = lane + 32 * i, rl = q / CPR, col = q % CPR;
-            const int64_t n = min(roww + rl, p.N - 1);
-            csrc[i] = reinterpret_cast<const uint8_t*>(p.wq + n * p.w_row) + (int64_t)g0 * SPG * KSB + col * 16;
+            const RowRef rr = row_ref(p, min(roww + rl, p.nrb * ROWS - 1));
+            const WSeg& sg = p.seg[rr.seg];
+            csrc[i] = reinterpret_cast<const uint8_t*>(sg.wq + rr.n * sg.w_row) + (int64_t)g0 * SPG * KSB + col * 16;
             cdst[i] = ring_s + (uint32_t)(rl * KSB + col * 16);
         }
     }
@@ -419,25 +476,52 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
     }
     __syncthreads();
 
-    // ---- sum the warps' K slices in slice order; without a cluster, store pairs of adjacent
-    // outputs; with one, keep the CTA's partial tile for the cluster-wide sum ----
-    const int rpairs = p.wr * (ROWS / 2);
-    const int total = NT * rpairs;
+    // ---- outputs: sum the warps' K slices in slice order; without a cluster, store; with one,
+    // keep the CTA's partial tile for the cluster-wide sum.  An output item is a pair of adjacent
+    // rows of one segment's y, or (gate/up layout) a pair of adjacent silu(gate) * up values, whose
+    // gate and up sums sit 16 logical rows apart in the same row block. ----
+    const int ipb = p.glu ? ROWS / 4 : ROWS / 2;   // items per row block
+    const int ipt = p.wr * ipb;                    // items per token
+    const int total = NT * ipt;
     const int64_t ybase = bo * p.yb[0] + bi * p.yb[1];
-    for (int i = threadIdx.x; i < total; i += blockDim.x) {
-        const int tt = i / rpairs, rp = i - tt * rpairs;
-        const int wrr = rp / (ROWS / 2), rl = 2 * (rp % (ROWS / 2));
-        const int64_t tok = tok0 + tt, n = rowc + wrr * ROWS + rl;
-        if (cs == 1 && (tok >= p.M || n >= p.N)) continue;
-        float v0 = 0.0f, v1 = 0.0f;
-        for (int k = 0; k < p.wk; ++k) {
-            const float* part = reinterpret_cast<const float*>(smem + (size_t)(k * p.wr + wrr) * RING_BYTES);
-            const float2 u = *reinterpret_cast<const float2*>(part + tt * RED_PITCH + rl);
-            v0 += u.x;
-            v1 += u.y;
+    // local logical row of item element e (0, 1) and half (0: the value, or gate; 1: up)
+    auto lrow = [&](int wrr, int it, int e, int half) {
+        return wrr * ROWS + (p.glu ? 2 * it + e + half * (ROWS / 2) : 2 * it + e);
+    };
+    auto emit = [&](int tt, int wrr, int it, const float (&v)[2][2]) {
+        const int64_t tok = tok0 + tt;
+        const RowRef rr = row_ref(p, rowc + lrow(wrr, it, 0, 0));
+        if (tok >= p.M || !rr.valid) return;
+        const WSeg& sg = p.seg[p.glu ? 0 : rr.seg];
+        const bool both = rr.n + 1 < sg.N;
+        float o0 = v[0][0], o1 = v[1][0];
+        if (p.glu) {
+            o0 = silu(v[0][0]) * v[0][1];
+            o1 = silu(v[1][0]) * v[1][1];
         }
-        if (cs == 1) store_pair<XT>(p.y, ybase + tok * p.y_row + n, v0, v1, n + 1 < p.N, p.yvec != 0, p.ydt);
-        else *reinterpret_cast<float2*>(cpart + tt * rows_cta + wrr * ROWS + rl) = make_float2(v0, v1);
+        if (sg.r) {   // residual: added in fp32 before the one rounding to y's dtype
+            const int64_t ro = ybase + tok * sg.r_row + rr.n;
+            o0 += load_out<XT>(sg.r, ro, p.ydt);
+            if (both) o1 += load_out<XT>(sg.r, ro + 1, p.ydt);
+        }
+        store_pair<XT>(sg.y, ybase + tok * sg.y_row + rr.n, o0, o1, both, p.yvec != 0, p.ydt);
+    };
+    for (int i = threadIdx.x; i < total; i += blockDim.x) {
+        const int tt = i / ipt, rp = i - tt * ipt;
+        const int wrr = rp / ipb, it = rp - wrr * ipb;
+        float v[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
+        for (int hf = 0; hf < (p.glu ? 2 : 1); ++hf) {
+            const int rl = lrow(wrr, it, 0, hf) - wrr * ROWS;   // even: the pair is one float2
+            for (int k = 0; k < p.wk; ++k) {
+                const float* part = reinterpret_cast<const float*>(smem + (size_t)(k * p.wr + wrr) * RING_BYTES);
+                const float2 u = *reinterpret_cast<const float2*>(part + tt * RED_PITCH + rl);
+                v[0][hf] += u.x;
+                v[1][hf] += u.y;
+            }
+            if (cs > 1)
+                *reinterpret_cast<float2*>(cpart + tt * rows_cta + wrr * ROWS + rl) = make_float2(v[0][hf], v[1][hf]);
+        }
+        if (cs == 1) emit(tt, wrr, it, v);
     }
     if (cs > 1) {
         // every CTA's partial tile is complete and visible cluster-wide (hardware barrier)
@@ -448,18 +532,18 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
         const int i0 = rank * per, i1 = min(i0 + per, total);
         const uint32_t cp_s = ptx::smem_u32(cpart);
         for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
-            const int tt = i / rpairs, rp = i - tt * rpairs;
-            const int wrr = rp / (ROWS / 2), rl = 2 * (rp % (ROWS / 2));
-            const int64_t tok = tok0 + tt, n = rowc + wrr * ROWS + rl;
-            if (tok >= p.M || n >= p.N) continue;
-            const uint32_t off = (uint32_t)((tt * rows_cta + wrr * ROWS + rl) * 4);
-            float v0 = 0.0f, v1 = 0.0f;
-            for (int q = 0; q < cs; ++q) {
-                const float2 u = ptx::ld_cluster_f2(ptx::mapa(cp_s + off, (uint32_t)q));
-                v0 += u.x;
-                v1 += u.y;
+            const int tt = i / ipt, rp = i - tt * ipt;
+            const int wrr = rp / ipb, it = rp - wrr * ipb;
+            float v[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
+            for (int hf = 0; hf < (p.glu ? 2 : 1); ++hf) {
+                const uint32_t off = (uint32_t)((tt * rows_cta + lrow(wrr, it, 0, hf)) * 4);
+                for (int q = 0; q < cs; ++q) {
+                    const float2 u = ptx::ld_cluster_f2(ptx::mapa(cp_s + off, (uint32_t)q));
+                    v[0][hf] += u.x;
+                    v[1][hf] += u.y;
+                }
             }
-            store_pair<XT>(p.y, ybase + tok * p.y_row + n, v0, v1, n + 1 < p.N, p.yvec != 0, p.ydt);
+            emit(tt, wrr, it, v);
         }
         // no CTA leaves while another may still read its partial tile
         asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");

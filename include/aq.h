@@ -172,6 +172,56 @@ aq_status aq_qmm_t_grouped(const aq_view* x_sorted, const int64_t* offsets, int 
                            int group, int bits, const aq_view* y_sorted, void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Fused calls of a decoder layer's decode step (warp-level kernel).       */
+/*                                                                        */
+/* The decode step the pages' bug reports run (transformers issue #47331, */
+/* reproduction: a Qwen3-0.6B decoder under generate(), every projection  */
+/* an affine_qmm_t on x [B, 1, hidden]; "mlx PR #4516": the narrow decode */
+/* projections dominate decode time) makes seven small calls per layer.   */
+/* These entry points do the same arithmetic as aq_qmm_t -- W exact,      */
+/* factored s*sum(q*x) + b*sum(x) with x widened to fp32 before it is     */
+/* summed -- in fewer launches.  x and every output must fold into one 2D */
+/* problem (no launch batch dims) and W is unbatched.                     */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * aq_qmm_t_multi -- n (1..3) matrices that share one input, in one launch:
+ *     y[j] = x . dequant(W_j)^T,  j < n       (e.g. the q, k and v projections)
+ * wq[j], scales[j], biases[j], y[j] as for aq_qmm_t, each W_j with its own N_j and
+ * the same K; no output may overlap another output or any input.
+ * One launch of the warp-level kernel when it takes every matrix (up to 32 rows in
+ * total, 2/4/8-bit codes, 16-byte aligned rows); otherwise one aq_qmm_t per matrix,
+ * in order, on the same stream (same results to the same bar).
+ */
+aq_status aq_qmm_t_multi(const aq_view* x, int n, const aq_view* const* wq, const aq_view* const* scales,
+                         const aq_view* const* biases, int group, int bits, const aq_view* const* y,
+                         void* stream);
+
+/*
+ * aq_qmm_t_swiglu -- the gated MLP input of the decoder layer, in one launch:
+ *     y = silu(x . dequant(W_gate)^T) * (x . dequant(W_up)^T),  silu(v) = v / (1 + exp(-v))
+ * Both contractions are complete fp32 sums before the activation; y is rounded once.
+ * W_gate and W_up: [N, K*bits/32] with their scales and biases; y: x.shape[:-1] + [N].
+ * (The activation is a reading: the issue names the model, whose MLP is
+ * down(silu(gate(h)) * up(h)); the pages do not spell it out.)
+ * Warp-level kernel only; AQ_ERR_UNSUPPORTED where it does not take the problem.
+ */
+aq_status aq_qmm_t_swiglu(const aq_view* x, const aq_view* wq_gate, const aq_view* s_gate,
+                          const aq_view* b_gate, const aq_view* wq_up, const aq_view* s_up,
+                          const aq_view* b_up, int group, int bits, const aq_view* y, void* stream);
+
+/*
+ * aq_qmm_t_residual -- a projection that adds into the residual stream, in one launch:
+ *     y = r + x . dequant(W)^T
+ * r has y's shape and dtype; the sum is formed in fp32 and rounded once.  r may be y
+ * itself (the same view: an in-place update) but must not overlap it otherwise.
+ * Warp-level kernel only; AQ_ERR_UNSUPPORTED where it does not take the problem.
+ */
+aq_status aq_qmm_t_residual(const aq_view* x, const aq_view* wq, const aq_view* scales,
+                            const aq_view* biases, int group, int bits, const aq_view* r,
+                            const aq_view* y, void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Introspection (host only, no GPU work).                                 */
 /* ---------------------------------------------------------------------- */
 

@@ -17,6 +17,8 @@ arrays into it.  Function-level citations are in the C file; in short:
 * ``dequant``     -- w' = s*q + b with the stored half-precision s, b, in fp64.
 * ``linear``      -- y = x . w'^T in fp64, reading x through its strided view.
 * ``linear_grouped`` -- the same per expert segment of a row-sorted x.
+* ``silu`` / ``swiglu`` -- silu(g) * u in fp64 (the gated MLP step of the fused
+  gate/up call).
 """
 from __future__ import annotations
 
@@ -77,6 +79,10 @@ def _load():
             lib.oracle_linear_grouped.restype = ci
             lib.oracle_factored_dot.argtypes = [vp, ci, vp, vp, vp, ci, i64, ci]
             lib.oracle_factored_dot.restype = ctypes.c_double
+            lib.oracle_silu.argtypes = [ctypes.c_double]
+            lib.oracle_silu.restype = ctypes.c_double
+            lib.oracle_swiglu.argtypes = [vp, vp, i64, vp]
+            lib.oracle_swiglu.restype = None
             lib.oracle_half_to_double.argtypes = [ctypes.c_uint16, ci]
             lib.oracle_half_to_double.restype = ctypes.c_double
             lib.oracle_float_to_half_rne.argtypes = [ctypes.c_float, ci]
@@ -296,3 +302,19 @@ def factored_dot(x_bits: np.ndarray, x_dtype: str, codes: np.ndarray, scale_bits
     bb = np.ascontiguousarray(bias_bits, dtype=np.uint16)
     return lib.oracle_factored_dot(_ptr(x), _dtype_code(x_dtype), _ptr(q), _ptr(sb), _ptr(bb),
                                    _dtype_code(sdtype), x.shape[-1], group)
+
+
+def silu(v: float) -> float:
+    """silu(v) = v / (1 + exp(-v)) in fp64."""
+    return _load().oracle_silu(float(v))
+
+
+def swiglu(g: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """silu(g) * u elementwise, fp64 (g, u: fp64 results of the gate and up contractions)."""
+    lib = _load()
+    g = np.ascontiguousarray(g, dtype=np.float64)
+    u = np.ascontiguousarray(u, dtype=np.float64)
+    assert g.shape == u.shape
+    out = np.empty(g.shape, np.float64)
+    lib.oracle_swiglu(_ptr(g), _ptr(u), g.size, _ptr(out))
+    return out

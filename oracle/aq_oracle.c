@@ -20,6 +20,11 @@
  *  - The affine rule w = scale*q + bias with scale = (max-min)/(2^bits-1),
  *    bias = min, round to nearest, clamp; 3/5/6-bit codes form a dense
  *    little-endian bitstream (the method statement that accompanies the pages).
+ *  - The gated MLP of the decoder that the decode workload is drawn from (transformers
+ *    issue #47331, reproduction: a Qwen3-0.6B decoder layer, whose MLP is
+ *    down(silu(gate(h)) * up(h))): silu(v) = v / (1 + exp(-v)), the one step of the
+ *    fused gate/up call that is not a contraction (a reading: the page names the model,
+ *    not its activation).
  *  - "mlx PR #4516" (load_vector fix): the bias term bias*sum(x) must be formed
  *    from inputs widened before they are added; the oracle does every sum in
  *    fp64, which is the exact value that fix aims at.
@@ -366,4 +371,16 @@ double oracle_factored_dot(const uint16_t* x, int xdtype, const uint8_t* codes,
                  oracle_half_to_double(bias_s[g], sdtype) * sx;
     }
     return total;
+}
+
+/*
+ * oracle_swiglu -- out[i] = silu(g[i]) * u[i], silu(v) = v / (1 + exp(-v)), all in fp64 (the
+ * gated MLP of the Qwen3-0.6B decoder of transformers issue #47331's reproduction; the
+ * activation is a reading, see the file header).  g and u are the fp64 results of the gate and
+ * up contractions.
+ */
+double oracle_silu(double v) { return v / (1.0 + exp(-v)); }
+
+void oracle_swiglu(const double* g, const double* u, int64_t n, double* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_silu(g[i]) * u[i];
 }

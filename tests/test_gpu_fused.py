@@ -1,0 +1,215 @@
+"""GPU parity of the fused decode-layer calls (warp-level kernel) against the oracle, and of a
+decode chain captured in a CUDA graph.
+
+* aq_qmm_t_multi: up to three matrices sharing x (the q, k, v projections), one launch;
+* aq_qmm_t_swiglu: silu(x . Wg^T) * (x . Wu^T), one launch;
+* aq_qmm_t_residual: r + x . W^T, in place or into a separate y;
+* a chain of decoder layers in which every call reads the previous call's output, launched as
+  programmatic dependents inside one CUDA graph and replayed: checks that no kernel reads its
+  input before the kernel that writes it has finished (the kernels prefetch weights before that
+  wait, never activations).
+
+The decoder layer the chain follows is the one of transformers issue #47331's reproduction (a
+Qwen3-0.6B decoder, every projection a quantized linear on x [B, 1, hidden]): per layer
+q, k, v = multi(h); h += o(v); a = swiglu(h); h += down(a); then lm_head(h).  Attention itself is
+outside the path: o reads v, which is what attention returns with a single cached position.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from group_wise_affine_qmv_b200 import aq, inputs
+from tests.parity import dtype_name, half_bits, oracle_linear_view, row_errors, to_device_quant
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+DEV = "cuda"
+
+
+def _q(w, group, bits, sdtype="bf16"):
+    Q = oracle.quantize(w.float().numpy(), group, bits, sdtype)
+    tdt = torch.bfloat16 if sdtype == "bf16" else torch.float16
+    return Q, to_device_quant(Q, DEV, tdt)
+
+
+def _kernel(x, wq, sc, bi, group, bits):
+    y = torch.empty(tuple(x.shape[:-1]) + (wq.shape[-2],), dtype=x.dtype, device=x.device)
+    return aq.aq_plan_linear(x, wq, sc, bi, group, bits, y)["kernel"]
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("M,Ns,K", [(1, (100, 37, 64), 512), (5, (100, 37, 64), 512), (8, (2048, 1024, 1024), 1024),
+                                    (32, (2048, 1024, 1024), 1024), (32, (33, 1, 300), 256), (16, (4099, 7), 4096)])
+def test_multi_matches_oracle(bits, M, Ns, K):
+    group = 64
+    x = inputs.normal((M, 1, K), 1.0, torch.bfloat16, seed=M + K)
+    xd = x.to(DEV)
+    Qs, ws = [], []
+    for j, N in enumerate(Ns):
+        Q, w = _q(inputs.normal((N, K), 0.02, seed=100 * j + N + bits), group, bits)
+        Qs.append(Q)
+        ws.append(w)
+    ys = aq.aq_qmm_t_multi(xd, ws, group, bits)
+    for Q, y in zip(Qs, ys):
+        err = row_errors(y, oracle_linear_view(x, Q.dequant()))
+        assert err.size == M and np.all(err <= 4e-3), (err.max(), int(err.argmax()))
+
+
+def test_multi_falls_back_to_plain_calls():
+    """40 rows: the warp-level kernel does not take them, so each matrix runs as a plain call."""
+    K, group, bits = 512, 64, 4
+    x = inputs.normal((40, K), 1.0, torch.bfloat16, seed=3)
+    Qs, ws = zip(*[_q(inputs.normal((N, K), 0.02, seed=N), group, bits) for N in (256, 130)])
+    ys = aq.aq_qmm_t_multi(x.to(DEV), list(ws), group, bits)
+    for Q, w, y in zip(Qs, ws, ys):
+        assert np.all(row_errors(y, oracle_linear_view(x, Q.dequant())) <= 4e-3)
+        assert torch.equal(y, aq.aq_qmm_t(x.to(DEV), *w, group, bits))
+
+
+def test_multi_rejects_overlapping_outputs():
+    K, group, bits = 256, 64, 4
+    _, w = _q(inputs.normal((64, K), 0.02, seed=1), group, bits)
+    x = torch.zeros(8, K, dtype=torch.bfloat16, device=DEV)
+    buf = torch.empty(8, 96, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(aq.AQError) as ei:
+        aq.aq_qmm_t_multi(x, [w, w], group, bits, outs=[buf[:, :64], buf[:, 32:96]])
+    assert ei.value.name == "AQ_ERR_OVERLAP"
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("M,N,K", [(1, 3072, 1024), (8, 1000, 1024), (32, 3072, 1024), (32, 17, 512),
+                                   (13, 4099, 2048)])
+def test_swiglu_matches_oracle(bits, M, N, K):
+    group = 64
+    x = inputs.normal((M, 1, K), 1.0, torch.bfloat16, seed=M * 3 + N)
+    xd = x.to(DEV)
+    Qg, wg = _q(inputs.normal((N, K), 0.02, seed=N + 1), group, bits)
+    Qu, wu = _q(inputs.normal((N, K), 0.02, seed=N + 2), group, bits)
+    y = aq.aq_qmm_t_swiglu(xd, wg, wu, group, bits)
+    g = oracle_linear_view(x, Qg.dequant())
+    u = oracle_linear_view(x, Qu.dequant())
+    ref = oracle.swiglu(g, u)
+    err = row_errors(y, ref)
+    assert err.size == M and np.all(err <= 4e-3), (err.max(), int(err.argmax()))
+    # fp32 output: the two contractions in fp32, the activation in fp32
+    y32 = aq.aq_qmm_t_swiglu(xd, wg, wu, group, bits, out_dtype=torch.float32)
+    assert np.all(row_errors(y32, ref) <= 1e-4)
+
+
+@pytest.mark.parametrize("xdtype", [torch.bfloat16, torch.float16])
+def test_swiglu_dtypes_and_groups(xdtype):
+    M, N, K, bits = 24, 520, 2048, 4
+    sd = dtype_name(torch.empty(0, dtype=xdtype))
+    x = inputs.normal((M, K), 1.0, xdtype, seed=5)
+    for group in (32, 64, 128):
+        Qg, wg = _q(inputs.normal((N, K), 0.02, seed=group), group, bits, sd)
+        Qu, wu = _q(inputs.normal((N, K), 0.02, seed=group + 1), group, bits, sd)
+        y = aq.aq_qmm_t_swiglu(x.to(DEV), wg, wu, group, bits)
+        ref = oracle.swiglu(oracle_linear_view(x, Qg.dequant()), oracle_linear_view(x, Qu.dequant()))
+        assert np.all(row_errors(y, ref) <= 4e-3), group
+
+
+def test_swiglu_unsupported_shape():
+    K, group, bits = 512, 64, 4
+    _, w = _q(inputs.normal((64, K), 0.02, seed=1), group, bits)
+    x = torch.zeros(40, K, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(aq.AQError) as ei:
+        aq.aq_qmm_t_swiglu(x, w, w, group, bits)
+    assert ei.value.name == "AQ_ERR_UNSUPPORTED"
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M", [1, 8, 32])
+@pytest.mark.parametrize("inplace", [False, True])
+def test_residual_matches_oracle(bits, M, inplace):
+    K, N, group = 1024, 1024, 64
+    x = inputs.normal((M, 1, K), 1.0, torch.bfloat16, seed=M + 7)
+    r = inputs.normal((M, 1, N), 1.0, torch.bfloat16, seed=M + 8)
+    Q, w = _q(inputs.normal((N, K), 0.02, seed=N + bits), group, bits)
+    rd = r.to(DEV)
+    if inplace:
+        y = aq.aq_qmm_t_residual(x.to(DEV), *w, group, bits, r=rd, out=rd)
+        assert y.data_ptr() == rd.data_ptr()
+    else:
+        y = aq.aq_qmm_t_residual(x.to(DEV), *w, group, bits, r=rd)
+        assert torch.equal(rd.cpu(), r)
+    ref = r.double().numpy() + oracle_linear_view(x, Q.dequant())
+    assert np.all(row_errors(y, ref) <= 4e-3)
+
+
+# ---------------------------------------------------------------------------
+# the decode chain, graph-captured, against the oracle's own chain
+# ---------------------------------------------------------------------------
+
+def _bf16_round(v: np.ndarray) -> np.ndarray:
+    """What the GPU stores for an fp64 value: the nearest bf16 (through fp32)."""
+    bits = oracle.float_to_half_bits(v.astype(np.float32), "bf16")
+    return oracle.half_to_double(bits, "bf16")
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_decode_chain_graph(bits):
+    layers, B, group, vocab = 3, inputs.DECODE_BATCH, inputs.DECODE_GROUP, 4096
+    proj = {name: (K, N) for name, K, N in inputs.DECODE_PROJ}
+    Q = {}
+    W = {}
+    for l in range(layers):
+        for i, name in enumerate(("q", "k", "v", "o", "gate", "up", "down")):
+            K, N = proj[name]
+            Q[l, name], W[l, name] = _q(inputs.decode_w(K, N, seed=1000 * l + i), group, bits)
+    Q["lm"], W["lm"] = _q(inputs.decode_w(1024, vocab, seed=5), group, bits)
+    h0 = inputs.decode_x(1024, seed=11)
+    h0d = h0.to(DEV)
+    h = torch.empty_like(h0d)
+    q = torch.empty(B, 1, 2048, dtype=torch.bfloat16, device=DEV)
+    k = torch.empty(B, 1, 1024, dtype=torch.bfloat16, device=DEV)
+    v = torch.empty_like(k)
+    a = torch.empty(B, 1, 3072, dtype=torch.bfloat16, device=DEV)
+    logits = torch.empty(B, 1, vocab, dtype=torch.bfloat16, device=DEV)
+
+    def step():
+        for l in range(layers):
+            aq.aq_qmm_t_multi(h0d if l == 0 else h, [W[l, "q"], W[l, "k"], W[l, "v"]], group, bits, outs=[q, k, v])
+            aq.aq_qmm_t_residual(v, *W[l, "o"], group, bits, r=h0d if l == 0 else h, out=h)
+            aq.aq_qmm_t_swiglu(h, W[l, "gate"], W[l, "up"], group, bits, out=a)
+            aq.aq_qmm_t_residual(a, *W[l, "down"], group, bits, r=h, out=h)
+        aq.aq_qmm_t(h, *W["lm"], group, bits, out=logits)
+
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.synchronize()
+    eager = logits.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    results = []
+    for _ in range(3):
+        logits.zero_()
+        h.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        results.append(logits.clone())
+    aq.aq_device_error()
+    del g
+    for r_ in results:
+        assert torch.equal(r_, eager)
+
+    # the oracle's chain: fp64 contractions, every stored activation rounded to bf16 as the GPU does
+    def _bf16_round_lin(xv, Qk):
+        xb = half_bits(torch.from_numpy(xv.astype(np.float32)).to(torch.bfloat16)).reshape(B, -1)
+        return oracle.linear_contig(xb, "bf16", Qk.dequant())
+
+    hv = h0.reshape(B, 1024).double().numpy()
+    for l in range(layers):
+        vv = _bf16_round(_bf16_round_lin(hv, Q[l, "v"]))
+        hv = _bf16_round(hv + _bf16_round_lin(vv, Q[l, "o"]))
+        av = _bf16_round(oracle.swiglu(_bf16_round_lin(hv, Q[l, "gate"]), _bf16_round_lin(hv, Q[l, "up"])))
+        hv = _bf16_round(hv + _bf16_round_lin(av, Q[l, "down"]))
+    ref = _bf16_round_lin(hv, Q["lm"])
+    err = row_errors(results[-1], ref)
+    assert err.size == B and np.all(err <= 4e-3), (err.max(), int(err.argmax()))
+    # and the residual stream after the last layer
+    assert np.all(row_errors(h, hv) <= 4e-3)

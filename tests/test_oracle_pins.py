@@ -388,3 +388,39 @@ def test_probe_error_magnitude_matches_issue(orc):
     ref = orc.linear_contig(lib_half_bits(x), "bf16", ref_w)
     err = np.abs(y_bf16 - ref).max(-1) / np.abs(ref).max(-1)
     assert np.all((err > 0.002) & (err < 0.012)), err
+
+
+# ---------------------------------------------------------------------------
+# the gated-MLP activation of the fused gate/up call
+# ---------------------------------------------------------------------------
+
+def test_silu_closed_values(orc):
+    """silu(v) = v * sigmoid(v): zero at zero; v*sigmoid(v) at hand-known sigmoid values
+    (sigmoid(1) = 1 / (1 + 1/e) = 0.7310585786300049, sigmoid(2) = 0.8807970779778823); tends to v
+    for large v and to 0 from below for large negative v; silu(v) - silu(-v) = v."""
+    assert orc.silu(0.0) == 0.0
+    assert abs(orc.silu(1.0) - 0.7310585786300049) <= 1e-15
+    assert abs(orc.silu(2.0) - 2 * 0.8807970779778823) <= 1e-15
+    assert abs(orc.silu(-1.0) - (-(1 - 0.7310585786300049))) <= 1e-15
+    assert orc.silu(40.0) == 40.0
+    assert -1e-15 < orc.silu(-40.0) < 0.0
+    for v in (0.25, 1.5, 3.0, 7.75):
+        assert abs((orc.silu(v) - orc.silu(-v)) - v) <= 1e-15 * max(1.0, v)
+    # minimum of silu near v = -1.2785 (silu'(v) = 0 there), value -0.2784645427610738
+    vs = np.linspace(-1.4, -1.15, 2001)
+    vals = np.array([orc.silu(v) for v in vs])
+    assert abs(vs[vals.argmin()] - (-1.2784645)) < 2e-4
+    assert abs(vals.min() - (-0.2784645427610738)) < 1e-9
+
+
+def test_swiglu_elementwise(orc):
+    """swiglu(g, u) = silu(g) * u element by element, any shape."""
+    g = np.array([[0.0, 1.0, -1.0], [2.0, 40.0, -3.5]])
+    u = np.array([[5.0, 2.0, -4.0], [0.5, 0.25, 1.0]])
+    out = orc.swiglu(g, u)
+    assert out.shape == g.shape
+    assert out[0, 0] == 0.0
+    assert abs(out[0, 1] - 2 * 0.7310585786300049) <= 1e-15
+    assert abs(out[0, 2] - (-4.0) * (-(1 - 0.7310585786300049))) <= 1e-15
+    assert abs(out[1, 0] - 0.5 * 2 * 0.8807970779778823) <= 1e-15
+    assert out[1, 1] == 10.0
