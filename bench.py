@@ -675,26 +675,49 @@ def reference(args):
 
 
 CASES = ("lm_head_w4", "lm_head_w8", "lm_head2x_w4", "prefill_w4", "prefill_w8", "k_w4", "k_w8", "down_w4",
-         "down_w8")
+         "down_w8", "qkv_w4", "qkv_w8", "gateup_w4", "gateup_w8", "layer_w4", "layer_w8")
 
 
 def single_case(name, reps):
     """One shape alone, for profiling: `reps` timed calls after two warm-up calls (CUDA events).
     lm_head*: x [32, 1, 1024] against W [151936, 1024] (2x: 303872 rows, > L2); k*, down*: x
     [32, 1, K] against the decode step's k (W [1024, 1024]) or down (W [1024, 3072]) projection;
-    prefill*: x [2, 2048, 4096] against W [14336, 4096]; G = 64, weights quantized on the device."""
+    qkv*: the fused q/k/v call; gateup*: the fused gate/up + silu*mul call; layer*: the four
+    chained launches of one decoder layer; prefill*: x [2, 2048, 4096] against W [14336, 4096];
+    G = 64, weights quantized on the device."""
     from group_wise_affine_qmv_b200 import aq
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     bits = int(name[-1])
+    B = inputs.DECODE_BATCH
+    if name.startswith(("qkv", "gateup", "layer")):
+        W, A = build_workload(device, 1)
+        W = {bits: W[bits]}
+        m = W[bits]["layers"][0]
+        Ab = A[bits]
+        if name.startswith("qkv"):
+            fn = lambda: aq.aq_qmm_t_multi(A["h0"], [m["q"], m["k"], m["v"]], GROUP, bits,
+                                           outs=[Ab["q"], Ab["k"], Ab["v"]])
+            nbytes = layer_launch_bytes(bits)[0]
+        elif name.startswith("gateup"):
+            fn = lambda: aq.aq_qmm_t_swiglu(A["h0"], m["gate"], m["up"], GROUP, bits, out=Ab["a"])
+            nbytes = layer_launch_bytes(bits)[2]
+        else:
+            fn = lambda: run_layers(W, A, bits)
+            nbytes = sum(layer_launch_bytes(bits))
+        ms = time_calls(fn, reps, torch.cuda.current_stream())
+        aq.aq_device_error()
+        print(json.dumps({"case": name, "bits": bits, "us": round(ms * 1e3, 2), "GBps": round(nbytes / ms / 1e6, 1)}),
+              flush=True)
+        return
     if name.startswith(("lm_head", "k_", "down_")):
         if name.startswith("lm_head"):
             K, N = 1024, inputs.LM_HEAD[2] * (2 if name.startswith("lm_head2x") else 1)
         else:
             _, K, N = {p[0]: p for p in inputs.DECODE_PROJ}[name.split("_")[0]]
         x = inputs.decode_x(K, device=device)
-        y = torch.empty(inputs.DECODE_BATCH, 1, N, dtype=torch.bfloat16, device=device)
-        M = inputs.DECODE_BATCH
+        y = torch.empty(B, 1, N, dtype=torch.bfloat16, device=device)
+        M = B
     else:
         K, N = inputs.PREFILL_W_UP[1], inputs.PREFILL_W_UP[0]
         x = inputs.normal((2, 2048, K), 1.0, torch.bfloat16, seed=5, device=device)

@@ -50,7 +50,7 @@ class AqPlan(ctypes.Structure):
                 ("y_row_stride", ctypes.c_int64), ("total_rows", ctypes.c_int64)]
 
 
-EXPORTED = ("aq_quantize", "aq_dequantize", "aq_qmv", "aq_qmm_t", "aq_qmm_t_grouped", "aq_qmm_t_multi",
+EXPORTED = ("aq_quantize", "aq_dequantize", "aq_dequantize_rows", "aq_qmv", "aq_qmm_t", "aq_qmm_t_grouped", "aq_qmm_t_multi",
             "aq_qmm_t_swiglu", "aq_qmm_t_residual", "aq_plan_linear", "aq_status_string", "aq_last_error_message",
             "aq_device_error", "aq_version")
 
@@ -77,6 +77,8 @@ def load_library(path: str = LIB_PATH):
         lib.aq_quantize.restype = ci
         lib.aq_dequantize.argtypes = [V, V, V, ci, ci, V, vp]
         lib.aq_dequantize.restype = ci
+        lib.aq_dequantize_rows.argtypes = [V, V, V, ci, ci, vp, ctypes.c_int64, V, vp]
+        lib.aq_dequantize_rows.restype = ci
         lib.aq_qmm_t_grouped.argtypes = [V, vp, ci, V, V, V, ci, ci, V, vp]
         lib.aq_qmm_t_grouped.restype = ci
         VA = ctypes.POINTER(V)
@@ -154,6 +156,21 @@ def aq_dequantize(wq, scales, biases, group: int, bits: int, dtype: torch.dtype 
     out = torch.empty((N, K), dtype=dtype, device=wq.device)
     with torch.cuda.device(wq.device):
         _check(lib, lib.aq_dequantize(view(wq), view(scales), view(biases), group, bits, view(out), _stream(wq)))
+    return out
+
+
+def aq_dequantize_rows(wq, scales, biases, group: int, bits: int, ids, dtype: torch.dtype = torch.bfloat16,
+                       out=None):
+    """Rows ids of the quantized table, dequantized: out [len(ids), K] (ids: int64 CUDA tensor)."""
+    lib = load_library()
+    if ids.dtype != torch.int64 or not ids.is_cuda or ids.dim() != 1 or not ids.is_contiguous():
+        raise TypeError("ids must be a contiguous 1D int64 CUDA tensor")
+    K = wq.shape[1] * 32 // bits
+    if out is None:
+        out = torch.empty((ids.numel(), K), dtype=dtype, device=wq.device)
+    with torch.cuda.device(wq.device):
+        _check(lib, lib.aq_dequantize_rows(view(wq), view(scales), view(biases), group, bits,
+                                           ctypes.c_void_p(ids.data_ptr()), ids.numel(), view(out), _stream(wq)))
     return out
 
 

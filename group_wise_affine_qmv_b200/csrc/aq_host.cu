@@ -478,6 +478,7 @@ AQ_API const char* aq_status_string(aq_status s) {
         case AQ_ERR_CUDA: return "AQ_ERR_CUDA";
         case AQ_ERR_DEVICE: return "AQ_ERR_DEVICE";
         case AQ_ERR_TIMEOUT: return "AQ_ERR_TIMEOUT";
+        case AQ_ERR_INDEX: return "AQ_ERR_INDEX";
     }
     return "AQ_ERR_UNKNOWN";
 }
@@ -519,6 +520,7 @@ AQ_API aq_status aq_quantize(const aq_view* w, int group, int bits, const aq_vie
     if (numel(w) == 0) return AQ_OK;
     if ((st = check_device()) != AQ_OK) return st;
     aq::QuantArgs a;
+    memset(&a, 0, sizeof a);
     a.w = w->data;
     a.wq = (uint32_t*)wq->data;
     a.scales = scales->data;
@@ -544,6 +546,7 @@ AQ_API aq_status aq_dequantize(const aq_view* wq, const aq_view* scales, const a
     if (numel(w_out) == 0) return AQ_OK;
     if ((st = check_device()) != AQ_OK) return st;
     aq::QuantArgs a;
+    memset(&a, 0, sizeof a);
     a.w = w_out->data;
     a.wq = (uint32_t*)wq->data;
     a.scales = scales->data;
@@ -633,7 +636,9 @@ AQ_API aq_status aq_device_error(void* stream) {
     int v = 0;
     cudaError_t e = aq::read_and_clear_device_error(&v, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
-    if (v != 0) return fail(AQ_ERR_TIMEOUT, "a kernel's bounded wait expired (code %d)", v);
+    if (v & aq::DEVERR_TIMEOUT) return fail(AQ_ERR_TIMEOUT, "a kernel's bounded wait expired (code %d)", v);
+    if (v & aq::DEVERR_INDEX) return fail(AQ_ERR_INDEX, "a row id was outside the table (code %d)", v);
+    if (v != 0) return fail(AQ_ERR_CUDA, "unknown device error code %d", v);
     return AQ_OK;
 }
 
@@ -752,4 +757,56 @@ AQ_API aq_status aq_qmm_t_residual(const aq_view* x, const aq_view* wq, const aq
     mp.r = r->data;
     mp.r_row = Rr.plan.y_row_stride;
     return launch_fused(mp, stream);
+}
+
+AQ_API aq_status aq_dequantize_rows(const aq_view* wq, const aq_view* scales, const aq_view* biases, int group,
+                                    int bits, const int64_t* ids, int64_t n_ids, const aq_view* out,
+                                    void* stream) {
+    g_msg[0] = 0;
+    aq_status st;
+    if ((st = check_view(out, "out", 2, 2)) != AQ_OK) return st;
+    if (n_ids < 0) return fail(AQ_ERR_SHAPE, "n_ids < 0");
+    if (out->shape[0] != n_ids) return fail(AQ_ERR_SHAPE, "out must have n_ids rows");
+    if ((st = check_output(out, "out")) != AQ_OK) return st;
+    if ((st = check_view(wq, "wq", 2, 2)) != AQ_OK) return st;
+    if ((st = check_view(scales, "scales", 2, 2)) != AQ_OK) return st;
+    if ((st = check_view(biases, "biases", 2, 2)) != AQ_OK) return st;
+    if ((st = check_bits_group(bits, group)) != AQ_OK) return st;
+    if (!(out->dtype == AQ_F32 || is_half(out->dtype))) return fail(AQ_ERR_DTYPE, "out must be f32, bf16 or f16");
+    if (wq->dtype != AQ_U32) return fail(AQ_ERR_DTYPE, "wq must be u32");
+    if (!is_half(scales->dtype) || biases->dtype != scales->dtype)
+        return fail(AQ_ERR_DTYPE, "scales/biases must be bf16 or f16 (same dtype)");
+    const int64_t V = wq->shape[0], K = out->shape[1];
+    if (K % group != 0) return fail(AQ_ERR_GROUP, "K=%lld not a multiple of group=%d", (long long)K, group);
+    if (wq->shape[1] != K * bits / 32) return fail(AQ_ERR_SHAPE, "wq must be [V, K*bits/32]");
+    if (scales->shape[0] != V || scales->shape[1] != K / group || biases->shape[0] != V ||
+        biases->shape[1] != K / group)
+        return fail(AQ_ERR_SHAPE, "scales/biases must be [V, K/group]");
+    if (numel(wq) > 0 && !aligned16(wq->data)) return fail(AQ_ERR_ALIGN, "wq data must be 16-byte aligned");
+    if (overlaps(out, wq) || overlaps(out, scales) || overlaps(out, biases))
+        return fail(AQ_ERR_OVERLAP, "out overlaps the table");
+    if (n_ids == 0 || out->shape[1] == 0) return AQ_OK;
+    if (!ids) return fail(AQ_ERR_NULL, "ids is NULL");
+    if ((st = check_device()) != AQ_OK) return st;
+    aq::QuantArgs a;
+    memset(&a, 0, sizeof a);
+    a.w = out->data;
+    a.wq = (uint32_t*)wq->data;
+    a.scales = scales->data;
+    a.biases = biases->data;
+    a.w_row = out->stride[0];
+    a.wq_row = wq->stride[0];
+    a.s_row = scales->stride[0];
+    a.b_row = biases->stride[0];
+    a.N = n_ids;
+    a.K = out->shape[1];
+    a.group = group;
+    a.bits = bits;
+    a.ids = ids;
+    a.V = wq->shape[0];
+    cudaError_t e = aq::device_error_ptr(&a.err);
+    if (e != cudaSuccess) return cuda_fail(e, "device error word");
+    e = aq::launch_dequantize(a, (aq::DT)out->dtype, (aq::DT)scales->dtype, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "row gather launch");
+    return AQ_OK;
 }

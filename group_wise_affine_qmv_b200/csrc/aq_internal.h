@@ -44,6 +44,11 @@ struct QuantArgs {
     int64_t w_row, wq_row, s_row, b_row;
     int64_t N, K;
     int group, bits;
+    // dequantize only: row t of the output is row ids[t] of W (ids on the device, V rows of W);
+    // an id outside [0, V) gives a row of zeros and sets DEVERR_INDEX in *err
+    const int64_t* ids;
+    int64_t V;
+    int* err;
 };
 cudaError_t launch_quantize(const QuantArgs& a, DT wdt, DT sdt, cudaStream_t s);
 cudaError_t launch_dequantize(const QuantArgs& a, DT wdt, DT sdt, cudaStream_t s);
@@ -98,7 +103,11 @@ bool warp_mma_supported(const MmaProblem& p);
 bool warp_mma_preferred(const MmaProblem& p);
 cudaError_t launch_warp_mma(const MmaProblem& p, cudaStream_t s);
 
-// Device-side error word (set by kernels whose bounded waits expire).
+// Device-side error word: bits set by kernels (a bounded wait expired; an index out of range).
+constexpr int DEVERR_TIMEOUT = 1;
+constexpr int DEVERR_INDEX = 2;
 cudaError_t read_and_clear_device_error(int* value, cudaStream_t s);
+// its device address on the current device
+cudaError_t device_error_ptr(int** p);
 
 }  // namespace aq

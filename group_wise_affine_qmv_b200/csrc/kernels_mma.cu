@@ -14,8 +14,9 @@
 
 namespace aq {
 
-// Set (to 1) by any tensor-core CTA whose bounded wait expired; read and cleared by
-// aq_device_error().  Kernels receive its address in their parameters.
+// Error bits set on the device (DEVERR_TIMEOUT by any tensor-core CTA whose bounded wait expired,
+// DEVERR_INDEX by a row gather given an id out of range); read and cleared by aq_device_error().
+// Kernels receive its address in their parameters.
 __device__ int g_device_error = 0;
 
 namespace {
@@ -339,6 +340,15 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
         case 8: return launch<8>(bf, pb.group, prm, grid, smem, stream);
     }
     return cudaErrorInvalidValue;
+}
+
+cudaError_t device_error_ptr(int** out) {
+    static void* cache[64] = {nullptr};
+    void* a = nullptr;
+    cudaError_t e = symbol_address(g_device_error, cache, &a);
+    if (e != cudaSuccess) return e;
+    *out = static_cast<int*>(a);
+    return cudaSuccess;
 }
 
 cudaError_t read_and_clear_device_error(int* value, cudaStream_t s) {

@@ -80,6 +80,8 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(const QuantArgs a
 }
 
 // One thread per 32-code chunk of a row: out = fma(scale, q, bias) in fp32, rounded to WT.
+// With a.ids (row gather, "Metal Kernel Bits=8 Final Report" section 3.2: dequantize_row for one
+// token id) output row n reads W row ids[n]; an id outside [0, V) writes zeros and flags it.
 template <typename WT, typename ST>
 __global__ void __launch_bounds__(256) dequantize_kernel(const QuantArgs a) {
     const int64_t chunks = a.K / 32;
@@ -88,7 +90,17 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const QuantArgs a) {
     const uint32_t mask = (1u << bits) - 1u;
     for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < total;
          t += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t n = t / chunks, c = t % chunks;
+        const int64_t row = t / chunks, c = t % chunks;
+        int64_t n = row;
+        if (a.ids) {
+            n = a.ids[row];
+            if (n < 0 || n >= a.V) {
+                WT* out = (WT*)a.w + row * a.w_row + c * 32;
+                for (int i = 0; i < 32; ++i) store_out(out + i, 0.0f);
+                if (c == 0) atomicOr(a.err, DEVERR_INDEX);
+                continue;
+            }
+        }
         const uint32_t* wp = a.wq + n * a.wq_row + c * bits;
         uint32_t w[9];
         for (int i = 0; i < bits; ++i) w[i] = __ldg(wp + i);
@@ -96,7 +108,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const QuantArgs a) {
         const int64_t g = (c * 32) / a.group;
         const float s = to_float<ST>((const ST*)a.scales + n * a.s_row + g);
         const float b = to_float<ST>((const ST*)a.biases + n * a.b_row + g);
-        WT* out = (WT*)a.w + n * a.w_row + c * 32;
+        WT* out = (WT*)a.w + row * a.w_row + c * 32;
         for (int i = 0; i < 32; ++i) {
             const int pos = i * bits;
             const int wi = pos >> 5, sh = pos & 31;

@@ -135,7 +135,7 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const Params& p, int ms) {
 
 __device__ __forceinline__ void raise_abort(const Params& p, int* abort) {
     *(volatile int*)abort = 1;
-    atomicExch(p.err, ERR_TIMEOUT);
+    atomicOr(p.err, ERR_TIMEOUT);
 }
 
 __device__ __forceinline__ int total_tiles(const Params& p, const Smem& s) {
@@ -323,7 +323,7 @@ __device__ __forceinline__ void build_xtab(const Params& p, const TileInfo& ti, 
             for (int v0 = 0; v0 < VPG; v0 += XV) {
                 uint4 buf[XV];
 #pragma unroll
-                for (int v = 0; v < XV; ++v) buf[v] = __ldg(row + v0 + v);
+                for (int v = 0; v < XV; ++v) buf[v] = __ldcg(row + v0 + v);   // x: L2, never a stale L1 line
 #pragma unroll
                 for (int v = 0; v < XV; ++v) {
                     float f[8];

@@ -165,11 +165,15 @@ __device__ __forceinline__ void load_lane_words(const uint8_t* p, uint32_t* w) {
     }
 }
 
+// Activations (x, a residual) may have been written by the previous kernel in the stream, which
+// a programmatic dependent starts next to: an L1 line of such a buffer, cached on this SM by an
+// earlier kernel, could still hold the old values.  Every global read of them goes to L2 (.cg),
+// which is coherent; only weights are read through L1.
 // element `off` of a tensor of y's dtype (fp32, or the activation dtype XT), as fp32
 template <typename XT>
 __device__ __forceinline__ float load_out(const void* r, int64_t off, int ydt) {
-    if (ydt == (int)DT::F32) return reinterpret_cast<const float*>(r)[off];
-    return half_bits_to_float(reinterpret_cast<const uint16_t*>(r)[off], XT{});
+    if (ydt == (int)DT::F32) return __ldcg(reinterpret_cast<const float*>(r) + off);
+    return half_bits_to_float(__ldcg(reinterpret_cast<const unsigned short*>(r) + off), XT{});
 }
 
 template <typename XT>
@@ -353,7 +357,7 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
                                                                       (int64_t)(cg0 + gl) * G);
             uint4 v[G / 8];
 #pragma unroll
-            for (int u = 0; u < G / 8; ++u) v[u] = src[u];
+            for (int u = 0; u < G / 8; ++u) v[u] = p.xsm ? src[u] : __ldcg(src + u);
             float sum = 0.0f;
 #pragma unroll
             for (int u = 0; u < G / 8; ++u) {
@@ -425,7 +429,10 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
         for (int t = 0; t < NTL; ++t) {
             uint4 xv[XV];
 #pragma unroll
-            for (int v = 0; v < XV; ++v) xv[v] = reinterpret_cast<const uint4*>(xrow[t] + kx2)[v];
+            for (int v = 0; v < XV; ++v) {
+                const uint4* xp4 = reinterpret_cast<const uint4*>(xrow[t] + kx2) + v;
+                xv[v] = p.xsm ? *xp4 : __ldcg(xp4);
+            }
             const uint32_t* xw = reinterpret_cast<const uint32_t*>(xv);
 #pragma unroll
             for (int s = 0; s < STEPS; ++s)

@@ -156,6 +156,28 @@ def linear4d_case(seed: int = 4):
 
 
 # ---------------------------------------------------------------------------
+# quantized embedding table ("Metal Kernel Bits=8 Final Report", section 4.1)
+# ---------------------------------------------------------------------------
+
+EMBED_ROWS = 262144
+EMBED_WORDS = 352          # uint32 words per row: K = 352 * 32 / bits
+EMBED_GROUPS = 44          # scales per row: G = K / 44 (32 at 8 bits, 64 at 4 bits)
+
+
+def embedding_table(bits: int, rows: int = EMBED_ROWS, sdtype=torch.bfloat16, seed: int = 0, device: str = "cpu"):
+    """A packed table of random codes (uniform random uint32 words) with random scales
+    (|N(0, 0.01)|) and biases (N(0, 0.05)) in the half dtype: (wq int32 [rows, 352],
+    scales [rows, 44], biases [rows, 44], K, group)."""
+    g = gen(seed, device)
+    wq = torch.randint(-2 ** 31, 2 ** 31, (rows, EMBED_WORDS), generator=g, dtype=torch.int64,
+                       device=device).to(torch.int32)
+    sc = torch.randn(rows, EMBED_GROUPS, generator=g, device=device).abs_().mul_(0.01).to(sdtype)
+    bi = torch.randn(rows, EMBED_GROUPS, generator=g, device=device).mul_(0.05).to(sdtype)
+    K = EMBED_WORDS * 32 // bits
+    return wq, sc, bi, K, K // EMBED_GROUPS
+
+
+# ---------------------------------------------------------------------------
 # prefill and the expert bank
 # ---------------------------------------------------------------------------
 

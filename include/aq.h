@@ -62,7 +62,8 @@ typedef enum aq_status {
     AQ_ERR_OVERLAP = 10,     /* the output overlaps an input or itself               */
     AQ_ERR_CUDA = 11,        /* a CUDA runtime/driver call or a launch failed        */
     AQ_ERR_DEVICE = 12,      /* current device is not an sm_100 (B200-class) GPU     */
-    AQ_ERR_TIMEOUT = 13      /* a kernel's bounded pipeline wait expired (device)    */
+    AQ_ERR_TIMEOUT = 13,     /* a kernel's bounded pipeline wait expired (device)    */
+    AQ_ERR_INDEX = 14        /* a row id on the device was out of range (device)     */
 } aq_status;
 
 typedef enum aq_dtype {
@@ -108,6 +109,24 @@ aq_status aq_quantize(const aq_view* w, int group, int bits, const aq_view* wq,
  */
 aq_status aq_dequantize(const aq_view* wq, const aq_view* scales, const aq_view* biases,
                         int group, int bits, const aq_view* w_out, void* stream);
+
+/*
+ * aq_dequantize_rows -- embedding lookup on a quantized table, one row per id:
+ *     out[t, k] = scale[ids[t], k/G] * q[ids[t], k] + bias[ids[t], k/G],   t < n_ids
+ *   evaluated in fp32 and rounded once to out's dtype (the values aq_dequantize gives).
+ *   ("Metal Kernel Bits=8 Final Report", sections 3.1-3.2 and 5.1: dequantize_row and
+ *   dequantize_row_8bit turn the row of one token id into activations, called from
+ *   dequantizeRow(weight:tokenId:output:); its embedding table is [262144, 352] uint32,
+ *   scales [262144, 44].)
+ * wq [V, K*bits/32] AQ_U32; scales/biases [V, K/group] AQ_BF16|AQ_F16 (rank 2).
+ * ids: DEVICE pointer to n_ids int64 row ids (not readable on the host).  An id outside
+ *   [0, V) gives a row of zeros and sets a device error that aq_device_error() returns as
+ *   AQ_ERR_INDEX.
+ * out [n_ids, K] AQ_F32, AQ_BF16 or AQ_F16, must not overlap the table.
+ */
+aq_status aq_dequantize_rows(const aq_view* wq, const aq_view* scales, const aq_view* biases,
+                             int group, int bits, const int64_t* ids, int64_t n_ids,
+                             const aq_view* out, void* stream);
 
 /*
  * aq_qmm_t -- y = x . dequant(W)^T for any number of rows.
@@ -274,7 +293,8 @@ const char* aq_last_error_message(void);
 /*
  * Reads and clears the device-side error word of the current device after
  * synchronizing `stream`.  Returns AQ_OK if no kernel recorded an error,
- * AQ_ERR_TIMEOUT if a bounded wait expired, AQ_ERR_CUDA if the read failed.
+ * AQ_ERR_TIMEOUT if a bounded wait expired, AQ_ERR_INDEX if a row gather met an
+ * id outside its table, AQ_ERR_CUDA if the read failed.
  */
 aq_status aq_device_error(void* stream);
 
