@@ -50,7 +50,7 @@ class AqPlan(ctypes.Structure):
                 ("y_row_stride", ctypes.c_int64), ("total_rows", ctypes.c_int64)]
 
 
-EXPORTED = ("aq_quantize", "aq_dequantize", "aq_dequantize_rows", "aq_qmv", "aq_qmm_t", "aq_qmm_t_grouped", "aq_qmm_t_multi",
+EXPORTED = ("aq_quantize", "aq_dequantize", "aq_dequantize_rows", "aq_qmv", "aq_qmm_t", "aq_qmm_t_grouped", "aq_qmv_gathered", "aq_qmm_t_multi",
             "aq_qmm_t_swiglu", "aq_qmm_t_residual", "aq_plan_linear", "aq_status_string", "aq_last_error_message",
             "aq_device_error", "aq_version")
 
@@ -81,6 +81,8 @@ def load_library(path: str = LIB_PATH):
         lib.aq_dequantize_rows.restype = ci
         lib.aq_qmm_t_grouped.argtypes = [V, vp, ci, V, V, V, ci, ci, V, vp]
         lib.aq_qmm_t_grouped.restype = ci
+        lib.aq_qmv_gathered.argtypes = [V, vp, vp, ctypes.c_int64, V, V, V, ci, ci, V, vp]
+        lib.aq_qmv_gathered.restype = ci
         VA = ctypes.POINTER(V)
         lib.aq_qmm_t_multi.argtypes = [V, ci, VA, VA, VA, ci, ci, VA, vp]
         lib.aq_qmm_t_multi.restype = ci
@@ -247,6 +249,24 @@ def aq_qmm_t_residual(x, wq, scales, biases, group: int, bits: int, r, out=None)
     with torch.cuda.device(x.device):
         _check(lib, lib.aq_qmm_t_residual(view(x), view(wq), view(scales), view(biases), group, bits, view(r),
                                           view(out), _stream(x)))
+    return out
+
+
+def aq_qmv_gathered(x, x_ids, w_ids, wq_bank, s_bank, b_bank, group: int, bits: int, out=None, out_dtype=None):
+    """y[i] = x[x_ids[i]] . dequant(W[w_ids[i]])^T (ids: contiguous 1D int64 CUDA tensors)."""
+    lib = load_library()
+    for ids in (x_ids, w_ids):
+        if ids.dtype != torch.int64 or not ids.is_cuda or ids.dim() != 1 or not ids.is_contiguous():
+            raise TypeError("ids must be contiguous 1D int64 CUDA tensors")
+    if x_ids.numel() != w_ids.numel():
+        raise ValueError("x_ids and w_ids must have the same length")
+    R = x_ids.numel()
+    if out is None:
+        out = torch.empty((R, wq_bank.shape[1]), dtype=out_dtype or x.dtype, device=x.device)
+    with torch.cuda.device(x.device):
+        _check(lib, lib.aq_qmv_gathered(view(x), ctypes.c_void_p(x_ids.data_ptr()), ctypes.c_void_p(w_ids.data_ptr()),
+                                        R, view(wq_bank), view(s_bank), view(b_bank), group, bits, view(out),
+                                        _stream(x)))
     return out
 
 

@@ -810,3 +810,73 @@ AQ_API aq_status aq_dequantize_rows(const aq_view* wq, const aq_view* scales, co
     if (e != cudaSuccess) return cuda_fail(e, "row gather launch");
     return AQ_OK;
 }
+
+AQ_API aq_status aq_qmv_gathered(const aq_view* x, const int64_t* x_ids, const int64_t* w_ids, int64_t n_rows,
+                                 const aq_view* wq_bank, const aq_view* s_bank, const aq_view* b_bank, int group,
+                                 int bits, const aq_view* y, void* stream) {
+    g_msg[0] = 0;
+    aq_status st;
+    if ((st = check_view(x, "x", 2, 2)) != AQ_OK) return st;
+    if ((st = check_view(wq_bank, "wq_bank", 3, 3)) != AQ_OK) return st;
+    if ((st = check_view(s_bank, "s_bank", 3, 3)) != AQ_OK) return st;
+    if ((st = check_view(b_bank, "b_bank", 3, 3)) != AQ_OK) return st;
+    if ((st = check_view(y, "y", 2, 2)) != AQ_OK) return st;
+    if ((st = check_output(y, "y")) != AQ_OK) return st;
+    if ((st = check_bits_group(bits, group)) != AQ_OK) return st;
+    if (!is_half(x->dtype)) return fail(AQ_ERR_DTYPE, "x must be bf16 or f16");
+    if (wq_bank->dtype != AQ_U32) return fail(AQ_ERR_DTYPE, "wq_bank must be u32");
+    if (s_bank->dtype != x->dtype || b_bank->dtype != x->dtype)
+        return fail(AQ_ERR_DTYPE, "scale/bias banks must have x's dtype");
+    if (y->dtype != x->dtype && y->dtype != AQ_F32) return fail(AQ_ERR_DTYPE, "y must have x's dtype or f32");
+    const int64_t T = x->shape[0], K = x->shape[1], E = wq_bank->shape[0], N = wq_bank->shape[1];
+    if (n_rows < 0) return fail(AQ_ERR_SHAPE, "n_rows < 0");
+    if (K % group != 0) return fail(AQ_ERR_GROUP, "K not a multiple of group");
+    if (wq_bank->shape[2] != K * bits / 32) return fail(AQ_ERR_SHAPE, "wq_bank last dim must be K*bits/32");
+    if (s_bank->shape[0] != E || b_bank->shape[0] != E || s_bank->shape[1] != N || b_bank->shape[1] != N ||
+        s_bank->shape[2] != K / group || b_bank->shape[2] != K / group)
+        return fail(AQ_ERR_SHAPE, "scale/bias banks must be [E, N, K/group]");
+    if (y->shape[0] != n_rows || y->shape[1] != N) return fail(AQ_ERR_SHAPE, "y must be [n_rows, N]");
+    if (numel(wq_bank) > 0) {
+        const int64_t need = (bits == 4 || bits == 8) ? 4 : (bits == 2 || bits == 6) ? 2 : 1;  // words
+        if (!aligned16(wq_bank->data) || wq_bank->stride[0] % need != 0 || (N > 1 && wq_bank->stride[1] % need != 0))
+            return fail(AQ_ERR_ALIGN, "wq_bank rows must be %lld-byte aligned", (long long)(need * 4));
+    }
+    if (overlaps(y, x) || overlaps(y, wq_bank) || overlaps(y, s_bank) || overlaps(y, b_bank))
+        return fail(AQ_ERR_OVERLAP, "y overlaps an input");
+    if (n_rows == 0 || N == 0) return AQ_OK;
+    if (!x_ids || !w_ids) return fail(AQ_ERR_NULL, "x_ids / w_ids is NULL");
+    if (n_rows > 65535) return fail(AQ_ERR_UNSUPPORTED, "more than 65535 gathered rows per call");
+    if ((st = check_device()) != AQ_OK) return st;
+    aq::QmvArgs a;
+    memset(&a, 0, sizeof a);
+    a.x = x->data;
+    a.wq = (const uint32_t*)wq_bank->data;
+    a.scales = s_bank->data;
+    a.biases = b_bank->data;
+    a.y = y->data;
+    a.x_row = x->stride[0];
+    a.y_row = y->stride[0];
+    a.w_row = wq_bank->stride[1];
+    a.s_row = s_bank->stride[1];
+    a.b_row = b_bank->stride[1];
+    a.M = 1;
+    a.N = N;
+    a.K = K;
+    a.log2g = log2i(group);
+    a.xvec = (aligned16(x->data) && (T <= 1 || x->stride[0] % 8 == 0)) ? 1 : 0;
+    a.bshape1 = 1;
+    a.xb[0] = x->stride[0];
+    a.yb[0] = y->stride[0];
+    a.wb[0] = wq_bank->stride[0];
+    a.sb[0] = s_bank->stride[0];
+    a.bb[0] = b_bank->stride[0];
+    a.x_ids = x_ids;
+    a.w_ids = w_ids;
+    a.x_rows = T;
+    a.w_entries = E;
+    cudaError_t e = aq::device_error_ptr(&a.err);
+    if (e != cudaSuccess) return cuda_fail(e, "device error word");
+    e = aq::launch_qmv(a, bits, (aq::DT)x->dtype, (aq::DT)y->dtype, n_rows, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gathered GEMV launch");
+    return AQ_OK;
+}

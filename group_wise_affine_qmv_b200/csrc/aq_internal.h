@@ -28,6 +28,14 @@ struct QmvArgs {
     int xvec;                      // 1: x rows 16-byte aligned (vector loads allowed)
     int64_t bshape1;               // size of the inner launch-batch dim (1 if none)
     int64_t xb[2], yb[2], wb[2], sb[2], bb[2];  // launch-batch strides (outer, inner)
+    // gathered rows (x_ids != nullptr): launch batch i is row i of y, computed from x row x_ids[i]
+    // and W bank entry w_ids[i] (xb[0] / wb[0] / sb[0] / bb[0] are the per-row / per-entry strides,
+    // yb[0] the row stride of y); ids outside [0, x_rows) / [0, w_entries) give a row of zeros
+    // and set DEVERR_INDEX in *err
+    const int64_t* x_ids;
+    const int64_t* w_ids;
+    int64_t x_rows, w_entries;
+    int* err;
 };
 
 // Launches the GEMV kernel for `nbatch` launch batches.  Returns cudaSuccess or the launch error.

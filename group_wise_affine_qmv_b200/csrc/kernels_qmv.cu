@@ -115,13 +115,30 @@ __global__ void __launch_bounds__(QMV_THREADS) qmv_kernel(const __grid_constant_
     const int64_t n0 = ((int64_t)blockIdx.x * QMV_WARPS + warp) * RPW;
     if (n0 >= a.N) return;
     const int64_t bidx = blockIdx.y;
-    const int64_t b1 = bidx % a.bshape1, b0 = bidx / a.bshape1;
+    int64_t b1 = bidx % a.bshape1, b0 = bidx / a.bshape1;
+    int64_t xo = b0 * a.xb[0] + b1 * a.xb[1], wo = b0 * a.wb[0] + b1 * a.wb[1];
+    int64_t so = b0 * a.sb[0] + b1 * a.sb[1], bo = b0 * a.bb[0] + b1 * a.bb[1];
+    if (a.x_ids) {
+        // gathered row bidx: x row and W bank entry from the device id arrays (read once per warp)
+        const int64_t xi = a.x_ids[bidx], wi = a.w_ids[bidx];
+        if (xi < 0 || xi >= a.x_rows || wi < 0 || wi >= a.w_entries) {
+            if (lane < RPW && n0 + lane < a.N) store_out((YT*)a.y + bidx * a.yb[0] + n0 + lane, 0.0f);
+            if (lane == 0 && n0 == 0) atomicOr(a.err, DEVERR_INDEX);
+            return;
+        }
+        xo = xi * a.xb[0];
+        wo = wi * a.wb[0];
+        so = wi * a.sb[0];
+        bo = wi * a.bb[0];
+        b0 = bidx;
+        b1 = 0;
+    }
 
-    const XT* xbase = (const XT*)a.x + b0 * a.xb[0] + b1 * a.xb[1];
+    const XT* xbase = (const XT*)a.x + xo;
     YT* ybase = (YT*)a.y + b0 * a.yb[0] + b1 * a.yb[1];
-    const uint32_t* wbase = a.wq + b0 * a.wb[0] + b1 * a.wb[1];
-    const XT* sbase = (const XT*)a.scales + b0 * a.sb[0] + b1 * a.sb[1];
-    const XT* bbase = (const XT*)a.biases + b0 * a.bb[0] + b1 * a.bb[1];
+    const uint32_t* wbase = a.wq + wo;
+    const XT* sbase = (const XT*)a.scales + so;
+    const XT* bbase = (const XT*)a.biases + bo;
 
     int64_t nrow[RPW];
 #pragma unroll

@@ -41,8 +41,24 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
+// Suspend-time hint of every try_wait, in ns (0: none, the hardware's own time limit).  A thread
+// suspended in try_wait resumes as soon as the phase completes, so the hint only decides how
+// often a waiting warp comes back to re-test (and to take an issue slot from the working warps).
+#ifndef AQ_MBAR_SUSPEND_NS
+#define AQ_MBAR_SUSPEND_NS 0
+#endif
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
     uint32_t ok;
+#if AQ_MBAR_SUSPEND_NS > 0
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity), "n"(AQ_MBAR_SUSPEND_NS)
+        : "memory");
+#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -50,6 +66,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
         : "=r"(ok)
         : "r"(bar_addr), "r"(parity)
         : "memory");
+#endif
     return ok != 0;
 }
 
@@ -77,9 +94,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (!done) {
         const long long c0 = clock64();
         const long long limit = (long long)(budget_ns * 2ull);
+        constexpr uint32_t CHECK = AQ_MBAR_SUSPEND_NS > 0 ? 0u : 63u;   // re-test budget/abort every Nth try
         for (uint32_t i = 1;; ++i) {
             if (mbar_try_wait(a, parity)) { done = true; break; }
-            if ((i & 63u) == 0 && (*abort || clock64() - c0 > limit)) break;
+            if ((i & CHECK) == 0 && (*abort || clock64() - c0 > limit)) break;
         }
     }
     return done;

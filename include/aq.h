@@ -190,6 +190,23 @@ aq_status aq_qmm_t_grouped(const aq_view* x_sorted, const int64_t* offsets, int 
                            const aq_view* wq_bank, const aq_view* s_bank, const aq_view* b_bank,
                            int group, int bits, const aq_view* y_sorted, void* stream);
 
+/*
+ * aq_qmv_gathered -- mixture-of-experts rows without a host-side sort (the "gathered QMV" that
+ * "mlx PR #4516" names next to its affine qmv kernels): for i < n_rows,
+ *     y[i] = x[x_ids[i]] . dequant(W_{w_ids[i]})^T
+ * so a decode step can route each token to its experts straight from the router's output.
+ * x [T, K] AQ_BF16|AQ_F16 (row stride free); wq_bank [E, N, K*bits/32] AQ_U32; s_bank,
+ * b_bank [E, N, K/group] in x's dtype (any row/entry strides that keep W rows aligned as for
+ * aq_qmm_t); x_ids, w_ids: DEVICE pointers to n_rows int64 ids (n_rows <= 65535);
+ * y [n_rows, N], x's dtype or AQ_F32.  Runs the CUDA-core GEMV, one row per id pair (each row
+ * streams its expert's weights: meant for decode, where rows are few).  An id outside
+ * [0, T) or [0, E) gives a row of zeros and a device error that aq_device_error() returns
+ * as AQ_ERR_INDEX.
+ */
+aq_status aq_qmv_gathered(const aq_view* x, const int64_t* x_ids, const int64_t* w_ids, int64_t n_rows,
+                          const aq_view* wq_bank, const aq_view* s_bank, const aq_view* b_bank,
+                          int group, int bits, const aq_view* y, void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* Fused calls of a decoder layer's decode step (warp-level kernel).       */
 /*                                                                        */

@@ -34,11 +34,6 @@ def _q(w, group, bits, sdtype="bf16"):
     return Q, to_device_quant(Q, DEV, tdt)
 
 
-def _kernel(x, wq, sc, bi, group, bits):
-    y = torch.empty(tuple(x.shape[:-1]) + (wq.shape[-2],), dtype=x.dtype, device=x.device)
-    return aq.aq_plan_linear(x, wq, sc, bi, group, bits, y)["kernel"]
-
-
 @pytest.mark.parametrize("bits", [2, 4, 8])
 @pytest.mark.parametrize("M,Ns,K", [(1, (100, 37, 64), 512), (5, (100, 37, 64), 512), (8, (2048, 1024, 1024), 1024),
                                     (32, (2048, 1024, 1024), 1024), (32, (33, 1, 300), 256), (16, (4099, 7), 4096)])
@@ -149,67 +144,121 @@ def _bf16_round(v: np.ndarray) -> np.ndarray:
     return oracle.half_to_double(bits, "bf16")
 
 
-@pytest.mark.parametrize("bits", [4, 8])
-def test_decode_chain_graph(bits):
-    layers, B, group, vocab = 3, inputs.DECODE_BATCH, inputs.DECODE_GROUP, 4096
+def _chain_setup(layers, bits, vocab, seed0=1000, logits_dtype=torch.bfloat16):
+    B, group = inputs.DECODE_BATCH, inputs.DECODE_GROUP
     proj = {name: (K, N) for name, K, N in inputs.DECODE_PROJ}
-    Q = {}
-    W = {}
+    Q, W = {}, {}
     for l in range(layers):
         for i, name in enumerate(("q", "k", "v", "o", "gate", "up", "down")):
             K, N = proj[name]
-            Q[l, name], W[l, name] = _q(inputs.decode_w(K, N, seed=1000 * l + i), group, bits)
+            Q[l, name], W[l, name] = _q(inputs.decode_w(K, N, seed=seed0 * (l + 1) + i), group, bits)
     Q["lm"], W["lm"] = _q(inputs.decode_w(1024, vocab, seed=5), group, bits)
     h0 = inputs.decode_x(1024, seed=11)
-    h0d = h0.to(DEV)
-    h = torch.empty_like(h0d)
-    q = torch.empty(B, 1, 2048, dtype=torch.bfloat16, device=DEV)
-    k = torch.empty(B, 1, 1024, dtype=torch.bfloat16, device=DEV)
-    v = torch.empty_like(k)
-    a = torch.empty(B, 1, 3072, dtype=torch.bfloat16, device=DEV)
-    logits = torch.empty(B, 1, vocab, dtype=torch.bfloat16, device=DEV)
+    bufs = {"h0": h0.to(DEV), "h": torch.empty(B, 1, 1024, dtype=torch.bfloat16, device=DEV),
+            "q": torch.empty(B, 1, 2048, dtype=torch.bfloat16, device=DEV),
+            "k": torch.empty(B, 1, 1024, dtype=torch.bfloat16, device=DEV),
+            "v": torch.empty(B, 1, 1024, dtype=torch.bfloat16, device=DEV),
+            "a": torch.empty(B, 1, 3072, dtype=torch.bfloat16, device=DEV),
+            "logits": torch.empty(B, 1, vocab, dtype=logits_dtype, device=DEV)}
+    return Q, W, h0, bufs
 
-    def step():
-        for l in range(layers):
-            aq.aq_qmm_t_multi(h0d if l == 0 else h, [W[l, "q"], W[l, "k"], W[l, "v"]], group, bits, outs=[q, k, v])
-            aq.aq_qmm_t_residual(v, *W[l, "o"], group, bits, r=h0d if l == 0 else h, out=h)
-            aq.aq_qmm_t_swiglu(h, W[l, "gate"], W[l, "up"], group, bits, out=a)
-            aq.aq_qmm_t_residual(a, *W[l, "down"], group, bits, r=h, out=h)
-        aq.aq_qmm_t(h, *W["lm"], group, bits, out=logits)
 
+def _chain_calls(W, bufs, layers, bits):
+    """The launches of the chain, in order, as closures (q, k, v = multi(h); h += o(v);
+    a = swiglu(h); h += down(a); ...; logits = lm_head(h))."""
+    group = inputs.DECODE_GROUP
+    b = bufs
+    calls = []
+    for l in range(layers):
+        src = b["h0"] if l == 0 else b["h"]
+        calls.append(lambda l=l, src=src: aq.aq_qmm_t_multi(src, [W[l, "q"], W[l, "k"], W[l, "v"]], group, bits,
+                                                            outs=[b["q"], b["k"], b["v"]]))
+        calls.append(lambda l=l, src=src: aq.aq_qmm_t_residual(b["v"], *W[l, "o"], group, bits, r=src, out=b["h"]))
+        calls.append(lambda l=l: aq.aq_qmm_t_swiglu(b["h"], W[l, "gate"], W[l, "up"], group, bits, out=b["a"]))
+        calls.append(lambda l=l: aq.aq_qmm_t_residual(b["a"], *W[l, "down"], group, bits, r=b["h"], out=b["h"]))
+    calls.append(lambda: aq.aq_qmm_t(b["h"], *W["lm"], group, bits, out=b["logits"]))
+    return calls
+
+
+def _graph_replays(calls, bufs, n=3):
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
-        step()
+        for c in calls:
+            c()
     torch.cuda.synchronize()
-    eager = logits.clone()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
-        step()
-    results = []
-    for _ in range(3):
-        logits.zero_()
-        h.zero_()
+        for c in calls:
+            c()
+    out = []
+    for _ in range(n):
+        for k in ("h", "logits", "a", "v"):
+            bufs[k].zero_()
         g.replay()
         torch.cuda.synchronize()
-        results.append(logits.clone())
+        out.append((bufs["logits"].clone(), bufs["h"].clone()))
     aq.aq_device_error()
     del g
-    for r_ in results:
-        assert torch.equal(r_, eager)
+    return out
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_decode_chain_graph_matches_oracle(bits):
+    """One chained decoder layer (four dependent launches) and lm_head, in one CUDA graph,
+    against the oracle's own chain; logits in fp32.
+
+    Why one layer: every stored activation is rounded to bf16 on both sides, and where the GPU's
+    fp32 sums and the oracle's fp64 sums fall on either side of a rounding boundary the two
+    chains carry values one bf16 step apart; each such step spreads through the next dense layer
+    and flips more roundings.  Simulated on the CPU (fp32 sums in shuffled orders against fp64
+    sums, these weights) the fp32 logits' per-row error is 1.6e-3 after one layer, 2.9-3.5e-3
+    after two and 5.0-5.5e-3 after three (1.6-34 % of the hidden state a step apart): past the
+    single-matmul bar from three layers on, at it from two.  Longer chains are checked for
+    ordering, bit for bit, below.
+    """
+    layers, vocab = 1, 4096
+    B = inputs.DECODE_BATCH
+    Q, W, h0, bufs = _chain_setup(layers, bits, vocab, logits_dtype=torch.float32)
+    results = _graph_replays(_chain_calls(W, bufs, layers, bits), bufs)
+    for r_ in results[1:]:
+        assert torch.equal(r_[0], results[0][0]) and torch.equal(r_[1], results[0][1])
 
     # the oracle's chain: fp64 contractions, every stored activation rounded to bf16 as the GPU does
-    def _bf16_round_lin(xv, Qk):
+    def lin(xv, Qk):
         xb = half_bits(torch.from_numpy(xv.astype(np.float32)).to(torch.bfloat16)).reshape(B, -1)
         return oracle.linear_contig(xb, "bf16", Qk.dequant())
 
     hv = h0.reshape(B, 1024).double().numpy()
     for l in range(layers):
-        vv = _bf16_round(_bf16_round_lin(hv, Q[l, "v"]))
-        hv = _bf16_round(hv + _bf16_round_lin(vv, Q[l, "o"]))
-        av = _bf16_round(oracle.swiglu(_bf16_round_lin(hv, Q[l, "gate"]), _bf16_round_lin(hv, Q[l, "up"])))
-        hv = _bf16_round(hv + _bf16_round_lin(av, Q[l, "down"]))
-    ref = _bf16_round_lin(hv, Q["lm"])
-    err = row_errors(results[-1], ref)
+        vv = _bf16_round(lin(hv, Q[l, "v"]))
+        hv = _bf16_round(hv + lin(vv, Q[l, "o"]))
+        av = _bf16_round(oracle.swiglu(lin(hv, Q[l, "gate"]), lin(hv, Q[l, "up"])))
+        hv = _bf16_round(hv + lin(av, Q[l, "down"]))
+    ref = lin(hv, Q["lm"])
+    logits, h_out = results[-1]
+    err = row_errors(logits, ref)
     assert err.size == B and np.all(err <= 4e-3), (err.max(), int(err.argmax()))
-    # and the residual stream after the last layer
-    assert np.all(row_errors(h, hv) <= 4e-3)
+    # the residual stream: every element within two bf16 steps of the oracle's value (one where the
+    # first residual's two sums straddled a rounding boundary, one more where the second did)
+    got = h_out.reshape(B, 1024).double().cpu().numpy()
+    step = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(hv), 2.0 ** -126))) - 7)
+    assert np.all(np.abs(got - hv) <= 2 * step * (1 + 1e-9))
+    assert np.mean(got != hv) < 0.05
+
+
+def test_decode_chain_ordering_bitwise():
+    """The full 28-layer chain (112 launches + lm_head), replayed from a CUDA graph in which every
+    launch is a programmatic dependent of the one before, gives exactly the bits of the same calls
+    run one at a time with the device drained after each: no kernel read an activation before the
+    kernel that writes it had finished, and none wrote one that an earlier kernel still read."""
+    layers, bits, vocab = inputs.DECODE_LAYERS, 4, 2048
+    _, W, _, bufs = _chain_setup(layers, bits, vocab, seed0=7)
+    calls = _chain_calls(W, bufs, layers, bits)
+    results = _graph_replays(calls, bufs, n=2)
+    for k in ("h", "logits", "a", "v"):
+        bufs[k].zero_()
+    for c in calls:
+        c()
+        torch.cuda.synchronize()
+    assert torch.equal(bufs["logits"], results[0][0]) and torch.equal(bufs["h"], results[0][1])
+    assert torch.equal(results[1][0], results[0][0])
