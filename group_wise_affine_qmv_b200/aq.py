@@ -52,7 +52,7 @@ class AqPlan(ctypes.Structure):
 
 EXPORTED = ("aq_quantize", "aq_dequantize", "aq_dequantize_rows", "aq_qmv", "aq_qmm_t", "aq_qmm_t_grouped", "aq_qmv_gathered", "aq_qmm_t_multi",
             "aq_qmm_t_swiglu", "aq_qmm_t_residual", "aq_plan_linear", "aq_status_string", "aq_last_error_message",
-            "aq_device_error", "aq_version")
+            "aq_device_error", "aq_check_bounded_wait", "aq_version")
 
 _lib = None
 _lock = threading.Lock()
@@ -98,6 +98,8 @@ def load_library(path: str = LIB_PATH):
         lib.aq_last_error_message.restype = ctypes.c_char_p
         lib.aq_device_error.argtypes = [vp]
         lib.aq_device_error.restype = ci
+        lib.aq_check_bounded_wait.argtypes = [ctypes.c_uint64, vp]
+        lib.aq_check_bounded_wait.restype = ci
         lib.aq_version.argtypes = []
         lib.aq_version.restype = ci
         _lib = lib
@@ -291,6 +293,15 @@ def aq_device_error(device=None):
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
     with torch.cuda.device(dev):
         _check(lib, lib.aq_device_error(torch.cuda.current_stream(dev).cuda_stream))
+
+
+def aq_check_bounded_wait(budget_ns: int, device=None):
+    """Enqueue the bounded-wait self-check (a wait on a barrier nothing completes, given up after
+    budget_ns); the next aq_device_error() then raises AQ_ERR_TIMEOUT."""
+    lib = load_library()
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        _check(lib, lib.aq_check_bounded_wait(int(budget_ns), torch.cuda.current_stream(dev).cuda_stream))
 
 
 def aq_version() -> int:

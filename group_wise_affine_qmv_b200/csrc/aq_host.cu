@@ -880,3 +880,13 @@ AQ_API aq_status aq_qmv_gathered(const aq_view* x, const int64_t* x_ids, const i
     if (e != cudaSuccess) return cuda_fail(e, "gathered GEMV launch");
     return AQ_OK;
 }
+
+AQ_API aq_status aq_check_bounded_wait(uint64_t budget_ns, void* stream) {
+    g_msg[0] = 0;
+    if (budget_ns == 0 || budget_ns > 1000000000ull) return fail(AQ_ERR_SHAPE, "budget_ns must be in (0, 1e9]");
+    aq_status st = check_device();
+    if (st != AQ_OK) return st;
+    cudaError_t e = aq::launch_bounded_wait_check(budget_ns, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "bounded-wait check launch");
+    return AQ_OK;
+}

@@ -117,5 +117,7 @@ constexpr int DEVERR_INDEX = 2;
 cudaError_t read_and_clear_device_error(int* value, cudaStream_t s);
 // its device address on the current device
 cudaError_t device_error_ptr(int** p);
+// one warp's bounded wait on a barrier nothing completes (budget in ns)
+cudaError_t launch_bounded_wait_check(uint64_t budget_ns, cudaStream_t s);
 
 }  // namespace aq

@@ -342,6 +342,30 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     return cudaErrorInvalidValue;
 }
 
+// Check of the bounded waits every pipeline kernel uses: one warp waits, with the same bounded
+// wait, on an mbarrier that nothing arrives on (no copy or MMA is tied to it), for `budget_ns`,
+// and records DEVERR_TIMEOUT as a pipeline kernel whose wait expired does.
+__global__ void __launch_bounds__(32) bounded_wait_check_kernel(int* err, uint64_t budget_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&bar, 1);
+        abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    __syncwarp();
+    const bool done = ptx::mbar_wait(&bar, 0, &abort_flag, budget_ns);
+    if (!done && threadIdx.x == 0) atomicOr(err, DEVERR_TIMEOUT);
+}
+
+cudaError_t launch_bounded_wait_check(uint64_t budget_ns, cudaStream_t s) {
+    int* err = nullptr;
+    cudaError_t e = device_error_ptr(&err);
+    if (e != cudaSuccess) return e;
+    bounded_wait_check_kernel<<<1, 32, 0, s>>>(err, budget_ns);
+    return cudaGetLastError();
+}
+
 cudaError_t device_error_ptr(int** out) {
     static void* cache[64] = {nullptr};
     void* a = nullptr;

@@ -315,6 +315,16 @@ const char* aq_last_error_message(void);
  */
 aq_status aq_device_error(void* stream);
 
+/*
+ * aq_check_bounded_wait -- exercises the bounded wait of the pipeline kernels without any
+ * fault: one warp waits, with the same bounded wait, on a barrier that nothing completes, gives
+ * up after budget_ns (0 < budget_ns <= 1e9) and records the timeout in the device error word,
+ * so that the next aq_device_error() returns AQ_ERR_TIMEOUT and clears it.  Nothing is in flight
+ * when it gives up: the context stays usable.  (No counterpart on the pages: a self-check of
+ * this library's failure reporting.)
+ */
+aq_status aq_check_bounded_wait(uint64_t budget_ns, void* stream);
+
 /* Library version: major*10000 + minor*100 + patch. */
 int aq_version(void);
 

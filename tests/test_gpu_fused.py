@@ -238,11 +238,15 @@ def test_decode_chain_graph_matches_oracle(bits):
     logits, h_out = results[-1]
     err = row_errors(logits, ref)
     assert err.size == B and np.all(err <= 4e-3), (err.max(), int(err.argmax()))
-    # the residual stream: every element within two bf16 steps of the oracle's value (one where the
-    # first residual's two sums straddled a rounding boundary, one more where the second did)
+    # the residual stream, element by element: within two bf16 steps of the oracle's value (one
+    # where the first residual's sums straddled a rounding boundary, one more where the second
+    # did) plus one bf16 step of the row's largest value (an input element one step apart moves a
+    # small output by an amount set by the inputs' scale, not by its own; a CPU simulation with
+    # shuffled fp32 sums used up to 0.8 of half that); and most elements equal
     got = h_out.reshape(B, 1024).double().cpu().numpy()
     step = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(hv), 2.0 ** -126))) - 7)
-    assert np.all(np.abs(got - hv) <= 2 * step * (1 + 1e-9))
+    row_scale = np.abs(hv).max(-1, keepdims=True)
+    assert np.all(np.abs(got - hv) <= 2 * step + 2.0 ** -8 * row_scale)
     assert np.mean(got != hv) < 0.05
 
 

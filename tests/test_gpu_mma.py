@@ -210,3 +210,22 @@ def test_odd_group_count_takes_gemv():
 
 def test_device_error_word_clear():
     aq.aq_device_error()
+
+
+def test_bounded_wait_reports_timeout():
+    """A bounded wait that runs out (on a barrier nothing completes, 2 ms budget) is reported as
+    AQ_ERR_TIMEOUT by aq_device_error, which clears it; the device stays usable and the next
+    call is correct with a clean error word."""
+    aq.aq_device_error()
+    aq.aq_check_bounded_wait(2_000_000)
+    with pytest.raises(aq.AQError) as ei:
+        aq.aq_device_error()
+    assert ei.value.name == "AQ_ERR_TIMEOUT"
+    aq.aq_device_error()
+    M, N, K, group, bits = 40, 300, 512, 64, 4
+    w = inputs.normal((N, K), 0.02, seed=81)
+    Q, (wq, sc, bi) = _q(w, group, bits)
+    x = inputs.normal((M, K), 1.0, torch.bfloat16, seed=82)
+    y = aq.aq_qmm_t(x.to(DEV), wq, sc, bi, group, bits)
+    aq.aq_device_error()
+    assert np.all(row_errors(y, oracle_linear_view(x, Q.dequant())) <= 4e-3)
