@@ -72,6 +72,7 @@ def sweep_bytes(layers):
 
 
 PROJ = {name: (K, N) for name, K, N in inputs.DECODE_PROJ}
+RMS_EPS = 1e-6   # the block inputs' RMS normalisation, fused into the q/k/v and gate/up calls
 HIDDEN = PROJ["q"][0]
 
 
@@ -368,15 +369,18 @@ def build_workload(device, layers):
 
 
 def run_layers(W, A, bits):
-    """The 28 chained decoder layers of one bit width (4 launches each)."""
+    """The 28 chained decoder layers of one bit width (4 launches each): q, k, v from the
+    RMS-normalised hidden state, o(v) added into it, gate/up + silu*mul from it normalised again,
+    down added into it."""
     from group_wise_affine_qmv_b200 import aq
     Wb, Ab = W[bits], A[bits]
     h0, h = A["h0"], Ab["h"]
     for layer, m in enumerate(Wb["layers"]):
         x_in = h0 if layer == 0 else h
-        aq.aq_qmm_t_multi(x_in, [m["q"], m["k"], m["v"]], GROUP, bits, outs=[Ab["q"], Ab["k"], Ab["v"]])
+        aq.aq_qmm_t_multi(x_in, [m["q"], m["k"], m["v"]], GROUP, bits, outs=[Ab["q"], Ab["k"], Ab["v"]],
+                          rms_eps=RMS_EPS)
         aq.aq_qmm_t_residual(Ab["v"], *m["o"], GROUP, bits, r=x_in, out=h)
-        aq.aq_qmm_t_swiglu(h, m["gate"], m["up"], GROUP, bits, out=Ab["a"])
+        aq.aq_qmm_t_swiglu(h, m["gate"], m["up"], GROUP, bits, out=Ab["a"], rms_eps=RMS_EPS)
         aq.aq_qmm_t_residual(Ab["a"], *m["down"], GROUP, bits, r=h, out=h)
     return 4 * len(Wb["layers"])
 
@@ -706,10 +710,10 @@ def single_case(name, reps):
         Ab = A[bits]
         if name.startswith("qkv"):
             fn = lambda: aq.aq_qmm_t_multi(A["h0"], [m["q"], m["k"], m["v"]], GROUP, bits,
-                                           outs=[Ab["q"], Ab["k"], Ab["v"]])
+                                           outs=[Ab["q"], Ab["k"], Ab["v"]], rms_eps=RMS_EPS)
             nbytes = layer_launch_bytes(bits)[0]
         elif name.startswith("gateup"):
-            fn = lambda: aq.aq_qmm_t_swiglu(A["h0"], m["gate"], m["up"], GROUP, bits, out=Ab["a"])
+            fn = lambda: aq.aq_qmm_t_swiglu(A["h0"], m["gate"], m["up"], GROUP, bits, out=Ab["a"], rms_eps=RMS_EPS)
             nbytes = layer_launch_bytes(bits)[2]
         else:
             fn = lambda: run_layers(W, A, bits)

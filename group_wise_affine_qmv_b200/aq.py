@@ -84,9 +84,9 @@ def load_library(path: str = LIB_PATH):
         lib.aq_qmv_gathered.argtypes = [V, vp, vp, ctypes.c_int64, V, V, V, ci, ci, V, vp]
         lib.aq_qmv_gathered.restype = ci
         VA = ctypes.POINTER(V)
-        lib.aq_qmm_t_multi.argtypes = [V, ci, VA, VA, VA, ci, ci, VA, vp]
+        lib.aq_qmm_t_multi.argtypes = [V, ci, VA, VA, VA, ci, ci, ctypes.c_float, VA, vp]
         lib.aq_qmm_t_multi.restype = ci
-        lib.aq_qmm_t_swiglu.argtypes = [V, V, V, V, V, V, V, ci, ci, V, vp]
+        lib.aq_qmm_t_swiglu.argtypes = [V, V, V, V, V, V, V, ci, ci, ctypes.c_float, V, vp]
         lib.aq_qmm_t_swiglu.restype = ci
         lib.aq_qmm_t_residual.argtypes = [V, V, V, V, ci, ci, V, V, vp]
         lib.aq_qmm_t_residual.restype = ci
@@ -216,9 +216,10 @@ def aq_qmm_t_grouped(x_sorted, offsets, wq_bank, s_bank, b_bank, group: int, bit
     return out
 
 
-def aq_qmm_t_multi(x, weights, group: int, bits: int, outs=None, out_dtype=None):
+def aq_qmm_t_multi(x, weights, group: int, bits: int, outs=None, out_dtype=None, rms_eps: float = 0.0):
     """y[j] = x . dequant(W_j)^T for up to three (wq, scales, biases) sharing x, in one launch
-    where the warp-level kernel takes them.  Returns the list of outputs."""
+    where the warp-level kernel takes them (rms_eps > 0: x RMS-normalised per token first).
+    Returns the list of outputs."""
     lib = load_library()
     n = len(weights)
     if outs is None:
@@ -228,18 +229,21 @@ def aq_qmm_t_multi(x, weights, group: int, bits: int, outs=None, out_dtype=None)
     keep = [[view(w[i]) for w in weights] for i in range(3)] + [[view(o) for o in outs]]
     arrs = [(V * n)(*[ctypes.pointer(v) for v in vs]) for vs in keep]
     with torch.cuda.device(x.device):
-        _check(lib, lib.aq_qmm_t_multi(view(x), n, arrs[0], arrs[1], arrs[2], group, bits, arrs[3], _stream(x)))
+        _check(lib, lib.aq_qmm_t_multi(view(x), n, arrs[0], arrs[1], arrs[2], group, bits, float(rms_eps), arrs[3],
+                                       _stream(x)))
     return outs
 
 
-def aq_qmm_t_swiglu(x, gate, up, group: int, bits: int, out=None, out_dtype=None):
-    """y = silu(x . dequant(W_gate)^T) * (x . dequant(W_up)^T); gate, up = (wq, scales, biases)."""
+def aq_qmm_t_swiglu(x, gate, up, group: int, bits: int, out=None, out_dtype=None, rms_eps: float = 0.0):
+    """y = silu(x . dequant(W_gate)^T) * (x . dequant(W_up)^T); gate, up = (wq, scales, biases);
+    rms_eps > 0: x RMS-normalised per token first."""
     lib = load_library()
     if out is None:
         out = torch.empty(tuple(x.shape[:-1]) + (gate[0].shape[-2],), dtype=out_dtype or x.dtype, device=x.device)
     with torch.cuda.device(x.device):
         _check(lib, lib.aq_qmm_t_swiglu(view(x), view(gate[0]), view(gate[1]), view(gate[2]), view(up[0]),
-                                        view(up[1]), view(up[2]), group, bits, view(out), _stream(x)))
+                                        view(up[1]), view(up[2]), group, bits, float(rms_eps), view(out),
+                                        _stream(x)))
     return out
 
 

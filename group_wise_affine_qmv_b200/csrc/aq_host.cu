@@ -643,10 +643,11 @@ AQ_API aq_status aq_device_error(void* stream) {
 }
 
 AQ_API aq_status aq_qmm_t_multi(const aq_view* x, int n, const aq_view* const* wq, const aq_view* const* scales,
-                                const aq_view* const* biases, int group, int bits, const aq_view* const* y,
-                                void* stream) {
+                                const aq_view* const* biases, int group, int bits, float rms_eps,
+                                const aq_view* const* y, void* stream) {
     g_msg[0] = 0;
     if (n < 1 || n > 3) return fail(AQ_ERR_UNSUPPORTED, "n=%d matrices (1..3 supported)", n);
+    if (!(rms_eps >= 0.0f)) return fail(AQ_ERR_SHAPE, "rms_eps must be >= 0");
     if (!wq || !scales || !biases || !y) return fail(AQ_ERR_NULL, "NULL array of views");
     Resolved R[3];
     bool all_warp = true;
@@ -669,7 +670,10 @@ AQ_API aq_status aq_qmm_t_multi(const aq_view* x, int n, const aq_view* const* w
         if (st != AQ_OK) ok = false;
         all_warp = ok && R[j].plan.M == R[0].plan.M && R[j].plan.x_row_stride == R[0].plan.x_row_stride;
     }
-    if (!all_warp || n == 1) {
+    if (rms_eps > 0.0f && !all_warp)
+        return fail(AQ_ERR_UNSUPPORTED, "an RMS-normalised input needs the warp-level kernel (up to 32 rows, "
+                                        "2/4/8-bit codes, 16-byte aligned rows)");
+    if (!all_warp || (n == 1 && rms_eps == 0.0f)) {
         // one plain call per matrix, in order, on the same stream
         for (int j = 0; j < n; ++j) {
             aq_status st = run_linear(x, wq[j], scales[j], biases[j], group, bits, y[j], stream, 0);
@@ -679,6 +683,7 @@ AQ_API aq_status aq_qmm_t_multi(const aq_view* x, int n, const aq_view* const* w
     }
     aq::MmaProblem mp = R[0].mp;
     mp.nseg = n;
+    mp.rms_eps = rms_eps;
     for (int j = 0; j < n; ++j) {
         mp.seg_wq[j] = R[j].mp.wq;
         mp.seg_scales[j] = R[j].mp.scales;
@@ -694,8 +699,10 @@ AQ_API aq_status aq_qmm_t_multi(const aq_view* x, int n, const aq_view* const* w
 
 AQ_API aq_status aq_qmm_t_swiglu(const aq_view* x, const aq_view* wq_gate, const aq_view* s_gate,
                                  const aq_view* b_gate, const aq_view* wq_up, const aq_view* s_up,
-                                 const aq_view* b_up, int group, int bits, const aq_view* y, void* stream) {
+                                 const aq_view* b_up, int group, int bits, float rms_eps, const aq_view* y,
+                                 void* stream) {
     g_msg[0] = 0;
+    if (!(rms_eps >= 0.0f)) return fail(AQ_ERR_SHAPE, "rms_eps must be >= 0");
     Resolved Rg, Ru;
     bool okg = false, oku = false;
     aq_status st = resolve_fused_part(x, wq_gate, s_gate, b_gate, group, bits, y, "aq_qmm_t_swiglu", &Rg, &okg);
@@ -711,6 +718,7 @@ AQ_API aq_status aq_qmm_t_swiglu(const aq_view* x, const aq_view* wq_gate, const
     aq::MmaProblem mp = Rg.mp;
     mp.nseg = 2;
     mp.glu = 1;
+    mp.rms_eps = rms_eps;
     const Resolved* parts[2] = {&Rg, &Ru};
     for (int j = 0; j < 2; ++j) {
         mp.seg_wq[j] = parts[j]->mp.wq;

@@ -95,6 +95,9 @@ struct MmaProblem {
     // optional residual of the plain call (warp-level kernel only): y = r + x . W^T
     const void* r;
     int64_t r_row;
+    // fused calls: rms_eps > 0 scales every output of token t by 1 / sqrt(mean_k x[t,k]^2 + rms_eps)
+    // (an RMS-normalised input, the norm's weight folded into W)
+    float rms_eps;
 };
 
 // Whether the tensor-core kernel can run this problem (alignment, bits, K), and why not.

@@ -78,9 +78,10 @@ Shape shape_for(const MmaProblem& p, int sms) {
     s.grid = dim3((unsigned)(((nrt + wr - 1) / wr) * cs), (unsigned)((p.M + nt - 1) / nt),
                   (unsigned)(p.nb[0] * p.nb[1]));
     s.x_pitch = (int)(2 * kgc * p.group + 16);
-    const size_t base = wm::smem_bytes(s.wr * s.wk, s.wr, (int)kg, s.kgc, cs, nt, s.x_pitch, false);
+    const bool rms = p.rms_eps > 0.0f;
+    const size_t base = wm::smem_bytes(s.wr * s.wk, s.wr, (int)kg, s.kgc, cs, nt, s.x_pitch, false, rms);
     s.xsm = base + (size_t)nt * s.x_pitch <= wm::SMEM_LIMIT;
-    s.smem = wm::smem_bytes(s.wr * s.wk, s.wr, (int)kg, s.kgc, cs, nt, s.x_pitch, s.xsm);
+    s.smem = wm::smem_bytes(s.wr * s.wk, s.wr, (int)kg, s.kgc, cs, nt, s.x_pitch, s.xsm, rms);
     return s;
 }
 
@@ -172,6 +173,8 @@ cudaError_t launch_warp_mma(const MmaProblem& pb, cudaStream_t stream) {
     p.xsm = s.xsm ? 1 : 0;
     p.x_pitch = s.x_pitch;
     p.sb16 = sb16 ? 1 : 0;
+    p.rms = pb.rms_eps > 0.0f ? 1 : 0;
+    p.rms_eps = pb.rms_eps;
     const bool bf = pb.xdt == DT::BF16;
     const int warps = s.wr * s.wk;
     switch (pb.bits) {

@@ -57,16 +57,20 @@ struct WParams {
     int xsm;                 // 1: the CTA's x tile is staged in shared memory
     int x_pitch;             // bytes per staged x row (2 K + 16: spreads the lanes over the banks)
     int sb16;                // 1: scale/bias rows are copied in 16-byte pieces (else 4-byte)
+    int rms;                 // 1: the outputs are scaled by 1 / sqrt(mean_k x[t,k]^2 + rms_eps) per token
+    float rms_eps;
 };
 
 constexpr size_t SMEM_LIMIT = 227 * 1024;
 
 // Dynamic shared memory of a launch: the warps' W rings, the sums of x per group and token of the
 // CTA's groups, the scales and biases of the CTA's rows, the CTA's partial tile when a cluster
-// splits K, and, when staged, the x tile.
-inline size_t smem_bytes(int warps, int wr, int kg, int kgc, int cs, int nt, int x_pitch, bool xsm) {
+// splits K, the sums of squares of x (per group and token, then per token) when the inputs are
+// RMS-normalised, and, when staged, the x tile.
+inline size_t smem_bytes(int warps, int wr, int kg, int kgc, int cs, int nt, int x_pitch, bool xsm, bool rms) {
     return (size_t)warps * RING_BYTES + (size_t)kgc * nt * sizeof(float) + (size_t)wr * ROWS * kg * 2 * 2 +
-           (cs > 1 ? (size_t)nt * wr * ROWS * sizeof(float) : 0) + (xsm ? (size_t)nt * x_pitch : 0);
+           (cs > 1 ? (size_t)nt * wr * ROWS * sizeof(float) : 0) + (rms ? (size_t)(kgc + 1) * nt * sizeof(float) : 0) +
+           (xsm ? (size_t)nt * x_pitch : 0);
 }
 
 // defined in warp_mma_kernel.cuh, instantiated in kernels_warp_mma_b<BITS>.cu

@@ -243,13 +243,15 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
     const int cs = p.cs;
     const int rank = cs > 1 ? (int)ptx::cluster_ctarank() : 0;   // K slice of this CTA in its cluster
     // [rings][sums of x: kgc x NT fp32][scales, biases: rows_cta x kg each]
-    // [partial tile: NT x rows_cta fp32, clusters only][x tile: NT x x_pitch]
+    // [partial tile: NT x rows_cta fp32, clusters only][sums of squares of x: (kgc + 1) x NT fp32,
+    // RMS-normalised inputs only][x tile: NT x x_pitch]
     uint8_t* ring = smem + (size_t)warp * RING_BYTES;
     float* xs = reinterpret_cast<float*>(smem + (size_t)nwarps * RING_BYTES);
     uint16_t* s_s = reinterpret_cast<uint16_t*>(xs + p.kgc * NT);
     uint16_t* s_b = s_s + rows_cta * kg;
     float* cpart = reinterpret_cast<float*>(s_b + rows_cta * kg);
-    uint8_t* xt = reinterpret_cast<uint8_t*>(cpart + (cs > 1 ? NT * rows_cta : 0));
+    float* xsq = cpart + (cs > 1 ? NT * rows_cta : 0);
+    uint8_t* xt = reinterpret_cast<uint8_t*>(xsq + (p.rms ? (p.kgc + 1) * NT : 0));
     const int xp = p.x_pitch;
 
     const int64_t bz = blockIdx.z;
@@ -358,18 +360,29 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
             uint4 v[G / 8];
 #pragma unroll
             for (int u = 0; u < G / 8; ++u) v[u] = p.xsm ? src[u] : __ldcg(src + u);
-            float sum = 0.0f;
+            float sum = 0.0f, sq = 0.0f;
 #pragma unroll
             for (int u = 0; u < G / 8; ++u) {
                 float f[8];
                 unpack8(v[u], f, XT{});
 #pragma unroll
-                for (int e = 0; e < 8; ++e) sum += f[e];
+                for (int e = 0; e < 8; ++e) {
+                    sum += f[e];
+                    sq = fmaf(f[e], f[e], sq);
+                }
             }
             xs[i] = sum;
+            if (p.rms) xsq[i] = sq;
         }
     }
     __syncthreads();
+    if (p.rms) {   // per token, the sum of squares over the CTA's K range, groups in order
+        for (int t = threadIdx.x; t < NT; t += blockDim.x) {
+            float s2 = 0.0f;
+            for (int gl = 0; gl < ckg; ++gl) s2 += xsq[gl * NT + t];
+            xsq[p.kgc * NT + t] = s2;
+        }
+    }
 
     // ---- this lane's rows of the scale/bias tiles and x rows ----
     int sb_row[4];   // (row - rowc) * kg for rows roww + 16 m + 8 h + r, index 2 m + h
@@ -495,16 +508,30 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
     auto lrow = [&](int wrr, int it, int e, int half) {
         return wrr * ROWS + (p.glu ? 2 * it + e + half * (ROWS / 2) : 2 * it + e);
     };
+    // RMS-normalised inputs: 1 / sqrt(mean_k x[t,k]^2 + eps) for token tt, the sum of squares
+    // added over the cluster's CTAs in rank order (every CTA's total is final once the first
+    // cluster barrier has passed, which precedes every call with cs > 1)
+    auto rms_scale = [&](int tt) -> float {
+        float s2 = 0.0f;
+        if (cs == 1) {
+            s2 = xsq[p.kgc * NT + tt];
+        } else {
+            const uint32_t a = ptx::smem_u32(xsq + p.kgc * NT + tt);
+            for (int q = 0; q < cs; ++q) s2 += ptx::ld_cluster_f32(ptx::mapa(a, (uint32_t)q));
+        }
+        return rsqrtf(s2 / (float)p.K + p.rms_eps);
+    };
     auto emit = [&](int tt, int wrr, int it, const float (&v)[2][2]) {
         const int64_t tok = tok0 + tt;
         const RowRef rr = row_ref(p, rowc + lrow(wrr, it, 0, 0));
         if (tok >= p.M || !rr.valid) return;
         const WSeg& sg = p.seg[p.glu ? 0 : rr.seg];
         const bool both = rr.n + 1 < sg.N;
-        float o0 = v[0][0], o1 = v[1][0];
+        const float sc = p.rms ? rms_scale(tt) : 1.0f;
+        float o0 = v[0][0] * sc, o1 = v[1][0] * sc;
         if (p.glu) {
-            o0 = silu(v[0][0]) * v[0][1];
-            o1 = silu(v[1][0]) * v[1][1];
+            o0 = silu(o0) * (v[0][1] * sc);
+            o1 = silu(o1) * (v[1][1] * sc);
         }
         if (sg.r) {   // residual: added in fp32 before the one rounding to y's dtype
             const int64_t ro = ybase + tok * sg.r_row + rr.n;

@@ -221,22 +221,34 @@ aq_status aq_qmv_gathered(const aq_view* x, const int64_t* x_ids, const int64_t*
 /* ---------------------------------------------------------------------- */
 
 /*
+ * Optional RMS-normalised input (rms_eps > 0) of aq_qmm_t_multi and aq_qmm_t_swiglu: the block
+ * inputs of the decoder are normalised per token (RMSNorm), and since the contraction is linear
+ * in x the kernel applies the norm to its result instead:
+ *     x . W^T  ->  (x . W^T) / sqrt(mean_k x[t, k]^2 + rms_eps)
+ * with the sum of squares of the widened x formed in fp32 next to sum(x); the norm's weight
+ * vector is taken as folded into W (the decoder's RMSNorm is not on the pages; it keeps a chain
+ * of layers at unit scale).  rms_eps = 0: no normalisation.
+ */
+
+/*
  * aq_qmm_t_multi -- n (1..3) matrices that share one input, in one launch:
  *     y[j] = x . dequant(W_j)^T,  j < n       (e.g. the q, k and v projections)
  * wq[j], scales[j], biases[j], y[j] as for aq_qmm_t, each W_j with its own N_j and
  * the same K; no output may overlap another output or any input.
  * One launch of the warp-level kernel when it takes every matrix (up to 32 rows in
- * total, 2/4/8-bit codes, 16-byte aligned rows); otherwise one aq_qmm_t per matrix,
- * in order, on the same stream (same results to the same bar).
+ * total, 2/4/8-bit codes, 16-byte aligned rows); otherwise, without rms_eps, one
+ * aq_qmm_t per matrix, in order, on the same stream (same results to the same bar),
+ * and with rms_eps > 0, AQ_ERR_UNSUPPORTED.
  */
 aq_status aq_qmm_t_multi(const aq_view* x, int n, const aq_view* const* wq, const aq_view* const* scales,
-                         const aq_view* const* biases, int group, int bits, const aq_view* const* y,
-                         void* stream);
+                         const aq_view* const* biases, int group, int bits, float rms_eps,
+                         const aq_view* const* y, void* stream);
 
 /*
  * aq_qmm_t_swiglu -- the gated MLP input of the decoder layer, in one launch:
  *     y = silu(x . dequant(W_gate)^T) * (x . dequant(W_up)^T),  silu(v) = v / (1 + exp(-v))
- * Both contractions are complete fp32 sums before the activation; y is rounded once.
+ * Both contractions are complete fp32 sums (each scaled by the RMS norm when rms_eps > 0)
+ * before the activation; y is rounded once.
  * W_gate and W_up: [N, K*bits/32] with their scales and biases; y: x.shape[:-1] + [N].
  * (The activation is a reading: the issue names the model, whose MLP is
  * down(silu(gate(h)) * up(h)); the pages do not spell it out.)
@@ -244,7 +256,8 @@ aq_status aq_qmm_t_multi(const aq_view* x, int n, const aq_view* const* wq, cons
  */
 aq_status aq_qmm_t_swiglu(const aq_view* x, const aq_view* wq_gate, const aq_view* s_gate,
                           const aq_view* b_gate, const aq_view* wq_up, const aq_view* s_up,
-                          const aq_view* b_up, int group, int bits, const aq_view* y, void* stream);
+                          const aq_view* b_up, int group, int bits, float rms_eps, const aq_view* y,
+                          void* stream);
 
 /*
  * aq_qmm_t_residual -- a projection that adds into the residual stream, in one launch:

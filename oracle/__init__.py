@@ -19,6 +19,7 @@ arrays into it.  Function-level citations are in the C file; in short:
 * ``linear_grouped`` -- the same per expert segment of a row-sorted x.
 * ``silu`` / ``swiglu`` -- silu(g) * u in fp64 (the gated MLP step of the fused
   gate/up call).
+* ``rms_inv`` -- 1 / sqrt(mean(x^2) + eps) per row (the normalised input option).
 """
 from __future__ import annotations
 
@@ -83,6 +84,8 @@ def _load():
             lib.oracle_silu.restype = ctypes.c_double
             lib.oracle_swiglu.argtypes = [vp, vp, i64, vp]
             lib.oracle_swiglu.restype = None
+            lib.oracle_rms_inv.argtypes = [vp, ci, i64, i64, ctypes.c_double, vp]
+            lib.oracle_rms_inv.restype = None
             lib.oracle_half_to_double.argtypes = [ctypes.c_uint16, ci]
             lib.oracle_half_to_double.restype = ctypes.c_double
             lib.oracle_float_to_half_rne.argtypes = [ctypes.c_float, ci]
@@ -318,3 +321,14 @@ def swiglu(g: np.ndarray, u: np.ndarray) -> np.ndarray:
     out = np.empty(g.shape, np.float64)
     lib.oracle_swiglu(_ptr(g), _ptr(u), g.size, _ptr(out))
     return out
+
+
+def rms_inv(x_bits: np.ndarray, x_dtype: str, eps: float) -> np.ndarray:
+    """1 / sqrt(mean_k x[t, k]^2 + eps) for every row of x [..., K] (half bits), fp64."""
+    lib = _load()
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    K = x.shape[-1]
+    rows = int(np.prod(x.shape[:-1]))
+    out = np.empty(rows, np.float64)
+    lib.oracle_rms_inv(_ptr(x), _dtype_code(x_dtype), rows, K, float(eps), _ptr(out))
+    return out.reshape(x.shape[:-1])

@@ -25,6 +25,9 @@
  *    down(silu(gate(h)) * up(h))): silu(v) = v / (1 + exp(-v)), the one step of the
  *    fused gate/up call that is not a contraction (a reading: the page names the model,
  *    not its activation).
+ *  - The same decoder normalises each block's input per token (RMSNorm,
+ *    x / sqrt(mean(x^2) + eps), its weight folded into W): a reading too, used by
+ *    the fused projections' optional normalised input.
  *  - "mlx PR #4516" (load_vector fix): the bias term bias*sum(x) must be formed
  *    from inputs widened before they are added; the oracle does every sum in
  *    fp64, which is the exact value that fix aims at.
@@ -383,4 +386,21 @@ double oracle_silu(double v) { return v / (1.0 + exp(-v)); }
 
 void oracle_swiglu(const double* g, const double* u, int64_t n, double* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_silu(g[i]) * u[i];
+}
+
+/*
+ * oracle_rms_inv -- per row t of x [rows, K] (half bits, contiguous), in fp64:
+ *     out[t] = 1 / sqrt(sum_k x[t,k]^2 / K + eps)
+ * the per-token factor of an RMS-normalised input (reading: the decoder's RMSNorm with its
+ * weight folded into W).
+ */
+void oracle_rms_inv(const uint16_t* x, int xdtype, int64_t rows, int64_t K, double eps, double* out) {
+    for (int64_t t = 0; t < rows; ++t) {
+        double s2 = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            const double v = oracle_half_to_double(x[t * K + k], xdtype);
+            s2 += v * v;
+        }
+        out[t] = 1.0 / sqrt(s2 / (double)K + eps);
+    }
 }

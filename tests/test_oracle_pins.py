@@ -424,3 +424,18 @@ def test_swiglu_elementwise(orc):
     assert abs(out[0, 2] - (-4.0) * (-(1 - 0.7310585786300049))) <= 1e-15
     assert abs(out[1, 0] - 0.5 * 2 * 0.8807970779778823) <= 1e-15
     assert out[1, 1] == 10.0
+
+
+def test_rms_inv_closed_values(orc):
+    """1 / sqrt(mean(x^2) + eps): a row of 3s and 4s alternating has mean square 12.5; a constant
+    row c has 1 / sqrt(c^2 + eps); scaling a row by 2 halves it (eps = 0); bf16 and f16 bits."""
+    def bits(vals, dt):
+        t_ = torch.tensor(vals, dtype=torch.float32).to(torch.bfloat16 if dt == "bf16" else torch.float16)
+        return lib_half_bits(t_)
+    for dt in ("bf16", "f16"):
+        r = orc.rms_inv(bits([[3.0, 4.0] * 8, [0.5] * 16, [6.0, 8.0] * 8], dt), dt, 0.0)
+        assert abs(r[0] - 1 / np.sqrt(12.5)) <= 1e-15
+        assert abs(r[1] - 2.0) <= 1e-15
+        assert abs(r[2] - r[0] / 2) <= 1e-15
+        e = orc.rms_inv(bits([[0.5] * 16], dt), dt, 1e-2)
+        assert abs(e[0] - 1 / np.sqrt(0.25 + 1e-2)) <= 1e-15
