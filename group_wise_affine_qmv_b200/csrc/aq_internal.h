@@ -114,6 +114,11 @@ bool warp_mma_supported(const MmaProblem& p);
 bool warp_mma_preferred(const MmaProblem& p);
 cudaError_t launch_warp_mma(const MmaProblem& p, cudaStream_t s);
 
+// A 2D tensor map over packed W rows ({words, rows} uint32, row stride in words), box
+// {box_words, box_rows}, no swizzle; false if the driver rejects it.
+bool encode_w_rows(void* map, const uint32_t* wq, int64_t words, int64_t rows, int64_t row_stride_words,
+                   int box_words, int box_rows);
+
 // Device-side error word: bits set by kernels (a bounded wait expired; an index out of range).
 constexpr int DEVERR_TIMEOUT = 1;
 constexpr int DEVERR_INDEX = 2;

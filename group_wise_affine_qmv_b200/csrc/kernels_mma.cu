@@ -366,6 +366,19 @@ cudaError_t launch_bounded_wait_check(uint64_t budget_ns, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+bool encode_w_rows(void* map, const uint32_t* wq, int64_t words, int64_t rows, int64_t row_stride_words,
+                   int box_words, int box_rows) {
+    auto encode = get_encode();
+    if (!encode) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)words, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(row_stride_words * 4)};
+    cuuint32_t box[2] = {(cuuint32_t)box_words, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return encode(static_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(wq), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t device_error_ptr(int** out) {
     static void* cache[64] = {nullptr};
     void* a = nullptr;

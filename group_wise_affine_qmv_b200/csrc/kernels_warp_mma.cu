@@ -175,6 +175,15 @@ cudaError_t launch_warp_mma(const MmaProblem& pb, cudaStream_t stream) {
     p.sb16 = sb16 ? 1 : 0;
     p.rms = pb.rms_eps > 0.0f ? 1 : 0;
     p.rms_eps = pb.rms_eps;
+    cudaError_t e = device_error_ptr(&p.err);
+    if (e != cudaSuccess) return e;
+    // W boxes: one ring sub-block (min(G, 64) codes) of 32 rows, or 16 rows per matrix for gate/up
+    const int ks = pb.group < 64 ? pb.group : 64;
+    const int box_words = ks * pb.bits / 32;
+    for (int i = 0; i < p.nseg; ++i)
+        if (!encode_w_rows(&p.tw[i], p.seg[i].wq, pb.K * pb.bits / 32, p.seg[i].N, p.seg[i].w_row, box_words,
+                           p.glu ? wm::ROWS / 2 : wm::ROWS))
+            return cudaErrorInvalidValue;
     const bool bf = pb.xdt == DT::BF16;
     const int warps = s.wr * s.wk;
     switch (pb.bits) {

@@ -41,24 +41,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
-// Suspend-time hint of every try_wait, in ns (0: none, the hardware's own time limit).  A thread
-// suspended in try_wait resumes as soon as the phase completes, so the hint only decides how
-// often a waiting warp comes back to re-test (and to take an issue slot from the working warps).
-#ifndef AQ_MBAR_SUSPEND_NS
-#define AQ_MBAR_SUSPEND_NS 0
-#endif
-
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
     uint32_t ok;
-#if AQ_MBAR_SUSPEND_NS > 0
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar_addr), "r"(parity), "n"(AQ_MBAR_SUSPEND_NS)
-        : "memory");
-#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -66,7 +50,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
         : "=r"(ok)
         : "r"(bar_addr), "r"(parity)
         : "memory");
-#endif
     return ok != 0;
 }
 
@@ -94,10 +77,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (!done) {
         const long long c0 = clock64();
         const long long limit = (long long)(budget_ns * 2ull);
-        constexpr uint32_t CHECK = AQ_MBAR_SUSPEND_NS > 0 ? 0u : 63u;   // re-test budget/abort every Nth try
         for (uint32_t i = 1;; ++i) {
             if (mbar_try_wait(a, parity)) { done = true; break; }
-            if ((i & CHECK) == 0 && (*abort || clock64() - c0 > limit)) break;
+            if ((i & 63u) == 0 && (*abort || clock64() - c0 > limit)) break;
         }
     }
     return done;
@@ -136,6 +118,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
         : "memory");
+}
+
+// contiguous bytes from global memory into this CTA's shared memory, completion (bytes) on an
+// mbarrier; both addresses 16-byte aligned, size a multiple of 16
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
 }
 
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t c0,

@@ -3,6 +3,7 @@
 // width in kernels_warp_mma_b{2,4,8}.cu).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -17,6 +18,7 @@ constexpr int MAX_TOKENS = 32;       // x rows per token tile: up to four n8 til
 constexpr int RING_BYTES = 8192;     // per-warp ring of W sub-blocks in shared memory
 constexpr int RED_PITCH = ROWS + 4;  // floats per token of a warp's partial y tile (bank spread)
 constexpr int MAX_XTAB_BYTES = 48 * 1024;
+constexpr uint64_t WAIT_NS = 2000000000ull;   // budget of every bounded wait (2 s)
 
 constexpr int MAX_SEGS = 3;          // W matrices sharing one x in one launch
 
@@ -37,6 +39,8 @@ struct WSeg {
 };
 
 struct WParams {
+    CUtensorMap tw[MAX_SEGS];  // W of each segment: 2D {K*bits/32 words, N rows}, box {sub-block words,
+                               // 32 rows (16 in the gate/up layout)}, no swizzle
     const uint16_t* x;       // [nb0, nb1, M, K] through xb / x_row
     WSeg seg[MAX_SEGS];
     int nseg;                // segments (1: a plain call)
@@ -56,7 +60,10 @@ struct WParams {
     int yvec;                // 1: pairs of adjacent y elements may be stored as one vector
     int xsm;                 // 1: the CTA's x tile is staged in shared memory
     int x_pitch;             // bytes per staged x row (2 K + 16: spreads the lanes over the banks)
-    int sb16;                // 1: scale/bias rows are copied in 16-byte pieces (else 4-byte)
+    int sb16;                // 1: each row block's scales and biases are copied as one bulk copy per
+                             //    segment part (K/group a multiple of 8, 16-byte aligned); else 4-byte
+                             //    cp.async copies
+    int* err;                // device error word (DEVERR_TIMEOUT when a bounded wait expires)
     int rms;                 // 1: the outputs are scaled by 1 / sqrt(mean_k x[t,k]^2 + rms_eps) per token
     float rms_eps;
 };
@@ -67,10 +74,14 @@ constexpr size_t SMEM_LIMIT = 227 * 1024;
 // CTA's groups, the scales and biases of the CTA's rows, the CTA's partial tile when a cluster
 // splits K, the sums of squares of x (per group and token, then per token) when the inputs are
 // RMS-normalised, and, when staged, the x tile.
+constexpr int MAX_RD = 16;           // ring slots per warp (one mbarrier each)
+constexpr size_t BAR_BYTES = (1 + MAX_WARPS * MAX_RD) * 8 + 16 + 128;   // staging + ring mbarriers, abort
+                                                                       // flag, base alignment
+
 inline size_t smem_bytes(int warps, int wr, int kg, int kgc, int cs, int nt, int x_pitch, bool xsm, bool rms) {
     return (size_t)warps * RING_BYTES + (size_t)kgc * nt * sizeof(float) + (size_t)wr * ROWS * kg * 2 * 2 +
            (cs > 1 ? (size_t)nt * wr * ROWS * sizeof(float) : 0) + (rms ? (size_t)(kgc + 1) * nt * sizeof(float) : 0) +
-           (xsm ? (size_t)nt * x_pitch : 0);
+           (xsm ? (size_t)nt * x_pitch : 0) + BAR_BYTES;
 }
 
 // defined in warp_mma_kernel.cuh, instantiated in kernels_warp_mma_b<BITS>.cu

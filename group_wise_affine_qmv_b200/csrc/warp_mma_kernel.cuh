@@ -61,16 +61,11 @@ struct Geo {
     static constexpr int KSB = KS * BITS / 8;          // bytes of one W row per sub-block
     static constexpr int LB = KSB / 4;                 // bytes of one W row per lane
     static constexpr int WS = LB / 4;                  // words of one W row per lane
-    static constexpr int RD = RING_BYTES / (ROWS * KSB) < 16 ? RING_BYTES / (ROWS * KSB) : 16;  // ring depth
-    static constexpr int CPR = KSB / 16;               // 16-byte copies per W row
-    static constexpr int CPL = ROWS * CPR / 32;        // 16-byte copies per lane per sub-block
+    static constexpr int RD = RING_BYTES / (ROWS * KSB) < MAX_RD ? RING_BYTES / (ROWS * KSB) : MAX_RD;  // ring depth
     static constexpr int XV = KS / 32;                 // 16-byte x vectors per lane per n tile
-    static_assert(WS >= 1 && CPL >= 1 && RD >= 2 && RD * ROWS * KSB <= RING_BYTES, "sub-block geometry");
+    static_assert(WS >= 1 && KSB % 16 == 0 && RD >= 2 && RD * ROWS * KSB <= RING_BYTES, "sub-block geometry");
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
@@ -230,10 +225,12 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
     constexpr bool BF = std::is_same<XT, bf16_t>::value;
     constexpr int NT = 8 * NTL;
     constexpr int KS = Gm::KS, SPG = Gm::SPG, STEPS = Gm::STEPS, KSB = Gm::KSB, LB = Gm::LB, WS = Gm::WS;
-    constexpr int RD = Gm::RD, CPR = Gm::CPR, CPL = Gm::CPL, XV = Gm::XV;
+    constexpr int RD = Gm::RD, XV = Gm::XV;
     constexpr float OFF = (BF && BITS < 8) ? 128.0f : 0.0f;   // code offset of the expanded A values
 
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    // TMA writes the ring slots: 128-byte aligned (every slot and half slot is a multiple of 128 bytes)
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nwarps = blockDim.x >> 5;
     const int rw = warp % p.wr, kw = warp / p.wr;
@@ -244,7 +241,7 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
     const int rank = cs > 1 ? (int)ptx::cluster_ctarank() : 0;   // K slice of this CTA in its cluster
     // [rings][sums of x: kgc x NT fp32][scales, biases: rows_cta x kg each]
     // [partial tile: NT x rows_cta fp32, clusters only][sums of squares of x: (kgc + 1) x NT fp32,
-    // RMS-normalised inputs only][x tile: NT x x_pitch]
+    // RMS-normalised inputs only][x tile: NT x x_pitch][mbarriers: staging, rings][abort flag]
     uint8_t* ring = smem + (size_t)warp * RING_BYTES;
     float* xs = reinterpret_cast<float*>(smem + (size_t)nwarps * RING_BYTES);
     uint16_t* s_s = reinterpret_cast<uint16_t*>(xs + p.kgc * NT);
@@ -252,6 +249,9 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
     float* cpart = reinterpret_cast<float*>(s_b + rows_cta * kg);
     float* xsq = cpart + (cs > 1 ? NT * rows_cta : 0);
     uint8_t* xt = reinterpret_cast<uint8_t*>(xsq + (p.rms ? (p.kgc + 1) * NT : 0));
+    uint64_t* sbar = reinterpret_cast<uint64_t*>(xt + (p.xsm ? NT * p.x_pitch : 0));
+    uint64_t* wfull = sbar + 1 + warp * MAX_RD;   // this warp's ring slots
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sbar + 1 + MAX_WARPS * MAX_RD);
     const int xp = p.x_pitch;
 
     const int64_t bz = blockIdx.z;
@@ -264,89 +264,133 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
     const int ckg = cg1 > cg0 ? cg1 - cg0 : 0;
     const int g0 = cg0 + kw * p.gpw;                             // groups of this warp
     const int g1 = min(g0 + p.gpw, cg1);
-    const int nsub = (roww / ROWS < p.nrb && g1 > g0) ? (g1 - g0) * SPG : 0;
+    const bool warp_rows = roww / ROWS < p.nrb;
+    const int nsub = (warp_rows && g1 > g0) ? (g1 - g0) * SPG : 0;
+    const bool staged = p.xsm || p.sb16;   // the staging barrier carries bulk copies
+
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(sbar, 1);
+        *abort_flag = 0;
+    }
+    if (lane == 0)
+        for (int s = 0; s < RD; ++s) ptx::mbar_init(&wfull[s], 1);
+    ptx::fence_mbar_init();
+
+    // The W box of this warp's rows for ring step j: one box of 32 rows, or (gate/up) two of 16 rows,
+    // one from each matrix.  TMA reads rows past a matrix's end as zeros.
+    const RowRef wr0 = row_ref(p, min(roww, p.nrb * ROWS - 1));
+    const RowRef wr1 = row_ref(p, min(roww + ROWS / 2, p.nrb * ROWS - 1));
+    auto load_w = [&](int j) {
+        const int slot = j % RD;
+        uint8_t* dst = ring + slot * ROWS * KSB;
+        const int32_t wc = (g0 * SPG + j) * (KSB / 4);   // word coordinate: a multiple of 16 bytes
+        ptx::mbar_arrive_expect_tx(&wfull[slot], (uint32_t)(ROWS * KSB));
+        if (p.glu) {
+            ptx::tma_load_2d(dst, &p.tw[0], &wfull[slot], wc, (int32_t)wr0.n);
+            ptx::tma_load_2d(dst + (ROWS / 2) * KSB, &p.tw[1], &wfull[slot], wc, (int32_t)wr1.n);
+        } else {
+            ptx::tma_load_2d(dst, &p.tw[wr0.seg], &wfull[slot], wc, (int32_t)wr0.n);
+        }
+    };
 
     ptx::pdl_launch_dependents();
-    // The CTA's weights (its rows' K range of W, and their scales and biases) go to L2 while the
-    // previous kernel in the stream may still run: prefetches change no value that any load sees,
-    // so they are safe before the wait; the copies below then hit L2.
-    if (ckg > 0) {
-        const uint32_t seg = (uint32_t)ckg * (G * BITS / 8);   // a multiple of 16 bytes
-        for (int rl = threadIdx.x; rl < rows_cta; rl += blockDim.x) {
-            if ((rowc + rl) / ROWS >= p.nrb) break;
-            const RowRef rr = row_ref(p, rowc + rl);
-            if (!rr.valid) continue;
+    // The CTA's weights go to L2 while the previous kernel in the stream may still run: prefetches
+    // change no value that any load sees, so they are safe before the wait; the copies below then
+    // hit L2.  One TMA prefetch per W box of this warp, and the scale/bias rows of its block.
+    if (lane == 0 && nsub > 0) {
+        for (int j = 0; j < nsub; ++j) {
+            const int32_t wc = (g0 * SPG + j) * (KSB / 4);
+            if (p.glu) {
+                ptx::tma_prefetch_2d(&p.tw[0], wc, (int32_t)wr0.n);
+                ptx::tma_prefetch_2d(&p.tw[1], wc, (int32_t)wr1.n);
+            } else {
+                ptx::tma_prefetch_2d(&p.tw[wr0.seg], wc, (int32_t)wr0.n);
+            }
+        }
+        for (int hp = 0; hp < (p.glu ? 2 : 1); ++hp) {
+            const RowRef& rr = hp ? wr1 : wr0;
             const WSeg& sg = p.seg[rr.seg];
-            ptx::prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(sg.wq + rr.n * sg.w_row) +
-                                      (size_t)cg0 * (G * BITS / 8), seg);
-            ptx::prefetch_l2_range(sg.scales + rr.n * kg + cg0, (size_t)ckg * 2, 0, 1);
-            ptx::prefetch_l2_range(sg.biases + rr.n * kg + cg0, (size_t)ckg * 2, 0, 1);
+            const int64_t nrow = min((int64_t)(p.glu ? ROWS / 2 : ROWS), sg.N - rr.n);
+            if (nrow > 0) {
+                ptx::prefetch_l2_range(sg.scales + rr.n * kg + g0, (size_t)((nrow - 1) * kg + (g1 - g0)) * 2, 0, 1);
+                ptx::prefetch_l2_range(sg.biases + rr.n * kg + g0, (size_t)((nrow - 1) * kg + (g1 - g0)) * 2, 0, 1);
+            }
         }
     }
+    __syncthreads();   // barrier initialisation visible to every thread and to the copy engine
     // x may be the output of the previous kernel in the stream: read nothing before it completed
     ptx::pdl_wait();
 
-    // ---- one copy group: the scales and biases of the CTA's rows, and the x tile when it fits ----
-    {
+    // ---- staging: the CTA's x tile (one bulk copy per token row) and the scales and biases of its
+    // row blocks (one bulk copy per block and matrix part), all on one mbarrier; the first RD W
+    // boxes of every warp on its ring ----
+    if (warp == 0 && staged) {
+        uint32_t bytes = p.xsm ? (uint32_t)(NT * ckg * G * 2) : 0u;
+        if (p.sb16) {
+            for (int b = 0; b < p.wr; ++b) {
+                const int64_t r0 = rowc + b * ROWS;
+                if (r0 / ROWS >= p.nrb) break;
+                for (int hp = 0; hp < (p.glu ? 2 : 1); ++hp) {
+                    const RowRef rr = row_ref(p, r0 + hp * (ROWS / 2));
+                    const int64_t nrow = min((int64_t)(p.glu ? ROWS / 2 : ROWS), p.seg[rr.seg].N - rr.n);
+                    if (nrow > 0) bytes += 2u * (uint32_t)(nrow * kg * 2);
+                }
+            }
+        }
+        if (lane == 0) ptx::mbar_arrive_expect_tx(sbar, bytes);
+        __syncwarp();
+        if (p.xsm && lane < NT) {   // codes [cg0 G, cg1 G) of token row `lane`
+            const int64_t tok = min(tok0 + lane, p.M - 1);
+            ptx::bulk_load(xt + lane * xp, x + tok * p.x_row + (int64_t)cg0 * G, (uint32_t)(ckg * G * 2), sbar);
+        }
+        if (p.sb16) {
+            const int parts = p.glu ? 2 : 1;
+            for (int i = lane; i < p.wr * parts; i += 32) {
+                const int b = i / parts, hp = i - b * parts;
+                const int64_t r0 = rowc + b * ROWS;
+                if (r0 / ROWS >= p.nrb) continue;
+                const RowRef rr = row_ref(p, r0 + hp * (ROWS / 2));
+                const WSeg& sg = p.seg[rr.seg];
+                const int64_t nrow = min((int64_t)(p.glu ? ROWS / 2 : ROWS), sg.N - rr.n);
+                if (nrow <= 0) continue;
+                const int so = (b * ROWS + hp * (ROWS / 2)) * kg;
+                ptx::bulk_load(s_s + so, sg.scales + rr.n * kg, (uint32_t)(nrow * kg * 2), sbar);
+                ptx::bulk_load(s_b + so, sg.biases + rr.n * kg, (uint32_t)(nrow * kg * 2), sbar);
+            }
+        }
+    }
+    if (!p.sb16) {   // 4-byte copies, rows past a matrix's end clamped to its last row
         const uint32_t ss = ptx::smem_u32(s_s), sb = ptx::smem_u32(s_b);
-        const int step = p.sb16 ? 8 : 2;          // elements per copy (16 or 4 bytes)
-        const int cpr = kg / step;
+        const int cpr = kg / 2;
         const int total = rows_cta * cpr;
         for (int i = threadIdx.x; i < total; i += blockDim.x) {
             const int rl = i / cpr, col = i - rl * cpr;
             const RowRef rr = row_ref(p, min(rowc + rl, p.nrb * ROWS - 1));
             const WSeg& sg = p.seg[rr.seg];
-            const int64_t go = rr.n * kg + col * step;
-            const uint32_t so = (uint32_t)((rl * kg + col * step) * 2);
-            if (p.sb16) {
-                cp_async16(ss + so, sg.scales + go);
-                cp_async16(sb + so, sg.biases + go);
-            } else {
-                cp_async4(ss + so, sg.scales + go);
-                cp_async4(sb + so, sg.biases + go);
-            }
-        }
-        if (p.xsm) {   // codes [cg0 G, cg1 G) of every token row
-            const uint32_t xb = ptx::smem_u32(xt);
-            const int xcpr = ckg * G / 8;
-            const int xtotal = NT * xcpr;
-            for (int i = threadIdx.x; i < xtotal; i += blockDim.x) {
-                const int t = i / xcpr, col = i - t * xcpr;
-                const int64_t tok = min(tok0 + t, p.M - 1);
-                cp_async16(xb + (uint32_t)(t * xp + col * 16), x + tok * p.x_row + (int64_t)cg0 * G + col * 8);
-            }
+            const int64_t go = rr.n * kg + col * 2;
+            const uint32_t so = (uint32_t)((rl * kg + col * 2) * 2);
+            cp_async4(ss + so, sg.scales + go);
+            cp_async4(sb + so, sg.biases + go);
         }
         cp_async_commit();
     }
+    if (lane == 0)
+        for (int j = 0; j < RD && j < nsub; ++j) load_w(j);
+    int issued = min(RD, nsub);   // W boxes issued on this warp's ring (warp-uniform count)
+    int waited = 0;               // ... and waited for
 
-    // ---- W ring: lane copies the 16-byte pieces lane + 32 i of each sub-block ----
-    const uint8_t* csrc[CPL];
-    uint32_t cdst[CPL];
-    {
-        const uint32_t ring_s = ptx::smem_u32(ring);
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int q = lane + 32 * i, rl = q / CPR, col = q % CPR;
-            const RowRef rr = row_ref(p, min(roww + rl, p.nrb * ROWS - 1));
-            const WSeg& sg = p.seg[rr.seg];
-            csrc[i] = reinterpret_cast<const uint8_t*>(sg.wq + rr.n * sg.w_row) + (int64_t)g0 * SPG * KSB + col * 16;
-            cdst[i] = ring_s + (uint32_t)(rl * KSB + col * 16);
-        }
+    if (staged && !ptx::mbar_wait(sbar, 0, abort_flag, WAIT_NS)) {
+        *abort_flag = 1;
+        atomicOr(p.err, DEVERR_TIMEOUT);
     }
-    auto issue = [&](int j) {
-        const uint32_t so = (uint32_t)((j % RD) * ROWS * KSB);
-        const int64_t go = (int64_t)j * KSB;
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) cp_async16(cdst[i] + so, csrc[i] + go);
-    };
-#pragma unroll
-    for (int j = 0; j < RD; ++j) {
-        if (j < nsub) issue(j);
-        cp_async_commit();   // one group per sub-block, empty past the end: wait counts stay uniform
+    if (!p.sb16) cp_async_wait<0>();
+    __syncthreads();
+    bool ok = *abort_flag == 0;   // CTA-uniform after the barrier
+    if (!ok && staged && threadIdx.x == 0) {
+        // a staging copy may still be in flight: let it land before its buffers are reused
+        volatile int never = 0;
+        ptx::mbar_wait(sbar, 0, &never, 200000000ull);
     }
-
-    cp_async_wait<RD>();     // this thread's part of the staging group has landed
-    __syncthreads();         // ... and every other thread's
 
     // ---- sums of x per group and token of the tile: xs[(g - cg0) * NT + t] (consecutive threads
     // take consecutive tokens of one group) ----
@@ -360,19 +404,20 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
             uint4 v[G / 8];
 #pragma unroll
             for (int u = 0; u < G / 8; ++u) v[u] = p.xsm ? src[u] : __ldcg(src + u);
-            float sum = 0.0f, sq = 0.0f;
+            // four independent partial sums (x widened to fp32 before any addition), then combined
+            float sum4[4] = {0.0f, 0.0f, 0.0f, 0.0f}, sq4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int u = 0; u < G / 8; ++u) {
                 float f[8];
                 unpack8(v[u], f, XT{});
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    sum += f[e];
-                    sq = fmaf(f[e], f[e], sq);
+                    sum4[e & 3] += f[e];
+                    sq4[e & 3] = fmaf(f[e], f[e], sq4[e & 3]);
                 }
             }
-            xs[i] = sum;
-            if (p.rms) xsq[i] = sq;
+            xs[i] = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+            if (p.rms) xsq[i] = (sq4[0] + sq4[1]) + (sq4[2] + sq4[3]);
         }
     }
     __syncthreads();
@@ -420,9 +465,17 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
 #pragma unroll
                     for (int e = 0; e < 4; ++e) d[m][t][e] = 0.0f;
         }
-        // codes of this sub-block from the ring
-        cp_async_wait<RD - 1>();
-        __syncwarp();
+        // codes of this sub-block from the ring (a bounded wait; after an expiry the warp computes
+        // on whatever the slot holds and the error word says the results are void)
+        if (ok) {
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(&wfull[j % RD], (uint32_t)((j / RD) & 1), abort_flag, WAIT_NS));
+            if (ok) {
+                waited = j + 1;
+            } else if (lane == 0) {
+                *abort_flag = 1;
+                atomicOr(p.err, DEVERR_TIMEOUT);
+            }
+        }
         uint32_t wv[4][WS];
         {
             const uint8_t* slot = rd_lane + (j % RD) * ROWS * KSB;
@@ -430,8 +483,10 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
             for (int mh = 0; mh < 4; ++mh) load_lane_words<LB>(slot + (16 * (mh >> 1) + 8 * (mh & 1)) * KSB, wv[mh]);
         }
         __syncwarp();   // every lane has read the slot before it is refilled
-        if (j + RD < nsub) issue(j + RD);
-        cp_async_commit();
+        if (ok && j + RD < nsub) {
+            if (lane == 0) load_w(j + RD);
+            issued = j + RD + 1;
+        }
 
         uint32_t a[4][STEPS][2];
 #pragma unroll
@@ -479,8 +534,13 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
         }
     }
 
-    // ---- partial tile of this warp into its own ring (no copy is in flight any more) ----
-    cp_async_wait<0>();
+    // ---- partial tile of this warp into its own ring.  Every W box issued has been waited for,
+    // unless a wait expired: then the warp first waits (bounded, ignoring the abort flag) for the
+    // boxes still in flight, so that no copy lands in the ring after it is reused or freed ----
+    if (waited < issued && lane == 0) {
+        volatile int never = 0;
+        for (int j = waited; j < issued; ++j) ptx::mbar_wait(&wfull[j % RD], (uint32_t)((j / RD) & 1), &never, 200000000ull);
+    }
     __syncwarp();
     {
         float* red = reinterpret_cast<float*>(ring);
@@ -500,8 +560,9 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
     // keep the CTA's partial tile for the cluster-wide sum.  An output item is a pair of adjacent
     // rows of one segment's y, or (gate/up layout) a pair of adjacent silu(gate) * up values, whose
     // gate and up sums sit 16 logical rows apart in the same row block. ----
-    const int ipb = p.glu ? ROWS / 4 : ROWS / 2;   // items per row block
-    const int ipt = p.wr * ipb;                    // items per token
+    const int lipb = p.glu ? 3 : 4;                // log2 of the items per row block (8 or 16)
+    const int lipt = lipb + (31 - __clz(p.wr));    // log2 of the items per token (wr: a power of two)
+    const int ipb = 1 << lipb, ipt = 1 << lipt;
     const int total = NT * ipt;
     const int64_t ybase = bo * p.yb[0] + bi * p.yb[1];
     // local logical row of item element e (0, 1) and half (0: the value, or gate; 1: up)
@@ -541,8 +602,8 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
         store_pair<XT>(sg.y, ybase + tok * sg.y_row + rr.n, o0, o1, both, p.yvec != 0, p.ydt);
     };
     for (int i = threadIdx.x; i < total; i += blockDim.x) {
-        const int tt = i / ipt, rp = i - tt * ipt;
-        const int wrr = rp / ipb, it = rp - wrr * ipb;
+        const int tt = i >> lipt, rp = i & (ipt - 1);
+        const int wrr = rp >> lipb, it = rp & (ipb - 1);
         float v[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
         for (int hf = 0; hf < (p.glu ? 2 : 1); ++hf) {
             const int rl = lrow(wrr, it, 0, hf) - wrr * ROWS;   // even: the pair is one float2
@@ -566,8 +627,8 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
         const int i0 = rank * per, i1 = min(i0 + per, total);
         const uint32_t cp_s = ptx::smem_u32(cpart);
         for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
-            const int tt = i / ipt, rp = i - tt * ipt;
-            const int wrr = rp / ipb, it = rp - wrr * ipb;
+            const int tt = i >> lipt, rp = i & (ipt - 1);
+            const int wrr = rp >> lipb, it = rp & (ipb - 1);
             float v[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
             for (int hf = 0; hf < (p.glu ? 2 : 1); ++hf) {
                 const uint32_t off = (uint32_t)((tt * rows_cta + lrow(wrr, it, 0, hf)) * 4);
