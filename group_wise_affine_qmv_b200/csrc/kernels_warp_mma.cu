@@ -22,13 +22,14 @@ int sm_count() {
     return cached[dev];
 }
 
-int tokens_per_tile(int64_t M) { return M <= 8 ? 8 : M <= 16 ? 16 : 32; }
+int tokens_per_tile(int64_t M) { return M <= 8 ? 8 : wm::TILE_TOKENS; }
 
 // scales and biases of a CTA's rows, staged in shared memory
 constexpr int64_t SB_MAX_BYTES = 64 * 1024;
 
 struct Shape {
     int ntl, wr, wk, gpw, cs, kgc;
+    int rd, ring_bytes;
     int x_pitch;
     bool xsm;
     dim3 grid;
@@ -56,7 +57,7 @@ Shape shape_for(const MmaProblem& p, int sms) {
     const int64_t kg = p.K / p.group;
     const int64_t nrt = row_blocks(p);
     const int64_t rows_all = p.M * p.nb[0] * p.nb[1];
-    const int64_t units = (rows_all + wm::MAX_TOKENS - 1) / wm::MAX_TOKENS;
+    const int64_t units = (rows_all + wm::TILE_TOKENS - 1) / wm::TILE_TOKENS;
     int wr = 1;
     while (wr < wm::MAX_WARPS && ((nrt + 2 * wr - 1) / (2 * wr)) * units >= sms &&
            (int64_t)(2 * wr) * wm::ROWS * kg * 4 <= SB_MAX_BYTES)
@@ -78,10 +79,19 @@ Shape shape_for(const MmaProblem& p, int sms) {
     s.grid = dim3((unsigned)(((nrt + wr - 1) / wr) * cs), (unsigned)((p.M + nt - 1) / nt),
                   (unsigned)(p.nb[0] * p.nb[1]));
     s.x_pitch = (int)(2 * kgc * p.group + 16);
+    // ring: a warp's sub-blocks, up to the depth RING_BYTES allows; at least the warp's partial tile
+    const int ks = p.group < 64 ? p.group : 64, ksb = ks * p.bits / 8, spg = p.group / ks;
+    int rdmax = wm::RING_BYTES / (wm::ROWS * ksb);
+    if (rdmax > wm::MAX_RD) rdmax = wm::MAX_RD;
+    s.rd = (int)(gpw * spg < rdmax ? gpw * spg : rdmax);
+    if (s.rd < 1) s.rd = 1;
+    s.ring_bytes = s.rd * wm::ROWS * ksb;
+    const int red_bytes = nt * wm::RED_PITCH * 4;
+    if (s.ring_bytes < red_bytes) s.ring_bytes = (red_bytes + 127) / 128 * 128;
     const bool rms = p.rms_eps > 0.0f;
-    const size_t base = wm::smem_bytes(s.wr * s.wk, s.wr, (int)kg, s.kgc, cs, nt, s.x_pitch, false, rms);
+    const size_t base = wm::smem_bytes(s.wr * s.wk, s.ring_bytes, s.wr, (int)kg, s.kgc, cs, nt, s.x_pitch, false, rms);
     s.xsm = base + (size_t)nt * s.x_pitch <= wm::SMEM_LIMIT;
-    s.smem = wm::smem_bytes(s.wr * s.wk, s.wr, (int)kg, s.kgc, cs, nt, s.x_pitch, s.xsm, rms);
+    s.smem = wm::smem_bytes(s.wr * s.wk, s.ring_bytes, s.wr, (int)kg, s.kgc, cs, nt, s.x_pitch, s.xsm, rms);
     return s;
 }
 
@@ -109,9 +119,9 @@ bool warp_mma_supported(const MmaProblem& p) {
 // Whether the warp kernel is the faster choice for a problem it supports.  Measured on B200 at
 // 8/16/32 tokens against the tcgen05 small-M kernel (decode shapes, K 1024..3072, N 1024..151936):
 // the warp kernel wins every case of up to 16 tokens, and at 32 tokens when each warp of a
-// one-row-block CTA has at most two sub-blocks of K (after a cluster split of K); with more K
-// per warp, or many row blocks per CTA (lm_head), its serial per-warp work outweighs the tcgen05
-// kernel's fixed costs.  The choice depends on N, K and the total rows only.
+// one-row-block CTA has at most four sub-blocks of K (after a cluster split of K); with many row
+// blocks per CTA (lm_head), its serial per-warp work outweighs the tcgen05 kernel's fixed costs.
+// The choice depends on N, K and the total rows only.
 bool warp_mma_preferred(const MmaProblem& p) {
 #if defined(AQ_WARP_MMA) && AQ_WARP_MMA == 2
     return true;
@@ -119,7 +129,7 @@ bool warp_mma_preferred(const MmaProblem& p) {
     const Shape s = shape_for(p, sm_count());
     if (p.M * p.nb[0] * p.nb[1] <= 16) return true;
     const int spg = p.group > 64 ? p.group / 64 : 1;
-    return s.wr == 1 && s.gpw * spg <= 2;
+    return s.wr == 1 && s.gpw * spg <= 4;
 }
 
 cudaError_t launch_warp_mma(const MmaProblem& pb, cudaStream_t stream) {
@@ -173,6 +183,8 @@ cudaError_t launch_warp_mma(const MmaProblem& pb, cudaStream_t stream) {
     p.xsm = s.xsm ? 1 : 0;
     p.x_pitch = s.x_pitch;
     p.sb16 = sb16 ? 1 : 0;
+    p.rd = s.rd;
+    p.ring_bytes = s.ring_bytes;
     p.rms = pb.rms_eps > 0.0f ? 1 : 0;
     p.rms_eps = pb.rms_eps;
     cudaError_t e = device_error_ptr(&p.err);

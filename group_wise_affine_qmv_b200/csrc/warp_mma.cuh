@@ -14,8 +14,9 @@ namespace wm {
 constexpr int ROWS = 32;             // W rows per warp: two m16 tiles of mma.sync
 constexpr int MAX_WARPS = 8;         // warps per CTA
 constexpr int MAX_CLUSTER = 4;       // CTAs of a cluster splitting K
-constexpr int MAX_TOKENS = 32;       // x rows per token tile: up to four n8 tiles
-constexpr int RING_BYTES = 8192;     // per-warp ring of W sub-blocks in shared memory
+constexpr int MAX_TOKENS = 32;       // rows of x (in total) the kernel is chosen for
+constexpr int TILE_TOKENS = 16;      // x rows per token tile: up to two n8 tiles (two CTAs fit an SM)
+constexpr int RING_BYTES = 8192;     // most bytes of a warp's ring of W sub-blocks in shared memory
 constexpr int RED_PITCH = ROWS + 4;  // floats per token of a warp's partial y tile (bank spread)
 constexpr int MAX_XTAB_BYTES = 48 * 1024;
 constexpr uint64_t WAIT_NS = 2000000000ull;   // budget of every bounded wait (2 s)
@@ -64,6 +65,8 @@ struct WParams {
                              //    segment part (K/group a multiple of 8, 16-byte aligned); else 4-byte
                              //    cp.async copies
     int* err;                // device error word (DEVERR_TIMEOUT when a bounded wait expires)
+    int rd;                  // ring slots per warp (a warp's sub-blocks, at most the ring's depth)
+    int ring_bytes;          // bytes of a warp's ring (also holds its partial y tile at the end)
     int rms;                 // 1: the outputs are scaled by 1 / sqrt(mean_k x[t,k]^2 + rms_eps) per token
     float rms_eps;
 };
@@ -78,8 +81,9 @@ constexpr int MAX_RD = 16;           // ring slots per warp (one mbarrier each)
 constexpr size_t BAR_BYTES = (1 + MAX_WARPS * MAX_RD) * 8 + 16 + 128;   // staging + ring mbarriers, abort
                                                                        // flag, base alignment
 
-inline size_t smem_bytes(int warps, int wr, int kg, int kgc, int cs, int nt, int x_pitch, bool xsm, bool rms) {
-    return (size_t)warps * RING_BYTES + (size_t)kgc * nt * sizeof(float) + (size_t)wr * ROWS * kg * 2 * 2 +
+inline size_t smem_bytes(int warps, int ring_bytes, int wr, int kg, int kgc, int cs, int nt, int x_pitch, bool xsm,
+                         bool rms) {
+    return (size_t)warps * ring_bytes + (size_t)kgc * nt * sizeof(float) + (size_t)wr * ROWS * kg * 2 * 2 +
            (cs > 1 ? (size_t)nt * wr * ROWS * sizeof(float) : 0) + (rms ? (size_t)(kgc + 1) * nt * sizeof(float) : 0) +
            (xsm ? (size_t)nt * x_pitch : 0) + BAR_BYTES;
 }

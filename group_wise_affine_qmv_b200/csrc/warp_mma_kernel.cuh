@@ -61,9 +61,8 @@ struct Geo {
     static constexpr int KSB = KS * BITS / 8;          // bytes of one W row per sub-block
     static constexpr int LB = KSB / 4;                 // bytes of one W row per lane
     static constexpr int WS = LB / 4;                  // words of one W row per lane
-    static constexpr int RD = RING_BYTES / (ROWS * KSB) < MAX_RD ? RING_BYTES / (ROWS * KSB) : MAX_RD;  // ring depth
     static constexpr int XV = KS / 32;                 // 16-byte x vectors per lane per n tile
-    static_assert(WS >= 1 && KSB % 16 == 0 && RD >= 2 && RD * ROWS * KSB <= RING_BYTES, "sub-block geometry");
+    static_assert(WS >= 1 && KSB % 16 == 0 && 2 * ROWS * KSB <= RING_BYTES, "sub-block geometry");
 };
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -220,12 +219,13 @@ __device__ __forceinline__ RowRef row_ref(const WParams& p, int64_t r) {
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
 
 template <int BITS, typename XT, int G, int NTL>
-__global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __grid_constant__ WParams p) {
+__global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __grid_constant__ WParams p) {
     using Gm = Geo<BITS, G>;
     constexpr bool BF = std::is_same<XT, bf16_t>::value;
     constexpr int NT = 8 * NTL;
     constexpr int KS = Gm::KS, SPG = Gm::SPG, STEPS = Gm::STEPS, KSB = Gm::KSB, LB = Gm::LB, WS = Gm::WS;
-    constexpr int RD = Gm::RD, XV = Gm::XV;
+    constexpr int XV = Gm::XV;
+    const int RD = p.rd;   // ring slots of this warp
     constexpr float OFF = (BF && BITS < 8) ? 128.0f : 0.0f;   // code offset of the expanded A values
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -242,8 +242,8 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
     // [rings][sums of x: kgc x NT fp32][scales, biases: rows_cta x kg each]
     // [partial tile: NT x rows_cta fp32, clusters only][sums of squares of x: (kgc + 1) x NT fp32,
     // RMS-normalised inputs only][x tile: NT x x_pitch][mbarriers: staging, rings][abort flag]
-    uint8_t* ring = smem + (size_t)warp * RING_BYTES;
-    float* xs = reinterpret_cast<float*>(smem + (size_t)nwarps * RING_BYTES);
+    uint8_t* ring = smem + (size_t)warp * p.ring_bytes;
+    float* xs = reinterpret_cast<float*>(smem + (size_t)nwarps * p.ring_bytes);
     uint16_t* s_s = reinterpret_cast<uint16_t*>(xs + p.kgc * NT);
     uint16_t* s_b = s_s + rows_cta * kg;
     float* cpart = reinterpret_cast<float*>(s_b + rows_cta * kg);
@@ -608,7 +608,7 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 1) qmm_warp_kernel(const __gri
         for (int hf = 0; hf < (p.glu ? 2 : 1); ++hf) {
             const int rl = lrow(wrr, it, 0, hf) - wrr * ROWS;   // even: the pair is one float2
             for (int k = 0; k < p.wk; ++k) {
-                const float* part = reinterpret_cast<const float*>(smem + (size_t)(k * p.wr + wrr) * RING_BYTES);
+                const float* part = reinterpret_cast<const float*>(smem + (size_t)(k * p.wr + wrr) * p.ring_bytes);
                 const float2 u = *reinterpret_cast<const float2*>(part + tt * RED_PITCH + rl);
                 v[0][hf] += u.x;
                 v[1][hf] += u.y;
@@ -686,7 +686,6 @@ cudaError_t launch_n(int ntl, const WParams& p, dim3 grid, int warps, size_t sme
     switch (ntl) {
         case 1: return launch_t<BITS, XT, G, 1>(p, grid, warps, smem, s);
         case 2: return launch_t<BITS, XT, G, 2>(p, grid, warps, smem, s);
-        case 4: return launch_t<BITS, XT, G, 4>(p, grid, warps, smem, s);
     }
     return cudaErrorInvalidValue;
 }
