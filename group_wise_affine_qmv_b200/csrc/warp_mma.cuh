@@ -78,7 +78,7 @@ constexpr size_t SMEM_LIMIT = 227 * 1024;
 // splits K, the sums of squares of x (per group and token, then per token) when the inputs are
 // RMS-normalised, and, when staged, the x tile.
 constexpr int MAX_RD = 16;           // ring slots per warp (one mbarrier each)
-constexpr size_t BAR_BYTES = (1 + MAX_WARPS * MAX_RD) * 8 + 16 + 128;   // staging + ring mbarriers, abort
+constexpr size_t BAR_BYTES = (2 + MAX_WARPS * MAX_RD) * 8 + 16 + 128;   // staging + ring mbarriers, abort
                                                                        // flag, base alignment
 
 inline size_t smem_bytes(int warps, int ring_bytes, int wr, int kg, int kgc, int cs, int nt, int x_pitch, bool xsm,

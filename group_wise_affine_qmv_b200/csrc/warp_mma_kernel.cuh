@@ -250,8 +250,8 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     float* xsq = cpart + (cs > 1 ? NT * rows_cta : 0);
     uint8_t* xt = reinterpret_cast<uint8_t*>(xsq + (p.rms ? (p.kgc + 1) * NT : 0));
     uint64_t* sbar = reinterpret_cast<uint64_t*>(xt + (p.xsm ? NT * p.x_pitch : 0));
-    uint64_t* wfull = sbar + 1 + warp * MAX_RD;   // this warp's ring slots
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(sbar + 1 + MAX_WARPS * MAX_RD);
+    uint64_t* wfull = sbar + 2 + warp * MAX_RD;   // this warp's ring slots
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sbar + 2 + MAX_WARPS * MAX_RD);
     const int xp = p.x_pitch;
 
     const int64_t bz = blockIdx.z;
@@ -266,10 +266,10 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     const int g1 = min(g0 + p.gpw, cg1);
     const bool warp_rows = roww / ROWS < p.nrb;
     const int nsub = (warp_rows && g1 > g0) ? (g1 - g0) * SPG : 0;
-    const bool staged = p.xsm || p.sb16;   // the staging barrier carries bulk copies
 
     if (threadIdx.x == 0) {
-        ptx::mbar_init(sbar, 1);
+        ptx::mbar_init(&sbar[0], 1);
+        ptx::mbar_init(&sbar[1], 1);
         *abort_flag = 0;
     }
     if (lane == 0)
@@ -321,42 +321,44 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     // x may be the output of the previous kernel in the stream: read nothing before it completed
     ptx::pdl_wait();
 
-    // ---- staging: the CTA's x tile (one bulk copy per token row) and the scales and biases of its
-    // row blocks (one bulk copy per block and matrix part), all on one mbarrier; the first RD W
-    // boxes of every warp on its ring ----
-    if (warp == 0 && staged) {
-        uint32_t bytes = p.xsm ? (uint32_t)(NT * ckg * G * 2) : 0u;
-        if (p.sb16) {
-            for (int b = 0; b < p.wr; ++b) {
-                const int64_t r0 = rowc + b * ROWS;
-                if (r0 / ROWS >= p.nrb) break;
-                for (int hp = 0; hp < (p.glu ? 2 : 1); ++hp) {
-                    const RowRef rr = row_ref(p, r0 + hp * (ROWS / 2));
-                    const int64_t nrow = min((int64_t)(p.glu ? ROWS / 2 : ROWS), p.seg[rr.seg].N - rr.n);
-                    if (nrow > 0) bytes += 2u * (uint32_t)(nrow * kg * 2);
-                }
-            }
-        }
-        if (lane == 0) ptx::mbar_arrive_expect_tx(sbar, bytes);
+    // ---- staging: the CTA's x tile (one bulk copy per token row, issued by warp 0 on sbar[0]) and
+    // the scales and biases of its row blocks (one bulk copy per block and matrix part, issued by
+    // warp 1 when there is one, on sbar[1], so that the two sets of copies are issued in parallel);
+    // each issuing warp arms its own barrier first.  The first RD W boxes of every warp are already
+    // on its ring ----
+    const int sb_warp = nwarps > 1 ? 1 : 0;
+    if (warp == 0 && p.xsm) {
+        if (lane == 0) ptx::mbar_arrive_expect_tx(&sbar[0], (uint32_t)(NT * ckg * G * 2));
         __syncwarp();
-        if (p.xsm && lane < NT) {   // codes [cg0 G, cg1 G) of token row `lane`
+        if (lane < NT) {   // codes [cg0 G, cg1 G) of token row `lane`
             const int64_t tok = min(tok0 + lane, p.M - 1);
-            ptx::bulk_load(xt + lane * xp, x + tok * p.x_row + (int64_t)cg0 * G, (uint32_t)(ckg * G * 2), sbar);
+            ptx::bulk_load(xt + lane * xp, x + tok * p.x_row + (int64_t)cg0 * G, (uint32_t)(ckg * G * 2), &sbar[0]);
         }
-        if (p.sb16) {
-            const int parts = p.glu ? 2 : 1;
-            for (int i = lane; i < p.wr * parts; i += 32) {
-                const int b = i / parts, hp = i - b * parts;
-                const int64_t r0 = rowc + b * ROWS;
-                if (r0 / ROWS >= p.nrb) continue;
-                const RowRef rr = row_ref(p, r0 + hp * (ROWS / 2));
-                const WSeg& sg = p.seg[rr.seg];
-                const int64_t nrow = min((int64_t)(p.glu ? ROWS / 2 : ROWS), sg.N - rr.n);
-                if (nrow <= 0) continue;
-                const int so = (b * ROWS + hp * (ROWS / 2)) * kg;
-                ptx::bulk_load(s_s + so, sg.scales + rr.n * kg, (uint32_t)(nrow * kg * 2), sbar);
-                ptx::bulk_load(s_b + so, sg.biases + rr.n * kg, (uint32_t)(nrow * kg * 2), sbar);
-            }
+    }
+    if (warp == sb_warp && p.sb16) {
+        // lane i: part hp of row block b (i < wr * parts <= 16)
+        const int parts = p.glu ? 2 : 1;
+        const int b = lane / parts, hp = lane - b * parts;
+        const int64_t r0 = rowc + b * ROWS;
+        int64_t nrow = 0, n0 = 0;
+        int sgi = 0;
+        if (lane < p.wr * parts && r0 / ROWS < p.nrb) {
+            const RowRef rr = row_ref(p, r0 + hp * (ROWS / 2));
+            sgi = rr.seg;
+            n0 = rr.n;
+            nrow = min((int64_t)(p.glu ? ROWS / 2 : ROWS), p.seg[sgi].N - n0);
+            if (nrow < 0) nrow = 0;
+        }
+        uint32_t bytes = 2u * (uint32_t)(nrow * kg * 2);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+        if (lane == 0) ptx::mbar_arrive_expect_tx(&sbar[1], bytes);
+        __syncwarp();
+        if (nrow > 0) {
+            const WSeg& sg = p.seg[sgi];
+            const int so = (b * ROWS + hp * (ROWS / 2)) * kg;
+            ptx::bulk_load(s_s + so, sg.scales + n0 * kg, (uint32_t)(nrow * kg * 2), &sbar[1]);
+            ptx::bulk_load(s_b + so, sg.biases + n0 * kg, (uint32_t)(nrow * kg * 2), &sbar[1]);
         }
     }
     if (!p.sb16) {   // 4-byte copies, rows past a matrix's end clamped to its last row
@@ -379,17 +381,19 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     int issued = min(RD, nsub);   // W boxes issued on this warp's ring (warp-uniform count)
     int waited = 0;               // ... and waited for
 
-    if (staged && !ptx::mbar_wait(sbar, 0, abort_flag, WAIT_NS)) {
+    if ((p.xsm && !ptx::mbar_wait(&sbar[0], 0, abort_flag, WAIT_NS)) ||
+        (p.sb16 && !ptx::mbar_wait(&sbar[1], 0, abort_flag, WAIT_NS))) {
         *abort_flag = 1;
         atomicOr(p.err, DEVERR_TIMEOUT);
     }
     if (!p.sb16) cp_async_wait<0>();
     __syncthreads();
     bool ok = *abort_flag == 0;   // CTA-uniform after the barrier
-    if (!ok && staged && threadIdx.x == 0) {
+    if (!ok && threadIdx.x == 0) {
         // a staging copy may still be in flight: let it land before its buffers are reused
         volatile int never = 0;
-        ptx::mbar_wait(sbar, 0, &never, 200000000ull);
+        if (p.xsm) ptx::mbar_wait(&sbar[0], 0, &never, 200000000ull);
+        if (p.sb16) ptx::mbar_wait(&sbar[1], 0, &never, 200000000ull);
     }
 
     // ---- sums of x per group and token of the tile: xs[(g - cg0) * NT + t] (consecutive threads
