@@ -89,9 +89,9 @@ Shape shape_for(const MmaProblem& p, int sms) {
     const int red_bytes = nt * wm::RED_PITCH * 4;
     if (s.ring_bytes < red_bytes) s.ring_bytes = (red_bytes + 127) / 128 * 128;
     const bool rms = p.rms_eps > 0.0f;
-    const size_t base = wm::smem_bytes(s.wr * s.wk, s.ring_bytes, s.wr, (int)kg, s.kgc, cs, nt, s.x_pitch, false, rms);
+    const size_t base = wm::smem_bytes(s.wr * s.wk, s.ring_bytes, s.wr, (int)kg, cs, nt, s.x_pitch, false, rms);
     s.xsm = base + (size_t)nt * s.x_pitch <= wm::SMEM_LIMIT;
-    s.smem = wm::smem_bytes(s.wr * s.wk, s.ring_bytes, s.wr, (int)kg, s.kgc, cs, nt, s.x_pitch, s.xsm, rms);
+    s.smem = wm::smem_bytes(s.wr * s.wk, s.ring_bytes, s.wr, (int)kg, cs, nt, s.x_pitch, s.xsm, rms);
     return s;
 }
 

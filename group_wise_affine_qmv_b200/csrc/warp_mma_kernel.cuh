@@ -239,16 +239,15 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     const int rows_cta = p.wr * ROWS;
     const int cs = p.cs;
     const int rank = cs > 1 ? (int)ptx::cluster_ctarank() : 0;   // K slice of this CTA in its cluster
-    // [rings][sums of x: kgc x NT fp32][scales, biases: rows_cta x kg each]
-    // [partial tile: NT x rows_cta fp32, clusters only][sums of squares of x: (kgc + 1) x NT fp32,
-    // RMS-normalised inputs only][x tile: NT x x_pitch][mbarriers: staging, rings][abort flag]
+    // [rings][scales, biases: rows_cta x kg each][partial tile: NT x rows_cta fp32, clusters only]
+    // [sums of squares of x, RMS-normalised inputs only: MAX_WARPS + 1 rows of NT fp32, one per
+    // K-slice warp, then the CTA's total][x tile: NT x x_pitch][mbarriers: staging, rings][abort flag]
     uint8_t* ring = smem + (size_t)warp * p.ring_bytes;
-    float* xs = reinterpret_cast<float*>(smem + (size_t)nwarps * p.ring_bytes);
-    uint16_t* s_s = reinterpret_cast<uint16_t*>(xs + p.kgc * NT);
+    uint16_t* s_s = reinterpret_cast<uint16_t*>(smem + (size_t)nwarps * p.ring_bytes);
     uint16_t* s_b = s_s + rows_cta * kg;
     float* cpart = reinterpret_cast<float*>(s_b + rows_cta * kg);
     float* xsq = cpart + (cs > 1 ? NT * rows_cta : 0);
-    uint8_t* xt = reinterpret_cast<uint8_t*>(xsq + (p.rms ? (p.kgc + 1) * NT : 0));
+    uint8_t* xt = reinterpret_cast<uint8_t*>(xsq + (p.rms ? (MAX_WARPS + 1) * NT : 0));
     uint64_t* sbar = reinterpret_cast<uint64_t*>(xt + (p.xsm ? NT * p.x_pitch : 0));
     uint64_t* wfull = sbar + 2 + warp * MAX_RD;   // this warp's ring slots
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sbar + 2 + MAX_WARPS * MAX_RD);
@@ -280,8 +279,7 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     // one from each matrix.  TMA reads rows past a matrix's end as zeros.
     const RowRef wr0 = row_ref(p, min(roww, p.nrb * ROWS - 1));
     const RowRef wr1 = row_ref(p, min(roww + ROWS / 2, p.nrb * ROWS - 1));
-    auto load_w = [&](int j) {
-        const int slot = j % RD;
+    auto load_w = [&](int j, int slot) {
         uint8_t* dst = ring + slot * ROWS * KSB;
         const int32_t wc = (g0 * SPG + j) * (KSB / 4);   // word coordinate: a multiple of 16 bytes
         ptx::mbar_arrive_expect_tx(&wfull[slot], (uint32_t)(ROWS * KSB));
@@ -294,19 +292,11 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     };
 
     ptx::pdl_launch_dependents();
-    // The CTA's weights go to L2 while the previous kernel in the stream may still run: prefetches
-    // change no value that any load sees, so they are safe before the wait; the copies below then
-    // hit L2.  One TMA prefetch per W box of this warp, and the scale/bias rows of its block.
+    // The scale/bias rows of the warp's block go to L2 while the previous kernel in the stream may
+    // still run: a prefetch changes no value that any load sees, so it is safe before the wait.
+    // (A TMA prefetch of the W boxes as well was measured to slow a chain of decode launches: the
+    // boxes themselves are read once, right after the wait.)
     if (lane == 0 && nsub > 0) {
-        for (int j = 0; j < nsub; ++j) {
-            const int32_t wc = (g0 * SPG + j) * (KSB / 4);
-            if (p.glu) {
-                ptx::tma_prefetch_2d(&p.tw[0], wc, (int32_t)wr0.n);
-                ptx::tma_prefetch_2d(&p.tw[1], wc, (int32_t)wr1.n);
-            } else {
-                ptx::tma_prefetch_2d(&p.tw[wr0.seg], wc, (int32_t)wr0.n);
-            }
-        }
         for (int hp = 0; hp < (p.glu ? 2 : 1); ++hp) {
             const RowRef& rr = hp ? wr1 : wr0;
             const WSeg& sg = p.seg[rr.seg];
@@ -377,7 +367,7 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
         cp_async_commit();
     }
     if (lane == 0)
-        for (int j = 0; j < RD && j < nsub; ++j) load_w(j);
+        for (int j = 0; j < RD && j < nsub; ++j) load_w(j, j);
     int issued = min(RD, nsub);   // W boxes issued on this warp's ring (warp-uniform count)
     int waited = 0;               // ... and waited for
 
@@ -394,43 +384,6 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
         volatile int never = 0;
         if (p.xsm) ptx::mbar_wait(&sbar[0], 0, &never, 200000000ull);
         if (p.sb16) ptx::mbar_wait(&sbar[1], 0, &never, 200000000ull);
-    }
-
-    // ---- sums of x per group and token of the tile: xs[(g - cg0) * NT + t] (consecutive threads
-    // take consecutive tokens of one group) ----
-    {
-        const int total = ckg * NT;
-        for (int i = threadIdx.x; i < total; i += blockDim.x) {
-            const int gl = i / NT, t = i - gl * NT;
-            const uint4* src = p.xsm ? reinterpret_cast<const uint4*>(xt + t * xp + gl * G * 2)
-                                     : reinterpret_cast<const uint4*>(x + min(tok0 + t, p.M - 1) * p.x_row +
-                                                                      (int64_t)(cg0 + gl) * G);
-            uint4 v[G / 8];
-#pragma unroll
-            for (int u = 0; u < G / 8; ++u) v[u] = p.xsm ? src[u] : __ldcg(src + u);
-            // four independent partial sums (x widened to fp32 before any addition), then combined
-            float sum4[4] = {0.0f, 0.0f, 0.0f, 0.0f}, sq4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-            for (int u = 0; u < G / 8; ++u) {
-                float f[8];
-                unpack8(v[u], f, XT{});
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    sum4[e & 3] += f[e];
-                    sq4[e & 3] = fmaf(f[e], f[e], sq4[e & 3]);
-                }
-            }
-            xs[i] = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-            if (p.rms) xsq[i] = (sq4[0] + sq4[1]) + (sq4[2] + sq4[3]);
-        }
-    }
-    __syncthreads();
-    if (p.rms) {   // per token, the sum of squares over the CTA's K range, groups in order
-        for (int t = threadIdx.x; t < NT; t += blockDim.x) {
-            float s2 = 0.0f;
-            for (int gl = 0; gl < ckg; ++gl) s2 += xsq[gl * NT + t];
-            xsq[p.kgc * NT + t] = s2;
-        }
     }
 
     // ---- this lane's rows of the scale/bias tiles and x rows ----
@@ -457,22 +410,34 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[m][t][e] = 0.0f;
     float d[2][NTL][4];
+    // X of the group for this lane's tokens, from an all-ones A tile on the tensor cores: every
+    // row of the product holds the column sums of the x tile, so a lane's accumulator elements
+    // 0 and 1 are X for tokens 2c and 2c + 1 of n tile t (the products are exact, the sums fp32)
+    float xsum[NTL][4];
+    const uint32_t ONES = BF ? 0x3F803F80u : 0x3C003C00u;   // (1, 1) in the activation dtype
+    // RMS-normalised inputs: sum of squares of this lane's x values (token 8 t + r), two chains
+    float sq[NTL][2];
+#pragma unroll
+    for (int t = 0; t < NTL; ++t) sq[t][0] = sq[t][1] = 0.0f;
+    int slot = 0;          // ring slot of sub-block j, and the parity of its fill
+    uint32_t par = 0;
 
 #pragma unroll 1
     for (int j = 0; j < nsub; ++j) {
         const int g = g0 + j / SPG, sub = j % SPG;
         if (sub == 0) {
 #pragma unroll
-            for (int m = 0; m < 2; ++m)
+            for (int t = 0; t < NTL; ++t)
 #pragma unroll
-                for (int t = 0; t < NTL; ++t)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) d[m][t][e] = 0.0f;
+                for (int e = 0; e < 4; ++e) {
+                    d[0][t][e] = d[1][t][e] = 0.0f;
+                    xsum[t][e] = 0.0f;
+                }
         }
         // codes of this sub-block from the ring (a bounded wait; after an expiry the warp computes
         // on whatever the slot holds and the error word says the results are void)
         if (ok) {
-            ok = __all_sync(0xffffffffu, ptx::mbar_wait(&wfull[j % RD], (uint32_t)((j / RD) & 1), abort_flag, WAIT_NS));
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(&wfull[slot], par, abort_flag, WAIT_NS));
             if (ok) {
                 waited = j + 1;
             } else if (lane == 0) {
@@ -482,14 +447,18 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
         }
         uint32_t wv[4][WS];
         {
-            const uint8_t* slot = rd_lane + (j % RD) * ROWS * KSB;
+            const uint8_t* sp = rd_lane + slot * ROWS * KSB;
 #pragma unroll
-            for (int mh = 0; mh < 4; ++mh) load_lane_words<LB>(slot + (16 * (mh >> 1) + 8 * (mh & 1)) * KSB, wv[mh]);
+            for (int mh = 0; mh < 4; ++mh) load_lane_words<LB>(sp + (16 * (mh >> 1) + 8 * (mh & 1)) * KSB, wv[mh]);
         }
         __syncwarp();   // every lane has read the slot before it is refilled
         if (ok && j + RD < nsub) {
-            if (lane == 0) load_w(j + RD);
+            if (lane == 0) load_w(j + RD, slot);
             issued = j + RD + 1;
+        }
+        if (++slot == RD) {
+            slot = 0;
+            par ^= 1u;
         }
 
         uint32_t a[4][STEPS][2];
@@ -507,11 +476,22 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
             }
             const uint32_t* xw = reinterpret_cast<const uint32_t*>(xv);
 #pragma unroll
-            for (int s = 0; s < STEPS; ++s)
+            for (int s = 0; s < STEPS; ++s) {
 #pragma unroll
                 for (int m = 0; m < 2; ++m)
                     mma16816<BF>(d[m][t], a[2 * m][s][0], a[2 * m + 1][s][0], a[2 * m][s][1], a[2 * m + 1][s][1],
                                  xw[2 * s], xw[2 * s + 1]);
+                mma16816<BF>(xsum[t], ONES, ONES, ONES, ONES, xw[2 * s], xw[2 * s + 1]);
+            }
+            if (p.rms) {
+#pragma unroll
+                for (int v = 0; v < XV; ++v) {
+                    float f[8];
+                    unpack8(xv[v], f, XT{});
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) sq[t][e & 1] = fmaf(f[e], f[e], sq[t][e & 1]);
+                }
+            }
         }
 
         if (sub == SPG - 1) {   // fold the group: acc += s * D + (b - OFF * s) * X
@@ -522,10 +502,9 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
                 bv[mh] = half_bits_to_float(s_b[sb_row[mh] + g], XT{});
                 if (OFF != 0.0f) bv[mh] = fmaf(-OFF, sv[mh], bv[mh]);
             }
-            const float* xg = xs + (g - cg0) * NT + 2 * c;
 #pragma unroll
             for (int t = 0; t < NTL; ++t) {
-                const float2 X = *reinterpret_cast<const float2*>(xg + 8 * t);
+                const float2 X = make_float2(xsum[t][0], xsum[t][1]);
 #pragma unroll
                 for (int m = 0; m < 2; ++m)
 #pragma unroll
@@ -546,6 +525,15 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
         for (int j = waited; j < issued; ++j) ptx::mbar_wait(&wfull[j % RD], (uint32_t)((j / RD) & 1), &never, 200000000ull);
     }
     __syncwarp();
+    if (p.rms) {   // the warp's sum of squares per token (its K slice), over the 4 lanes of a row
+#pragma unroll
+        for (int t = 0; t < NTL; ++t) {
+            float v = sq[t][0] + sq[t][1];
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            if (rw == 0 && c == 0) xsq[kw * NT + 8 * t + r] = v;
+        }
+    }
     {
         float* red = reinterpret_cast<float*>(ring);
 #pragma unroll
@@ -573,15 +561,15 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     auto lrow = [&](int wrr, int it, int e, int half) {
         return wrr * ROWS + (p.glu ? 2 * it + e + half * (ROWS / 2) : 2 * it + e);
     };
-    // RMS-normalised inputs: 1 / sqrt(mean_k x[t,k]^2 + eps) for token tt, the sum of squares
-    // added over the cluster's CTAs in rank order (every CTA's total is final once the first
-    // cluster barrier has passed, which precedes every call with cs > 1)
+    // RMS-normalised inputs: 1 / sqrt(mean_k x[t,k]^2 + eps) for token tt: the K-slice warps' sums
+    // of squares added in slice order, then (clusters) the CTAs' totals in rank order (every CTA's
+    // total is written before the first cluster barrier, which precedes every call with cs > 1)
     auto rms_scale = [&](int tt) -> float {
         float s2 = 0.0f;
         if (cs == 1) {
-            s2 = xsq[p.kgc * NT + tt];
+            for (int k = 0; k < p.wk; ++k) s2 += xsq[k * NT + tt];
         } else {
-            const uint32_t a = ptx::smem_u32(xsq + p.kgc * NT + tt);
+            const uint32_t a = ptx::smem_u32(xsq + MAX_WARPS * NT + tt);
             for (int q = 0; q < cs; ++q) s2 += ptx::ld_cluster_f32(ptx::mapa(a, (uint32_t)q));
         }
         return rsqrtf(s2 / (float)p.K + p.rms_eps);
@@ -623,6 +611,11 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
         if (cs == 1) emit(tt, wrr, it, v);
     }
     if (cs > 1) {
+        if (p.rms && threadIdx.x < NT) {   // the CTA's sum of squares per token, slices in order
+            float s2 = 0.0f;
+            for (int k = 0; k < p.wk; ++k) s2 += xsq[k * NT + threadIdx.x];
+            xsq[MAX_WARPS * NT + threadIdx.x] = s2;
+        }
         // every CTA's partial tile is complete and visible cluster-wide (hardware barrier)
         asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
         // this CTA's share of the tile: the CTAs' partials added in rank order over distributed
