@@ -266,9 +266,10 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     const bool warp_rows = roww / ROWS < p.nrb;
     const int nsub = (warp_rows && g1 > g0) ? (g1 - g0) * SPG : 0;
 
+    const int sb_parts = p.glu ? 2 : 1;   // scale/bias copies per row block: one per matrix part
     if (threadIdx.x == 0) {
         ptx::mbar_init(&sbar[0], 1);
-        ptx::mbar_init(&sbar[1], 1);
+        ptx::mbar_init(&sbar[1], p.wr * sb_parts);
         *abort_flag = 0;
     }
     if (lane == 0)
@@ -311,44 +312,42 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     // x may be the output of the previous kernel in the stream: read nothing before it completed
     ptx::pdl_wait();
 
-    // ---- staging: the CTA's x tile (one bulk copy per token row, issued by warp 0 on sbar[0]) and
-    // the scales and biases of its row blocks (one bulk copy per block and matrix part, issued by
-    // warp 1 when there is one, on sbar[1], so that the two sets of copies are issued in parallel);
-    // each issuing warp arms its own barrier first.  The first RD W boxes of every warp are already
-    // on its ring ----
-    const int sb_warp = nwarps > 1 ? 1 : 0;
-    if (warp == 0 && p.xsm) {
-        if (lane == 0) ptx::mbar_arrive_expect_tx(&sbar[0], (uint32_t)(NT * ckg * G * 2));
-        __syncwarp();
-        if (lane < NT) {   // codes [cg0 G, cg1 G) of token row `lane`
-            const int64_t tok = min(tok0 + lane, p.M - 1);
-            ptx::bulk_load(xt + lane * xp, x + tok * p.x_row + (int64_t)cg0 * G, (uint32_t)(ckg * G * 2), &sbar[0]);
+    // ---- staging: the CTA's x tile (one bulk copy per token row) on sbar[0], armed once with the
+    // tile's bytes; the scales and biases of its row blocks (one bulk copy each per block and
+    // matrix part) on sbar[1], where every copying thread arrives with its own bytes.  The copies
+    // are spread over the warps (the issue of bulk copies is serial within a warp), x rows from
+    // lane 0 up and scale/bias parts after them; a copy completing before the barrier is armed
+    // leaves its phase open, as the arming arrival is still pending.  The first RD W boxes of every
+    // warp then go on its ring ----
+    if (p.xsm) {
+        if (threadIdx.x == 0) ptx::mbar_arrive_expect_tx(&sbar[0], (uint32_t)(NT * ckg * G * 2));
+        const int tr = warp + nwarps * lane;   // codes [cg0 G, cg1 G) of token row tr
+        if (tr < NT) {
+            const int64_t tok = min(tok0 + tr, p.M - 1);
+            ptx::bulk_load(xt + tr * xp, x + tok * p.x_row + (int64_t)cg0 * G, (uint32_t)(ckg * G * 2), &sbar[0]);
         }
     }
-    if (warp == sb_warp && p.sb16) {
-        // lane i: part hp of row block b (i < wr * parts <= 16)
-        const int parts = p.glu ? 2 : 1;
-        const int b = lane / parts, hp = lane - b * parts;
-        const int64_t r0 = rowc + b * ROWS;
-        int64_t nrow = 0, n0 = 0;
-        int sgi = 0;
-        if (lane < p.wr * parts && r0 / ROWS < p.nrb) {
-            const RowRef rr = row_ref(p, r0 + hp * (ROWS / 2));
-            sgi = rr.seg;
-            n0 = rr.n;
-            nrow = min((int64_t)(p.glu ? ROWS / 2 : ROWS), p.seg[sgi].N - n0);
-            if (nrow < 0) nrow = 0;
-        }
-        uint32_t bytes = 2u * (uint32_t)(nrow * kg * 2);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
-        if (lane == 0) ptx::mbar_arrive_expect_tx(&sbar[1], bytes);
-        __syncwarp();
-        if (nrow > 0) {
-            const WSeg& sg = p.seg[sgi];
-            const int so = (b * ROWS + hp * (ROWS / 2)) * kg;
-            ptx::bulk_load(s_s + so, sg.scales + n0 * kg, (uint32_t)(nrow * kg * 2), &sbar[1]);
-            ptx::bulk_load(s_b + so, sg.biases + n0 * kg, (uint32_t)(nrow * kg * 2), &sbar[1]);
+    if (p.sb16) {
+        const int q = warp + nwarps * lane - (p.xsm ? NT : 0);   // part q: block q / parts, half q % parts
+        if (q >= 0 && q < p.wr * sb_parts) {
+            const int b = q / sb_parts, hp = q - b * sb_parts;
+            const int64_t r0 = rowc + b * ROWS;
+            int64_t nrow = 0, n0 = 0;
+            int sgi = 0;
+            if (r0 / ROWS < p.nrb) {
+                const RowRef rr = row_ref(p, r0 + hp * (ROWS / 2));
+                sgi = rr.seg;
+                n0 = rr.n;
+                nrow = min((int64_t)(p.glu ? ROWS / 2 : ROWS), p.seg[sgi].N - n0);
+                if (nrow < 0) nrow = 0;
+            }
+            ptx::mbar_arrive_expect_tx(&sbar[1], 2u * (uint32_t)(nrow * kg * 2));
+            if (nrow > 0) {
+                const WSeg& sg = p.seg[sgi];
+                const int so = (b * ROWS + hp * (ROWS / 2)) * kg;
+                ptx::bulk_load(s_s + so, sg.scales + n0 * kg, (uint32_t)(nrow * kg * 2), &sbar[1]);
+                ptx::bulk_load(s_b + so, sg.biases + n0 * kg, (uint32_t)(nrow * kg * 2), &sbar[1]);
+            }
         }
     }
     if (!p.sb16) {   // 4-byte copies, rows past a matrix's end clamped to its last row
@@ -517,6 +516,37 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
         }
     }
 
+    // ---- outputs: sum the warps' K slices in slice order; without a cluster, store; with one,
+    // keep the CTA's partial tile for the cluster-wide sum.  An output item is a pair of adjacent
+    // rows of one segment's y, or (gate/up layout) a pair of adjacent silu(gate) * up values, whose
+    // gate and up sums sit 16 logical rows apart in the same row block. ----
+    const int lipb = p.glu ? 3 : 4;                // log2 of the items per row block (8 or 16)
+    const int lipt = lipb + (31 - __clz(p.wr));    // log2 of the items per token (wr: a power of two)
+    const int ipb = 1 << lipb, ipt = 1 << lipt;
+    const int total = NT * ipt;
+    const int64_t ybase = bo * p.yb[0] + bi * p.yb[1];
+    // local logical row of item element e (0, 1) and half (0: the value, or gate; 1: up)
+    auto lrow = [&](int wrr, int it, int e, int half) {
+        return wrr * ROWS + (p.glu ? 2 * it + e + half * (ROWS / 2) : 2 * it + e);
+    };
+    // the items this CTA emits: all of them, or with a cluster its rank's share
+    const int per = cs > 1 ? (total + cs - 1) / cs : total;
+    const int i_lo = cs > 1 ? rank * per : 0, i_hi = min(i_lo + per, total);
+    // residual (plain calls only) of this thread's first item, read now: its L2 latency overlaps
+    // the partial-tile barrier and sums (and with a cluster, the cluster barrier)
+    float r_first[2] = {0.0f, 0.0f};
+    if (p.seg[0].r != nullptr && i_lo + (int)threadIdx.x < i_hi) {
+        const int i = i_lo + threadIdx.x;
+        const int tt = i >> lipt, rp = i & (ipt - 1);
+        const RowRef rr = row_ref(p, rowc + lrow(rp >> lipb, rp & (ipb - 1), 0, 0));
+        const int64_t tok = tok0 + tt;
+        if (tok < p.M && rr.valid) {
+            const int64_t ro = ybase + tok * p.seg[0].r_row + rr.n;
+            r_first[0] = load_out<XT>(p.seg[0].r, ro, p.ydt);
+            if (rr.n + 1 < p.seg[0].N) r_first[1] = load_out<XT>(p.seg[0].r, ro + 1, p.ydt);
+        }
+    }
+
     // ---- partial tile of this warp into its own ring.  Every W box issued has been waited for,
     // unless a wait expired: then the warp first waits (bounded, ignoring the abort flag) for the
     // boxes still in flight, so that no copy lands in the ring after it is reused or freed ----
@@ -548,19 +578,6 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     }
     __syncthreads();
 
-    // ---- outputs: sum the warps' K slices in slice order; without a cluster, store; with one,
-    // keep the CTA's partial tile for the cluster-wide sum.  An output item is a pair of adjacent
-    // rows of one segment's y, or (gate/up layout) a pair of adjacent silu(gate) * up values, whose
-    // gate and up sums sit 16 logical rows apart in the same row block. ----
-    const int lipb = p.glu ? 3 : 4;                // log2 of the items per row block (8 or 16)
-    const int lipt = lipb + (31 - __clz(p.wr));    // log2 of the items per token (wr: a power of two)
-    const int ipb = 1 << lipb, ipt = 1 << lipt;
-    const int total = NT * ipt;
-    const int64_t ybase = bo * p.yb[0] + bi * p.yb[1];
-    // local logical row of item element e (0, 1) and half (0: the value, or gate; 1: up)
-    auto lrow = [&](int wrr, int it, int e, int half) {
-        return wrr * ROWS + (p.glu ? 2 * it + e + half * (ROWS / 2) : 2 * it + e);
-    };
     // RMS-normalised inputs: 1 / sqrt(mean_k x[t,k]^2 + eps) for token tt: the K-slice warps' sums
     // of squares added in slice order, then (clusters) the CTAs' totals in rank order (every CTA's
     // total is written before the first cluster barrier, which precedes every call with cs > 1)
@@ -574,7 +591,7 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
         }
         return rsqrtf(s2 / (float)p.K + p.rms_eps);
     };
-    auto emit = [&](int tt, int wrr, int it, const float (&v)[2][2]) {
+    auto emit = [&](int i, int tt, int wrr, int it, const float (&v)[2][2]) {
         const int64_t tok = tok0 + tt;
         const RowRef rr = row_ref(p, rowc + lrow(wrr, it, 0, 0));
         if (tok >= p.M || !rr.valid) return;
@@ -587,9 +604,14 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
             o1 = silu(o1) * (v[1][1] * sc);
         }
         if (sg.r) {   // residual: added in fp32 before the one rounding to y's dtype
-            const int64_t ro = ybase + tok * sg.r_row + rr.n;
-            o0 += load_out<XT>(sg.r, ro, p.ydt);
-            if (both) o1 += load_out<XT>(sg.r, ro + 1, p.ydt);
+            if (i == i_lo + (int)threadIdx.x) {
+                o0 += r_first[0];
+                o1 += r_first[1];
+            } else {
+                const int64_t ro = ybase + tok * sg.r_row + rr.n;
+                o0 += load_out<XT>(sg.r, ro, p.ydt);
+                if (both) o1 += load_out<XT>(sg.r, ro + 1, p.ydt);
+            }
         }
         store_pair<XT>(sg.y, ybase + tok * sg.y_row + rr.n, o0, o1, both, p.yvec != 0, p.ydt);
     };
@@ -608,7 +630,7 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
             if (cs > 1)
                 *reinterpret_cast<float2*>(cpart + tt * rows_cta + wrr * ROWS + rl) = make_float2(v[0][hf], v[1][hf]);
         }
-        if (cs == 1) emit(tt, wrr, it, v);
+        if (cs == 1) emit(i, tt, wrr, it, v);
     }
     if (cs > 1) {
         if (p.rms && threadIdx.x < NT) {   // the CTA's sum of squares per token, slices in order
@@ -620,10 +642,8 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
         asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
         // this CTA's share of the tile: the CTAs' partials added in rank order over distributed
         // shared memory
-        const int per = (total + cs - 1) / cs;
-        const int i0 = rank * per, i1 = min(i0 + per, total);
         const uint32_t cp_s = ptx::smem_u32(cpart);
-        for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
+        for (int i = i_lo + threadIdx.x; i < i_hi; i += blockDim.x) {
             const int tt = i >> lipt, rp = i & (ipt - 1);
             const int wrr = rp >> lipb, it = rp & (ipb - 1);
             float v[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
@@ -635,7 +655,7 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
                     v[1][hf] += u.y;
                 }
             }
-            emit(tt, wrr, it, v);
+            emit(i, tt, wrr, it, v);
         }
         // no CTA leaves while another may still read its partial tile
         asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
