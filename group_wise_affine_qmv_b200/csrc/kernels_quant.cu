@@ -77,6 +77,10 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(const QuantArgs a
         }
         __syncwarp();
     }
+    // The matrix kernels stage their weights before their wait on the kernel before them in the
+    // stream.  This kernel never lets a dependent start early, and with every write performed
+    // device-wide before its threads exit, a matrix call right after it reads the new weights.
+    __threadfence();
 }
 
 // One thread per 32-code chunk of a row: out = fma(scale, q, bias) in fp32, rounded to WT.

@@ -293,43 +293,17 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     };
 
     ptx::pdl_launch_dependents();
-    // The scale/bias rows of the warp's block go to L2 while the previous kernel in the stream may
-    // still run: a prefetch changes no value that any load sees, so it is safe before the wait.
-    // (A TMA prefetch of the W boxes as well was measured to slow a chain of decode launches: the
-    // boxes themselves are read once, right after the wait.)
-    if (lane == 0 && nsub > 0) {
-        for (int hp = 0; hp < (p.glu ? 2 : 1); ++hp) {
-            const RowRef& rr = hp ? wr1 : wr0;
-            const WSeg& sg = p.seg[rr.seg];
-            const int64_t nrow = min((int64_t)(p.glu ? ROWS / 2 : ROWS), sg.N - rr.n);
-            if (nrow > 0) {
-                ptx::prefetch_l2_range(sg.scales + rr.n * kg + g0, (size_t)((nrow - 1) * kg + (g1 - g0)) * 2, 0, 1);
-                ptx::prefetch_l2_range(sg.biases + rr.n * kg + g0, (size_t)((nrow - 1) * kg + (g1 - g0)) * 2, 0, 1);
-            }
-        }
-    }
     __syncthreads();   // barrier initialisation visible to every thread and to the copy engine
-    // x may be the output of the previous kernel in the stream: read nothing before it completed
-    ptx::pdl_wait();
 
-    // ---- staging: the CTA's x tile (one bulk copy per token row) on sbar[0], armed once with the
-    // tile's bytes; the scales and biases of its row blocks (one bulk copy each per block and
-    // matrix part) on sbar[1], where every copying thread arrives with its own bytes.  The copies
-    // are spread over the warps (the issue of bulk copies is serial within a warp), x rows from
-    // lane 0 up and scale/bias parts after them; a copy completing before the barrier is armed
-    // leaves its phase open, as the arming arrival is still pending.  The first RD W boxes of every
-    // warp then go on its ring ----
-    if (p.xsm) {
-        if (threadIdx.x == 0) ptx::mbar_arrive_expect_tx(&sbar[0], (uint32_t)(NT * ckg * G * 2));
-        const int tr = warp + nwarps * lane;   // codes [cg0 G, cg1 G) of token row tr
-        if (tr < NT) {
-            const int64_t tok = min(tok0 + tr, p.M - 1);
-            ptx::bulk_load(xt + tr * xp, x + tok * p.x_row + (int64_t)cg0 * G, (uint32_t)(ckg * G * 2), &sbar[0]);
-        }
-    }
+    // ---- weights first.  W, its scales and its biases are constant operands of the call (the
+    // kernel before this one in the stream does not write them), so they are staged before the wait
+    // for that kernel and their copies overlap its tail: the scale/bias blocks of the CTA's rows
+    // (one bulk copy each per block and matrix part) on sbar[1], where every copying thread arrives
+    // with its own bytes, and the first RD W boxes of every warp on its ring.  Bulk copies are issued
+    // one at a time within a warp, so they are spread over the warps. ----
     if (p.sb16) {
-        const int q = warp + nwarps * lane - (p.xsm ? NT : 0);   // part q: block q / parts, half q % parts
-        if (q >= 0 && q < p.wr * sb_parts) {
+        const int q = warp + nwarps * lane;   // part q: block q / parts, half q % parts
+        if (q < p.wr * sb_parts) {
             const int b = q / sb_parts, hp = q - b * sb_parts;
             const int64_t r0 = rowc + b * ROWS;
             int64_t nrow = 0, n0 = 0;
@@ -367,6 +341,21 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     }
     if (lane == 0)
         for (int j = 0; j < RD && j < nsub; ++j) load_w(j, j);
+
+    // x may be the output of the previous kernel in the stream: read nothing before it completed
+    ptx::pdl_wait();
+
+    // ---- the CTA's x tile, one bulk copy per token row (spread over the warps) on sbar[0], armed
+    // once with the tile's bytes: a copy completing before the barrier is armed leaves its phase
+    // open, as the arming arrival is still pending ----
+    if (p.xsm) {
+        if (threadIdx.x == 0) ptx::mbar_arrive_expect_tx(&sbar[0], (uint32_t)(NT * ckg * G * 2));
+        const int tr = warp + nwarps * lane;   // codes [cg0 G, cg1 G) of token row tr
+        if (tr < NT) {
+            const int64_t tok = min(tok0 + tr, p.M - 1);
+            ptx::bulk_load(xt + tr * xp, x + tok * p.x_row + (int64_t)cg0 * G, (uint32_t)(ckg * G * 2), &sbar[0]);
+        }
+    }
     int issued = min(RD, nsub);   // W boxes issued on this warp's ring (warp-uniform count)
     int waited = 0;               // ... and waited for
 

@@ -38,6 +38,14 @@
  *  - Kernels never trap.  A kernel whose internal pipeline wait exceeds its
  *    bound records a device-side error instead; aq_device_error() reads and
  *    clears it (this one call synchronizes the stream).
+ *  - Weights are constant operands.  The tensor-core kernels may start while
+ *    the kernel before them in the stream still runs, and may read wq, scales
+ *    and biases before that kernel has completed (the activations x and r only
+ *    after it).  So the kernel immediately before a matrix call in its stream
+ *    must not write that call's weights, unless it is aq_quantize (whose
+ *    kernel lets no dependent start early and completes its writes before it
+ *    exits).  Weights written earlier in the stream, by a copy, or on another
+ *    stream and ordered by an event, are read correctly.
  */
 #ifndef AQ_H
 #define AQ_H
@@ -156,7 +164,9 @@ aq_status aq_dequantize_rows(const aq_view* wq, const aq_view* scales, const aq_
  * the GEMV.
  * Every kernel keeps W exact (integer codes, scale and bias in fp32).  The
  * tensor-core kernels are launched as programmatic dependents of the previous
- * kernel in the stream: only their set-up overlaps it; stream order is kept.
+ * kernel in the stream: their set-up and (warp-level kernel) the staging of
+ * the weights overlap it, x is read only after it completed (see "Weights are
+ * constant operands" above).
  * Data pointers must be 16-byte aligned.
  */
 aq_status aq_qmm_t(const aq_view* x, const aq_view* wq, const aq_view* scales,
