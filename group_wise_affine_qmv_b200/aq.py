@@ -139,15 +139,19 @@ def _check(lib, status: int):
 # entry points
 # ---------------------------------------------------------------------------
 
-def aq_quantize(w: torch.Tensor, group: int, bits: int, scale_dtype: torch.dtype | None = None):
-    """Group-wise affine quantization of w [N, K] -> (wq uint32 [N, K*bits/32], scales, biases)."""
+def aq_quantize(w: torch.Tensor, group: int, bits: int, scale_dtype: torch.dtype | None = None, out=None):
+    """Group-wise affine quantization of w [N, K] -> (wq uint32 [N, K*bits/32], scales, biases),
+    into ``out`` = (wq, scales, biases) when given."""
     lib = load_library()
     if scale_dtype is None:
         scale_dtype = w.dtype if w.dtype in (torch.bfloat16, torch.float16) else torch.bfloat16
     N, K = w.shape
-    wq = torch.empty((N, K * bits // 32), dtype=torch.int32, device=w.device)
-    sc = torch.empty((N, K // group), dtype=scale_dtype, device=w.device)
-    bi = torch.empty((N, K // group), dtype=scale_dtype, device=w.device)
+    if out is not None:
+        wq, sc, bi = out
+    else:
+        wq = torch.empty((N, K * bits // 32), dtype=torch.int32, device=w.device)
+        sc = torch.empty((N, K // group), dtype=scale_dtype, device=w.device)
+        bi = torch.empty((N, K // group), dtype=scale_dtype, device=w.device)
     with torch.cuda.device(w.device):
         _check(lib, lib.aq_quantize(view(w), group, bits, view(wq), view(sc), view(bi), _stream(w)))
     return wq, sc, bi

@@ -145,3 +145,27 @@ def test_decode_full_size(bits, shape, batch):
     ref = oracle.linear_contig(x.reshape(-1, K).view(torch.int16).numpy().view(np.uint16), "bf16", Q.dequant())
     err = row_errors(y, ref)
     assert np.all(err <= 4e-3), (name, batch, err.max())
+
+
+@pytest.mark.parametrize("rows", [8, 32, 40, 128])
+def test_weights_rewritten_right_before_the_call(rows):
+    """The matrix kernels stage their weights before their wait on the previous kernel in the
+    stream, and aq_quantize is documented as safe to run right before them: quantize new weights
+    into the same buffers and call the matrix op next, eight times on one stream with no
+    synchronisation, and compare every result bit for bit with the same call on freshly quantized
+    weights after a full synchronisation (8/32 rows: warp kernel, 40: tcgen05 small-M, 128: prefill)."""
+    K, N, group, bits = 1024, 2048, 64, 4
+    ws = [inputs.decode_w(K, N, seed=300 + i, device=DEV) for i in range(8)]
+    x = inputs.normal((rows, K), 1.0, torch.bfloat16, seed=301, device=DEV)
+    wq, sc, bi = aq.aq_quantize(ws[0], group, bits)
+    expect = {8: "warp_mma", 32: "warp_mma", 40: "tc_small_m", 128: "tc_prefill"}[rows]
+    assert _kernel(x, wq, sc, bi, group, bits) == expect
+    outs = []
+    for w in ws:
+        aq.aq_quantize(w, group, bits, out=(wq, sc, bi))
+        outs.append(aq.aq_qmm_t(x, wq, sc, bi, group, bits))
+    torch.cuda.synchronize()
+    for w, y in zip(ws, outs):
+        fresh = aq.aq_quantize(w, group, bits)
+        torch.cuda.synchronize()
+        assert torch.equal(y, aq.aq_qmm_t(x, *fresh, group, bits))
