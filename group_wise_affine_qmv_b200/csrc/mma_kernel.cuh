@@ -108,7 +108,7 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const Params& p, int ms) {
     q += p.xres ? (size_t)boxes * NT * 128 : (size_t)p.xst * SUB * NT * 128;
     s.ws = q;
     q += (size_t)p.stages * 128 * ROWB;
-    q = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(q) + 1023) & ~uintptr_t(1023));
+    q += (1024u - (uint32_t)((q - base) & 1023)) & 1023u;   // base is 1024-byte aligned
     s.xtab = reinterpret_cast<float*>(q);
     q += (size_t)min(ms * GPS, p.kg) * NT * 4;
     s.red = reinterpret_cast<float*>(q);
@@ -393,7 +393,9 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
     static_assert(GPS >= 1 && GPS <= 4 && SUB >= 2 && SUB <= 4, "stage geometry");
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // aligned by an offset from the shared array itself, so that every pointer derived from it stays
+    // in the shared address space (shared loads and stores, not generic ones)
+    uint8_t* base = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
     const int NWS = p.n_wstages;
     const int cs = p.ksplit;   // CTAs of a cluster splitting each tile's K (1: none)
     const Smem s = carve<SUB, ROWB, GPS>(base, p, cs > 1 ? split_max_stages(NWS, GPS, cs) : NWS);

@@ -56,7 +56,7 @@ __device__ __forceinline__ PSmem p_carve(uint8_t* base, const Params& p) {
     q += (size_t)p.xst * SUB * NTP * 128;
     s.ws = q;
     q += (size_t)p.stages * 128 * ROWB;
-    q = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(q) + 1023) & ~uintptr_t(1023));
+    q += (1024u - (uint32_t)((q - base) & 1023)) & 1023u;   // base is 1024-byte aligned
     s.sb = reinterpret_cast<uint16_t*>(q);
     q += 2 * 2 * 128 * SCP * 2;
     s.xg = reinterpret_cast<float*>(q);
@@ -121,7 +121,9 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
     static_assert(SUB >= 1 && SUB <= 2, "prefill stages hold one group of 64 or 128 codes");
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // aligned by an offset from the shared array itself, so that every pointer derived from it stays
+    // in the shared address space (shared loads and stores, not generic ones)
+    uint8_t* base = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
     const PSmem s = p_carve<SUB, ROWB>(base, p);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = p.stages, XS = p.xst;

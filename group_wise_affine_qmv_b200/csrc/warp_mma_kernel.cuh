@@ -230,7 +230,9 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
     // TMA writes the ring slots: 128-byte aligned (every slot and half slot is a multiple of 128 bytes)
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    // aligned by an offset from the shared array itself, so that every pointer derived from it stays
+    // in the shared address space (shared loads and stores, not generic ones)
+    uint8_t* smem = smem_raw + ((128u - (ptx::smem_u32(smem_raw) & 127u)) & 127u);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nwarps = blockDim.x >> 5;
     const int rw = warp % p.wr, kw = warp / p.wr;
