@@ -108,9 +108,10 @@ def test_warp_matches_other_kernels():
 
 
 def test_warp_kernel_choice():
-    """Up to 16 rows always take the warp kernel; 32 rows take it while each warp has at most two
-    64-code sub-blocks of K once a cluster splits K (every decode projection), the tcgen05 kernel
-    otherwise (lm_head: many row blocks per CTA; large K with many row blocks)."""
+    """Up to 8 rows always take the warp kernel; 16 rows while a warp has at most eight 64-code
+    sub-blocks of K (not lm_head); 32 rows while each warp of a one-row-block CTA has at most four
+    once a cluster splits K (every decode projection), the tcgen05 kernel otherwise (lm_head: many
+    row blocks per CTA; large K with many row blocks)."""
     def kern(M, K, N):
         x = torch.empty((M, 1, K), dtype=torch.bfloat16, device=DEV)
         wq = torch.empty((N, K // 8), dtype=torch.int32, device=DEV)
@@ -124,6 +125,8 @@ def test_warp_kernel_choice():
     assert kern(32, 1024, 151936) == "tc_small_m"
     assert kern(16, 3072, 1024) == "warp_mma"
     assert kern(8, 1024, 151936) == "warp_mma"
+    assert kern(16, 1024, 151936) == "tc_small_m"
+    assert kern(16, 1024, 4096) == "warp_mma"
     assert kern(4, 1024, 1024) == "gemv"
 
 
