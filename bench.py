@@ -688,7 +688,28 @@ def reference(args):
 
 
 CASES = ("lm_head_w4", "lm_head_w8", "lm_head2x_w4", "prefill_w4", "prefill_w8", "k_w4", "k_w8", "down_w4",
-         "down_w8", "qkv_w4", "qkv_w8", "gateup_w4", "gateup_w8", "layer_w4", "layer_w8")
+         "down_w8", "qkv_w4", "qkv_w8", "gateup_w4", "gateup_w8", "layer_w4", "layer_w8", "step")
+
+
+def step_case(reps):
+    """The timed decode step (28 layers and lm_head, bits 4 and 8: 226 launches), run eagerly once to
+    warm up and then `reps` times, for a launch list of exactly one or more steps."""
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    W, A = build_workload(device, inputs.DECODE_LAYERS)
+    run_step(W, A)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(reps):
+        launches = run_step(W, A)
+    a1.record(stream)
+    a1.synchronize()
+    from group_wise_affine_qmv_b200 import aq
+    aq.aq_device_error()
+    print(json.dumps({"case": "step", "launches_per_step": launches, "reps": reps,
+                      "ms_per_step": round(a0.elapsed_time(a1) / reps, 4), "graph": False}), flush=True)
 
 
 def single_case(name, reps):
@@ -759,6 +780,9 @@ def main():
     ap.add_argument("--case", choices=CASES, help="time one shape alone (profiling) instead of the benchmark")
     ap.add_argument("--reps", type=int, default=3, help="timed calls of --case")
     args = ap.parse_args()
+    if args.case == "step":
+        step_case(args.reps)
+        return
     if args.case:
         single_case(args.case, args.reps)
         return
