@@ -5,35 +5,40 @@
 // x . (s*q + b)^T, "mlx PR #4516", load_vector fix):
 //     y[t, n] = sum_g  s[n,g] * D[n,g,t]  +  b[n,g] * X[g,t]
 //     D[n,g,t] = sum_{k in g} q[n,k] * x[t,k]   (tensor cores, exact integer codes, fp32 sums)
-//     X[g,t]   = sum_{k in g} x[t,k]            (x widened to fp32 before it is summed)
+//     X[g,t]   = sum_{k in g} x[t,k]            (tensor cores against an all-ones tile: the
+//                                                products are exact, the sums fp32)
 //
 // Why a warp-level MMA here.  At a few dozen tokens the contraction has too few columns to keep
-// a tcgen05 tile busy: the time of the tensor-memory kernel goes into moving expanded codes
-// into tensor memory and each group's accumulator out of it, and its set-up (TMEM allocation,
-// barrier rings, a pipeline of specialised warps) dominates the small projections of a decode
-// step.  Here every step stays in the registers of one warp: the packed codes come from shared
-// memory, are expanded in place into mma.sync A fragments, and each group's accumulator is
-// folded into the running output with two FMAs per element.
+// a tcgen05 tile busy: a tcgen05.mma of 32 columns costs as much time as one of 64, the
+// tensor-memory kernel's time goes into moving expanded codes into tensor memory and each
+// group's accumulator out of it, and its set-up (TMEM allocation, barrier rings, a pipeline of
+// specialised warps) dominates the small projections of a decode step.  Here every step stays
+// in the registers of one warp: the packed codes come from shared memory, are expanded in place
+// into mma.sync A fragments, and each group's accumulator is folded into the running output with
+// two FMAs per element.
 //
 // Layout of the work.  A warp owns 32 W rows (two m16 tiles) x NT = 8*NTL tokens (NTL n8 tiles)
 // and a contiguous range of groups; a CTA holds wr x wk warps, wr blocks of rows times wk slices
 // of K, whose partial tiles are summed in shared memory in slice order at the end.  When one row
 // block per CTA would still leave most SMs idle, a thread-block cluster of cs CTAs splits the K
 // of each row block; after a cluster barrier every CTA adds the CTAs' partial tiles, in rank
-// order, for its share of the outputs over distributed shared memory.  No sum depends on timing.  Within a sub-block of KS = min(G, 64) codes, lane (r = lane/4,
-// c = lane%4) owns codes c*KS/4 .. c*KS/4 + KS/4 - 1 of W rows r and r+8 of each m tile, and of
-// x row r of each n tile; k step s of the MMA takes codes 4s .. 4s+3 of every lane's span.  The
-// order of k inside an MMA is thus a permutation of the group's codes, the same for A (codes)
-// and B (x), which leaves every group sum unchanged and lets a lane load its x as plain 16-byte
-// vectors and its codes as one 4-, 8- or 16-byte word run.
+// order, for its share of the outputs over distributed shared memory.  No sum depends on timing.
+// Within a sub-block of KS = min(G, 64) codes, lane (r = lane/4, c = lane%4) owns codes
+// c*KS/4 .. c*KS/4 + KS/4 - 1 of W rows r and r+8 of each m tile, and of x row r of each n tile;
+// k step s of the MMA takes codes 4s .. 4s+3 of every lane's span.  The order of k inside an MMA
+// is thus a permutation of the group's codes, the same for A (codes) and B (x), which leaves
+// every group sum unchanged and lets a lane load its x as plain 16-byte vectors and its codes as
+// one 4-, 8- or 16-byte word run.  Each n tile's x fragments also feed one more MMA per k step
+// with an all-ones A tile, whose every row is then X of the tile's tokens 2c and 2c + 1.
 //
-// Memory.  W streams through a per-warp ring of RD sub-blocks in shared memory, filled with
-// 16-byte cp.async copies that the 32 lanes of the warp share; a lane reads its fragment words
-// back after the ring slot's copy group completed and the warp synchronised, so no other warp
-// is involved.  At the start the CTA stages, in one cp.async group issued before the ring's,
-// the scales and biases of its rows and (when it fits in shared memory) its x tile, so that no
-// group waits on a DRAM round trip of its own; the sums X of the tile are then built once per
-// CTA into shared memory by all threads.  An x tile too large to stage is read through L1.
+// Memory.  W streams through a per-warp ring of RD sub-blocks in shared memory, each slot filled
+// by one TMA box (32 rows of one sub-block; gate/up: 16 rows of each matrix) completing on the
+// slot's mbarrier; a lane reads its fragment words back after the slot's wait and the warp's
+// synchronisation, and one lane refills the slot.  The scales and biases of the CTA's rows are
+// staged by bulk copies.  Both those copies and the first RD boxes of every ring are issued before
+// the wait on the previous kernel in the stream (weights are constant operands of the call); the
+// x tile (when it fits in shared memory), one bulk copy per token row, follows the wait.  An x
+// tile too large to stage is read through L2.
 //
 // Partial rows and tokens: loads of rows past N and of tokens past M are clamped to the last
 // valid one; only the final stores check bounds, so the inner loop carries no bounds test.
