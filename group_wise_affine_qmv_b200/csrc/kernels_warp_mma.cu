@@ -118,9 +118,9 @@ bool warp_mma_supported(const MmaProblem& p) {
 
 // Whether the warp kernel is the faster choice for a problem it supports.  Measured on B200 at
 // 8/16/32 tokens against the tcgen05 small-M kernel (decode shapes, K 1024..3072, N 1024..151936):
-// the warp kernel wins every case of up to 8 tokens; at 16 tokens while a warp has at most eight
-// 64-code sub-blocks of K (lm_head, sixteen per warp, takes 99 us against 64 us on the tcgen05
-// kernel); at 32 tokens when each warp of a one-row-block CTA has at most four sub-blocks (after
+// the warp kernel wins every case of up to 8 tokens; at 16 tokens unless the CTA holds the most
+// row blocks and a warp more than eight 64-code sub-blocks of K (lm_head: eight row blocks and
+// sixteen sub-blocks per warp, 99 us against 64 us on the tcgen05 kernel); at 32 tokens when each warp of a one-row-block CTA has at most four sub-blocks (after
 // a cluster split of K); with many row blocks per CTA its serial per-warp work outweighs the
 // tcgen05 kernel's fixed costs.
 // The choice depends on N, K and the total rows only.
@@ -132,7 +132,7 @@ bool warp_mma_preferred(const MmaProblem& p) {
     const int64_t rows = p.M * p.nb[0] * p.nb[1];
     const int spg = p.group > 64 ? p.group / 64 : 1;
     if (rows <= 8) return true;
-    if (rows <= 16) return s.gpw * spg <= 8;
+    if (rows <= 16) return !(s.wr == wm::MAX_WARPS && s.gpw * spg > 8);
     return s.wr == 1 && s.gpw * spg <= 4;
 }
 

@@ -153,8 +153,8 @@ aq_status aq_dequantize_rows(const aq_view* wq, const aq_view* scales, const aq_
  * Rows per launch batch decide the kernel (aq_plan_linear reports it): up to 4
  * rows (or a batched W), a CUDA-core GEMV; 5..32 rows in total with 2/4/8-bit
  * codes (2-bit codes need groups of 64/128), where measured faster (always up
- * to 8 rows; up to 16 rows unless a warp would hold more than eight 64-code
- * pieces of K, as on a 151936-row lm_head; at 32 rows unless N is so large that
+ * to 8 rows; up to 16 rows unless N is so large that a CTA holds many row
+ * blocks and a warp more than eight 64-code pieces of K (lm_head); at 32 rows unless N is so large that
  * a CTA holds many row blocks, or K per warp is long), a warp-level mma.sync kernel that expands W
  * in registers, K split over a thread-block cluster when row blocks are few;
  * other cases below 64 rows, a tcgen05/TMEM kernel on tiles

@@ -108,8 +108,8 @@ def test_warp_matches_other_kernels():
 
 
 def test_warp_kernel_choice():
-    """Up to 8 rows always take the warp kernel; 16 rows while a warp has at most eight 64-code
-    sub-blocks of K (not lm_head); 32 rows while each warp of a one-row-block CTA has at most four
+    """Up to 8 rows always take the warp kernel; 16 rows unless CTAs of eight row blocks would give
+    a warp more than eight 64-code sub-blocks of K (lm_head); 32 rows while each warp of a one-row-block CTA has at most four
     once a cluster splits K (every decode projection), the tcgen05 kernel otherwise (lm_head: many
     row blocks per CTA; large K with many row blocks)."""
     def kern(M, K, N):
