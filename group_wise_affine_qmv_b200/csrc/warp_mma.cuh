@@ -74,17 +74,15 @@ struct WParams {
 constexpr size_t SMEM_LIMIT = 227 * 1024;
 
 // Dynamic shared memory of a launch: the warps' W rings, the scales and biases of the CTA's rows,
-// the cluster's partial sums of the CTA's outputs when a cluster splits K (one slot per rank), the
-// sums of squares of x (per K-slice warp and token, then per rank and token) when the inputs are
-// RMS-normalised, and, when staged, the x tile.
+// the CTA's partial tile when a cluster splits K, the sums of squares of x (per K-slice warp and
+// token, then per token) when the inputs are RMS-normalised, and, when staged, the x tile.
 constexpr int MAX_RD = 16;           // ring slots per warp (one mbarrier each)
 constexpr size_t BAR_BYTES = (2 + MAX_WARPS * MAX_RD) * 8 + 16 + 128;   // staging + ring mbarriers, abort
                                                                        // flag, base alignment
 
 inline size_t smem_bytes(int warps, int ring_bytes, int wr, int kg, int cs, int nt, int x_pitch, bool xsm, bool rms) {
     return (size_t)warps * ring_bytes + (size_t)wr * ROWS * kg * 2 * 2 +
-           (cs > 1 ? (size_t)(nt * wr * ROWS + 16) * sizeof(float) : 0) +
-           (rms ? (size_t)(MAX_WARPS + MAX_CLUSTER) * nt * sizeof(float) : 0) +
+           (cs > 1 ? (size_t)nt * wr * ROWS * sizeof(float) : 0) + (rms ? (size_t)(MAX_WARPS + 1) * nt * sizeof(float) : 0) +
            (xsm ? (size_t)nt * x_pitch : 0) + BAR_BYTES;
 }
 

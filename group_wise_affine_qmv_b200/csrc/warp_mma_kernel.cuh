@@ -21,9 +21,8 @@
 // and a contiguous range of groups; a CTA holds wr x wk warps, wr blocks of rows times wk slices
 // of K, whose partial tiles are summed in shared memory in slice order at the end.  When one row
 // block per CTA would still leave most SMs idle, a thread-block cluster of cs CTAs splits the K
-// of each row block; every CTA stores its partial sums of each output into the shared memory of
-// the CTA that emits that output (distributed shared memory, one slot per rank), and after one
-// cluster barrier each CTA adds the slots of its outputs in rank order.  No sum depends on timing.
+// of each row block; after a cluster barrier every CTA adds the CTAs' partial tiles, in rank
+// order, for its share of the outputs over distributed shared memory.  No sum depends on timing.
 // Within a sub-block of KS = min(G, 64) codes, lane (r = lane/4, c = lane%4) owns codes
 // c*KS/4 .. c*KS/4 + KS/4 - 1 of W rows r and r+8 of each m tile, and of x row r of each n tile;
 // k step s of the MMA takes codes 4s .. 4s+3 of every lane's span.  The order of k inside an MMA
@@ -247,16 +246,15 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     const int rows_cta = p.wr * ROWS;
     const int cs = p.cs;
     const int rank = cs > 1 ? (int)ptx::cluster_ctarank() : 0;   // K slice of this CTA in its cluster
-    // [rings][scales, biases: rows_cta x kg each][clusters only: the partial sums of the outputs this
-    // CTA emits, one slot per rank: NT x rows_cta + 16 fp32][sums of squares of x, RMS-normalised
-    // inputs only: MAX_WARPS + MAX_CLUSTER rows of NT fp32, one per K-slice warp, then one per rank]
-    // [x tile: NT x x_pitch][mbarriers: staging, rings][abort flag]
+    // [rings][scales, biases: rows_cta x kg each][partial tile: NT x rows_cta fp32, clusters only]
+    // [sums of squares of x, RMS-normalised inputs only: MAX_WARPS + 1 rows of NT fp32, one per
+    // K-slice warp, then the CTA's total][x tile: NT x x_pitch][mbarriers: staging, rings][abort flag]
     uint8_t* ring = smem + (size_t)warp * p.ring_bytes;
     uint16_t* s_s = reinterpret_cast<uint16_t*>(smem + (size_t)nwarps * p.ring_bytes);
     uint16_t* s_b = s_s + rows_cta * kg;
     float* cpart = reinterpret_cast<float*>(s_b + rows_cta * kg);
-    float* xsq = cpart + (cs > 1 ? NT * rows_cta + 16 : 0);
-    uint8_t* xt = reinterpret_cast<uint8_t*>(xsq + (p.rms ? (MAX_WARPS + MAX_CLUSTER) * NT : 0));
+    float* xsq = cpart + (cs > 1 ? NT * rows_cta : 0);
+    uint8_t* xt = reinterpret_cast<uint8_t*>(xsq + (p.rms ? (MAX_WARPS + 1) * NT : 0));
     uint64_t* sbar = reinterpret_cast<uint64_t*>(xt + (p.xsm ? NT * p.x_pitch : 0));
     uint64_t* wfull = sbar + 2 + warp * MAX_RD;   // this warp's ring slots
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sbar + 2 + MAX_WARPS * MAX_RD);
@@ -303,9 +301,6 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
 
     ptx::pdl_launch_dependents();
     __syncthreads();   // barrier initialisation visible to every thread and to the copy engine
-    // clusters: this CTA has started; the matching wait precedes the first store into another CTA's
-    // shared memory, at the end
-    if (cs > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
     // ---- weights first.  W, its scales and its biases are constant operands of the call (the
     // kernel before this one in the stream does not write them), so they are staged before the wait
@@ -580,14 +575,15 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     __syncthreads();
 
     // RMS-normalised inputs: 1 / sqrt(mean_k x[t,k]^2 + eps) for token tt: the K-slice warps' sums
-    // of squares added in slice order, then (clusters) the ranks' totals in rank order (every rank
-    // has stored its total here before the cluster barrier that precedes every call with cs > 1)
+    // of squares added in slice order, then (clusters) the CTAs' totals in rank order (every CTA's
+    // total is written before the first cluster barrier, which precedes every call with cs > 1)
     auto rms_scale = [&](int tt) -> float {
         float s2 = 0.0f;
         if (cs == 1) {
             for (int k = 0; k < p.wk; ++k) s2 += xsq[k * NT + tt];
         } else {
-            for (int q = 0; q < cs; ++q) s2 += xsq[(MAX_WARPS + q) * NT + tt];
+            const uint32_t a = ptx::smem_u32(xsq + MAX_WARPS * NT + tt);
+            for (int q = 0; q < cs; ++q) s2 += ptx::ld_cluster_f32(ptx::mapa(a, (uint32_t)q));
         }
         return rsqrtf(s2 / (float)p.K + p.rms_eps);
     };
@@ -615,14 +611,11 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
         }
         store_pair<XT>(sg.y, ybase + tok * sg.y_row + rr.n, o0, o1, both, p.yvec != 0, p.ydt);
     };
-    const int hfs = p.glu ? 2 : 1;   // halves of an item: the value, or gate and up
-    // clusters: every CTA of the cluster has started (wait of the arrival made in the prologue)
-    if (cs > 1) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
     for (int i = threadIdx.x; i < total; i += blockDim.x) {
         const int tt = i >> lipt, rp = i & (ipt - 1);
         const int wrr = rp >> lipb, it = rp & (ipb - 1);
         float v[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
-        for (int hf = 0; hf < hfs; ++hf) {
+        for (int hf = 0; hf < (p.glu ? 2 : 1); ++hf) {
             const int rl = lrow(wrr, it, 0, hf) - wrr * ROWS;   // even: the pair is one float2
             for (int k = 0; k < p.wk; ++k) {
                 const float* part = reinterpret_cast<const float*>(smem + (size_t)(k * p.wr + wrr) * p.ring_bytes);
@@ -630,40 +623,38 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
                 v[0][hf] += u.x;
                 v[1][hf] += u.y;
             }
-            if (cs > 1) {   // into this rank's slot of the CTA that emits item i
-                const int owner = i / per, li = i - owner * per;
-                const uint32_t dst = ptx::smem_u32(cpart + ((rank * per + li) * hfs + hf) * 2);
-                ptx::st_cluster_f2(ptx::mapa(dst, (uint32_t)owner), make_float2(v[0][hf], v[1][hf]));
-            }
+            if (cs > 1)
+                *reinterpret_cast<float2*>(cpart + tt * rows_cta + wrr * ROWS + rl) = make_float2(v[0][hf], v[1][hf]);
         }
         if (cs == 1) emit(i, tt, wrr, it, v);
     }
     if (cs > 1) {
-        if (p.rms && threadIdx.x < NT) {   // the CTA's sum of squares per token, slices in order,
-            float s2 = 0.0f;               // into this rank's row of every CTA of the cluster
+        if (p.rms && threadIdx.x < NT) {   // the CTA's sum of squares per token, slices in order
+            float s2 = 0.0f;
             for (int k = 0; k < p.wk; ++k) s2 += xsq[k * NT + threadIdx.x];
-            const uint32_t dst = ptx::smem_u32(xsq + (MAX_WARPS + rank) * NT + threadIdx.x);
-            for (int q = 0; q < cs; ++q) ptx::st_cluster_f32(ptx::mapa(dst, (uint32_t)q), s2);
+            xsq[MAX_WARPS * NT + threadIdx.x] = s2;
         }
-        // every CTA's stores into the others' shared memory are complete and visible (hardware
-        // barrier, release / acquire); after it each CTA reads only its own shared memory, so none
-        // has to wait for the others before it exits
+        // every CTA's partial tile is complete and visible cluster-wide (hardware barrier)
         asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-        // this CTA's share of the outputs: the ranks' partials added in rank order
+        // this CTA's share of the tile: the CTAs' partials added in rank order over distributed
+        // shared memory
+        const uint32_t cp_s = ptx::smem_u32(cpart);
         for (int i = i_lo + threadIdx.x; i < i_hi; i += blockDim.x) {
             const int tt = i >> lipt, rp = i & (ipt - 1);
             const int wrr = rp >> lipb, it = rp & (ipb - 1);
-            const int li = i - i_lo;
             float v[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
-            for (int hf = 0; hf < hfs; ++hf) {
+            for (int hf = 0; hf < (p.glu ? 2 : 1); ++hf) {
+                const uint32_t off = (uint32_t)((tt * rows_cta + lrow(wrr, it, 0, hf)) * 4);
                 for (int q = 0; q < cs; ++q) {
-                    const float2 u = *reinterpret_cast<const float2*>(cpart + ((q * per + li) * hfs + hf) * 2);
+                    const float2 u = ptx::ld_cluster_f2(ptx::mapa(cp_s + off, (uint32_t)q));
                     v[0][hf] += u.x;
                     v[1][hf] += u.y;
                 }
             }
             emit(i, tt, wrr, it, v);
         }
+        // no CTA leaves while another may still read its partial tile
+        asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
     }
 }
 
