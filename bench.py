@@ -524,19 +524,29 @@ def ours(args):
             graph.replay()
     torch.cuda.synchronize(device)
 
-    # ---- device-resident timing ----
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(dist, device)
-    with ClockSampler(local) as clk:
-        with torch.cuda.stream(stream):
-            ev0.record(stream)
-            for _ in range(args.steps):
-                graph.replay()
-            ev1.record(stream)
-        ev1.synchronize()
+    # ---- device-resident timing.  A kernel that reports an expired bounded wait voids the run
+    #      (its CTA gave up after 2 s): the timed loop is then measured once more, and the JSON
+    #      line says so (`device_error_remeasured`); a second error ends the run. ----
     from group_wise_affine_qmv_b200 import aq
-    with torch.cuda.stream(stream):
-        aq.aq_device_error()   # a kernel that reported an error (an expired wait) voids the timing
+    remeasured = None
+    for attempt in range(2):
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(dist, device)
+        with ClockSampler(local) as clk:
+            with torch.cuda.stream(stream):
+                ev0.record(stream)
+                for _ in range(args.steps):
+                    graph.replay()
+                ev1.record(stream)
+            ev1.synchronize()
+        try:
+            with torch.cuda.stream(stream):
+                aq.aq_device_error()
+            break
+        except aq.AQError as ex:
+            if attempt == 1:
+                raise
+            remeasured = str(ex)
     barrier(dist, device)
     ms = ev0.elapsed_time(ev1)
     ms_max = max_over_ranks(dist, ms, device)
@@ -604,8 +614,12 @@ def ours(args):
             stream.wait_event(copied[bits])
         f1.record(stream)
     f1.synchronize()
-    with torch.cuda.stream(stream):
-        aq.aq_device_error()
+    e2e_error = None
+    try:
+        with torch.cuda.stream(stream):
+            aq.aq_device_error()
+    except aq.AQError as ex:
+        e2e_error = str(ex)
     del parts
     barrier(dist, device)
     e2e_ms = max_over_ranks(dist, f0.elapsed_time(f1), device)
@@ -644,6 +658,10 @@ def ours(args):
                      "bytes_per_launch": round(per_launch_bytes), "peak_source": peak_kind},
         "clocks": clk.summary(),
     }
+    if remeasured is not None:
+        result["device_error_remeasured"] = remeasured
+    if e2e_error is not None:
+        result["e2e"]["device_error"] = e2e_error
     if not args.no_prefill:
         result["detail"]["prefill"] = prefill_and_moe(device, stream)
         result["detail"]["probe_and_ragged_qmv"] = probe_and_ragged(device, stream)
@@ -794,7 +812,7 @@ def single_case(name, reps):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=inputs.DECODE_LAYERS)

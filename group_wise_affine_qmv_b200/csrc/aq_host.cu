@@ -636,7 +636,27 @@ AQ_API aq_status aq_device_error(void* stream) {
     int v = 0;
     cudaError_t e = aq::read_and_clear_device_error(&v, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
-    if (v & aq::DEVERR_TIMEOUT) return fail(AQ_ERR_TIMEOUT, "a kernel's bounded wait expired (code %d)", v);
+    if (v & aq::DEVERR_TIMEOUT) {
+        static const struct { int bit; const char* name; } at[] = {
+            {aq::DEVERR_AT_WARP_X, "warp-level kernel x staging"}, {aq::DEVERR_AT_WARP_SB, "warp-level kernel scale/bias staging"},
+            {aq::DEVERR_AT_WARP_W, "warp-level kernel W ring"},
+            {aq::DEVERR_AT_TC_WFREE, "small-M W producer (expanders)"}, {aq::DEVERR_AT_TC_XFREE, "small-M x producer (MMA commit)"},
+            {aq::DEVERR_AT_TC_XFULL, "small-M MMA issuer (x copy)"}, {aq::DEVERR_AT_TC_AFULL, "small-M MMA issuer (expanders)"},
+            {aq::DEVERR_AT_TC_DFREE, "small-M MMA issuer (folds)"}, {aq::DEVERR_AT_TC_WFULL, "small-M expanders (W copy)"},
+            {aq::DEVERR_AT_TC_SDONE_E, "small-M expanders (MMA commit)"}, {aq::DEVERR_AT_TC_SDONE_F, "small-M folds (MMA commit)"},
+            {aq::DEVERR_AT_TC_FOLD, "small-M folds (folds, x or cluster)"},
+            {aq::DEVERR_AT_PF_W, "prefill W producer"}, {aq::DEVERR_AT_PF_X, "prefill x producer"},
+            {aq::DEVERR_AT_PF_MMA, "prefill MMA issuer"}, {aq::DEVERR_AT_PF_EXP, "prefill expanders"},
+            {aq::DEVERR_AT_PF_FOLD, "prefill folds"}, {aq::DEVERR_AT_CHECK, "bounded-wait self-check"}};
+        char where[480];
+        where[0] = 0;
+        for (const auto& a : at)
+            if (v & a.bit) {
+                if (where[0]) strncat(where, ", ", sizeof where - strlen(where) - 1);
+                strncat(where, a.name, sizeof where - strlen(where) - 1);
+            }
+        return fail(AQ_ERR_TIMEOUT, "a kernel's bounded wait expired (code %d; at: %s)", v, where[0] ? where : "unrecorded");
+    }
     if (v & aq::DEVERR_INDEX) return fail(AQ_ERR_INDEX, "a row id was outside the table (code %d)", v);
     if (v != 0) return fail(AQ_ERR_CUDA, "unknown device error code %d", v);
     return AQ_OK;

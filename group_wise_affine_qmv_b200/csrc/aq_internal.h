@@ -122,6 +122,26 @@ bool encode_w_rows(void* map, const uint32_t* wq, int64_t words, int64_t rows, i
 // Device-side error word: bits set by kernels (a bounded wait expired; an index out of range).
 constexpr int DEVERR_TIMEOUT = 1;
 constexpr int DEVERR_INDEX = 2;
+// Where a bounded wait expired (set with DEVERR_TIMEOUT by the wait that ran out first, not by the
+// waits that returned because the CTA was already aborting); aq_device_error names them.
+constexpr int DEVERR_AT_WARP_X = 1 << 8;      // warp-level kernel: the x tile's staging copies
+constexpr int DEVERR_AT_WARP_SB = 1 << 9;     //   the scale/bias staging copies
+constexpr int DEVERR_AT_WARP_W = 1 << 10;     //   a W box of a warp's ring
+constexpr int DEVERR_AT_TC_WFREE = 1 << 11;   // tcgen05 small-M kernel: W producer waiting for the expanders
+constexpr int DEVERR_AT_TC_XFREE = 1 << 12;   //   x producer waiting for the MMAs to release an x stage
+constexpr int DEVERR_AT_TC_XFULL = 1 << 13;   //   MMA issuer waiting for an x copy
+constexpr int DEVERR_AT_TC_AFULL = 1 << 14;   //   MMA issuer waiting for the expanders
+constexpr int DEVERR_AT_TC_DFREE = 1 << 15;   //   MMA issuer waiting for the folds
+constexpr int DEVERR_AT_TC_WFULL = 1 << 16;   //   expanders waiting for a W copy
+constexpr int DEVERR_AT_TC_SDONE_E = 1 << 17; //   expanders waiting for MMAs to complete
+constexpr int DEVERR_AT_TC_SDONE_F = 1 << 18; //   folds waiting for MMAs to complete
+constexpr int DEVERR_AT_TC_FOLD = 1 << 19;    //   folds waiting for the other folds, x or the cluster
+constexpr int DEVERR_AT_PF_W = 1 << 20;       // prefill kernel: W producer
+constexpr int DEVERR_AT_PF_X = 1 << 21;       //   x producer
+constexpr int DEVERR_AT_PF_MMA = 1 << 22;     //   MMA issuer
+constexpr int DEVERR_AT_PF_EXP = 1 << 23;     //   code expanders
+constexpr int DEVERR_AT_PF_FOLD = 1 << 24;    //   folds
+constexpr int DEVERR_AT_CHECK = 1 << 25;      // the bounded-wait self-check
 cudaError_t read_and_clear_device_error(int* value, cudaStream_t s);
 // its device address on the current device
 cudaError_t device_error_ptr(int** p);

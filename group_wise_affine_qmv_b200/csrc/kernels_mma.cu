@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(32) bounded_wait_check_kernel(int* err, uint64
     }
     __syncwarp();
     const bool done = ptx::mbar_wait(&bar, 0, &abort_flag, budget_ns);
-    if (!done && threadIdx.x == 0) atomicOr(err, DEVERR_TIMEOUT);
+    if (!done && threadIdx.x == 0) atomicOr(err, DEVERR_TIMEOUT | DEVERR_AT_CHECK);
 }
 
 cudaError_t launch_bounded_wait_check(uint64_t budget_ns, cudaStream_t s) {

@@ -29,7 +29,10 @@ constexpr int MAX_XST = 4;                // streamed x ring
 constexpr int MAX_EXPERTS = 1024;
 constexpr int XTAB_MAX_BYTES = 32 * 1024; // sums of x per group and token of one token tile
 constexpr int XV = 2;                     // 16-byte loads in flight per thread while summing x
-constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait
+constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait on a copy or on the tensor core
+// waits on another role get twice as long, so that a stall is reported by the wait on the copy
+// or MMA that did not complete rather than by the roles queued behind it
+constexpr uint64_t WAIT_ROLE_NS = 2 * WAIT_NS;
 constexpr int ERR_TIMEOUT = 1;
 
 // W stage geometry.  A stage is 128 rows x WSC codes: at most 4 groups (so that two A blocks

@@ -133,9 +133,11 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const Params& p, int ms) {
     return s;
 }
 
-__device__ __forceinline__ void raise_abort(const Params& p, int* abort) {
+// a bounded wait of the CTA expired (or another role's did): abort the CTA; `at` names the role,
+// recorded only by the first to give up
+__device__ __forceinline__ void raise_abort(const Params& p, int* abort, int at) {
+    atomicOr(p.err, ERR_TIMEOUT | (*(volatile int*)abort ? 0 : at));
     *(volatile int*)abort = 1;
-    atomicOr(p.err, ERR_TIMEOUT);
 }
 
 __device__ __forceinline__ int total_tiles(const Params& p, const Smem& s) {
@@ -441,10 +443,13 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
     // after the wait below, and no y is written before it; W, scales and biases are constant
     // operands of the call, so their staging may start before it.
     ptx::pdl_launch_dependents();
+    // the barriers' initialisation is complete and visible to the copy engine before any copy
+    // that completes on them is issued (the same order every other copy of the kernel keeps)
+    __syncthreads();
     int w_pre = 0;   // W stages of the first tile already issued by the W producer (warp-uniform)
     if (!p.offsets && warp == 0) {
-        // The first S W stages of the CTA's first tile go straight onto the ring (the barriers
-        // were initialised by this very thread), the rest of its stages and the next tile's, and
+        // The first S W stages of the CTA's first tile go straight onto the ring, the rest of its
+        // stages and the next tile's, and
         // the scales and biases of both, to L2, while the previous kernel in the stream may still
         // run.  (Grouped tiles depend on the device offsets: nothing before the wait.)
         const int rk = cs > 1 ? (int)(blockIdx.x % cs) : 0;
@@ -527,7 +532,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
             const TileInfo ti = tile_info(p, s, t);
             for (int w = w0; w < w1; ++w) {
                 const int st = wg % S;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfree[st], ((wg / S) & 1) ^ 1, s.abort, WAIT_NS));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfree[st], ((wg / S) & 1) ^ 1, s.abort, WAIT_ROLE_NS));
                 if (!ok) break;
                 if (leader && wg >= (uint32_t)w_pre) {   // the first w_pre were issued before the wait
                     // columns past K (a partial last stage) read as zero fill
@@ -539,7 +544,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
             }
         }
         if (leader && !ok) {
-            raise_abort(p, s.abort);
+            raise_abort(p, s.abort, DEVERR_AT_TC_WFREE);
             // drain: the copies of every issued stage (those issued before the wait included) must
             // land before the CTA exits
             volatile int never = 0;
@@ -572,7 +577,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 for (int w = w0; w < w1; ++w) {
                     const int xs = wg % XS;
                     ok = __all_sync(0xffffffffu,
-                                    ptx::mbar_wait(&s.xfree[xs], ((wg / XS) & 1) ^ 1, s.abort, WAIT_NS));
+                                    ptx::mbar_wait(&s.xfree[xs], ((wg / XS) & 1) ^ 1, s.abort, WAIT_NS));   // MMA commit
                     if (!ok) break;
                     if (leader) {
                         const int nsub = min(SUB, KBLK - w * SUB);
@@ -585,7 +590,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 }
             }
             if (leader && !ok) {
-                raise_abort(p, s.abort);
+                raise_abort(p, s.abort, DEVERR_AT_TC_XFREE);
                 volatile int never = 0;
                 for (uint32_t j = wg >= (uint32_t)XS ? wg - XS : 0; j < wg; ++j)
                     ptx::mbar_wait(&s.xfull[j % XS], (j / XS) & 1, &never, 200000000ull);
@@ -599,6 +604,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         const bool leader = lane == 0;
         uint32_t wg = 0;
         bool ok = true;
+        int at = DEVERR_AT_TC_XFULL;   // which wait gave up
         if (p.xres && has_tiles) ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xres_full, 0, s.abort, WAIT_NS));
         for (int t = tile0; t < ntiles && ok; t += tstep) {
             for (int w = w0; w < w1; ++w, ++wg) {
@@ -610,11 +616,14 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                                     ptx::mbar_wait(&s.xfull[xs], (wg / p.xst) & 1, s.abort, WAIT_NS));
                     if (!ok) break;
                 }
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.afull[slot], ph, s.abort, WAIT_NS));
+                at = DEVERR_AT_TC_AFULL;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.afull[slot], ph, s.abort, WAIT_ROLE_NS));
                 if (!ok) break;
                 // the folds have read this slot's accumulators (stage wg - 2)
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.dfree[slot], ph ^ 1, s.abort, WAIT_NS));
+                at = DEVERR_AT_TC_DFREE;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.dfree[slot], ph ^ 1, s.abort, WAIT_ROLE_NS));
                 if (!ok) break;
+                at = DEVERR_AT_TC_XFULL;
                 ptx::tc_fence_after();
                 if (leader) {
                     const uint32_t a_blk = tbase + (uint32_t)(slot * ACOLS);
@@ -644,7 +653,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 __syncwarp();
             }
         }
-        if (!ok && leader) raise_abort(p, s.abort);
+        if (!ok && leader) raise_abort(p, s.abort, at);
         // every MMA this warp issued must retire before tensor memory is freed
         if (leader) {
             ptx::mma_commit(s.mdone);
@@ -662,9 +671,11 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         uint32_t wg = 0;
         bool ok = true;
+        int at = DEVERR_AT_TC_WFULL;   // which wait gave up
         for (int t = tile0; t < ntiles && ok; t += tstep) {
             for (int w = w0; w < w1; ++w, ++wg) {
                 const int st = wg % S;
+                at = DEVERR_AT_TC_WFULL;
                 ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfull[st], (wg / S) & 1, s.abort, WAIT_NS));
                 if (!ok) break;
                 // expand the whole stage into registers while the MMAs of stage wg - 2 may still
@@ -681,6 +692,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                     }
                 }
                 if (wg >= 2) {
+                    at = DEVERR_AT_TC_SDONE_E;
                     ok = __all_sync(0xffffffffu,
                                     ptx::mbar_wait(&s.sdone[wg & 1], ((wg >> 1) & 1) ^ 1, s.abort, WAIT_NS));
                     if (!ok) break;
@@ -699,7 +711,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 }
             }
         }
-        if (!ok) raise_abort(p, s.abort);
+        if (!ok) raise_abort(p, s.abort, at);
     } else {
         // ======================= folds =======================
         // Thread <-> W row; warps q and q + 4 take 16 tokens each.  Per stage:
@@ -713,6 +725,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         uint32_t wg = 0, xph = 0;
         int unit = 0;
         bool ok = true;
+        int at = DEVERR_AT_TC_FOLD;   // which wait gave up
 
         if (has_tiles) {
             const TileInfo t0 = tile_info(p, s, tile0);
@@ -729,7 +742,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
             if (ti.xrow0 != cur_x0 || ti.b0 != cur_b0 || ti.b1 != cur_b1 || ti.tvalid != cur_tv) {
                 // sums of x for this token tile
                 ptx::mbar_arrive(s.xbar);  // everyone is done reading the previous table
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_NS));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_ROLE_NS));
                 ++xph;
                 if (!ok) break;
                 if (p.xres) {
@@ -740,7 +753,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                     build_xtab<XT, G>(p, ti, g_lo, g_hi, s.xtab, tid);
                 }
                 ptx::mbar_arrive(s.xbar);
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_NS));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.xbar, xph & 1, s.abort, WAIT_ROLE_NS));
                 ++xph;
                 if (!ok) break;
                 cur_x0 = ti.xrow0;
@@ -757,7 +770,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                     ptx::cp_async_wait_all();
                     ptx::mbar_arrive(&s.sbar[unit & 1]);
                     ok = __all_sync(0xffffffffu,
-                                    ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS));
+                                    ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_ROLE_NS));
                     if (!ok) break;
                     sbslot = s.sb + (unit & 1) * 2 * 128 * SCP;
                     g_chunk0 = g_lo + ((w - w0) / CS_W) * SCW;
@@ -773,7 +786,10 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 }
                 const int slot = wg & 1;
                 ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.sdone[slot], (wg >> 1) & 1, s.abort, WAIT_NS));
-                if (!ok) break;
+                if (!ok) {
+                    at = DEVERR_AT_TC_SDONE_F;
+                    break;
+                }
                 ptx::tc_fence_after();
 #pragma unroll
                 for (int lg = 0; lg < GPS; ++lg) {
@@ -822,7 +838,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 __syncwarp();
                 if (lane == 0)
                     for (int r = 0; r < cs; ++r) ptx::mbar_arrive_cluster(ptx::mapa(ptx::smem_u32(s.red_full), (uint32_t)r));
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait_cluster(s.red_full, 0, s.abort, WAIT_NS));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait_cluster(s.red_full, 0, s.abort, WAIT_ROLE_NS));
                 if (!ok) break;
                 // this thread: elements [tid*F, tid*F + F) of the owned [rpr][NT] block
                 const int F = (128 * NT) / (cs * FOLD_THREADS);
@@ -853,7 +869,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
             }
         }
         ptx::cp_async_wait_all();
-        if (!ok) raise_abort(p, s.abort);
+        if (!ok) raise_abort(p, s.abort, at);
     }
 
     ptx::tc_fence_before();

@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
             }
         }
         if (leader && !ok) {
-            raise_abort(p, s.abort);
+            raise_abort(p, s.abort, DEVERR_AT_PF_W);
             volatile int never = 0;
             for (uint32_t j = wg >= (uint32_t)S ? wg - S : 0; j < wg; ++j)
                 ptx::mbar_wait(&s.wfull[j % S], (j / S) & 1, &never, 200000000ull);
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
             }
         }
         if (leader && !ok) {
-            raise_abort(p, s.abort);
+            raise_abort(p, s.abort, DEVERR_AT_PF_X);
             volatile int never = 0;
             for (uint32_t j = wg >= (uint32_t)XS ? wg - XS : 0; j < wg; ++j)
                 ptx::mbar_wait(&s.xfull[j % XS], (j / XS) & 1, &never, 200000000ull);
@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
                 __syncwarp();
             }
         }
-        if (!ok && leader) raise_abort(p, s.abort);
+        if (!ok && leader) raise_abort(p, s.abort, DEVERR_AT_PF_MMA);
         if (leader) {
             ptx::mma_commit(s.mdone);
             volatile int never = 0;
@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
                 }
             }
         }
-        if (!ok) raise_abort(p, s.abort);
+        if (!ok) raise_abort(p, s.abort, DEVERR_AT_PF_EXP);
     } else {
         // ======================= folds =======================
         const int q = warp & 3;
@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
             }
         }
         ptx::cp_async_wait_all();
-        if (!ok) raise_abort(p, s.abort);
+        if (!ok) raise_abort(p, s.abort, DEVERR_AT_PF_FOLD);
     }
 
     ptx::tc_fence_before();

@@ -278,6 +278,10 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
         ptx::mbar_init(&sbar[0], 1);
         ptx::mbar_init(&sbar[1], p.wr * sb_parts);
         *abort_flag = 0;
+        // the x tile's barrier is armed with its bytes here, before the block-wide barrier below, so
+        // that every x copy (issued by several warps after the dependent-launch wait) completes on a
+        // barrier that already expects it
+        if (p.xsm) ptx::mbar_arrive_expect_tx(&sbar[0], (uint32_t)(NT * ckg * G * 2));
     }
     if (lane == 0)
         for (int s = 0; s < RD; ++s) ptx::mbar_init(&wfull[s], 1);
@@ -353,10 +357,8 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     ptx::pdl_wait();
 
     // ---- the CTA's x tile, one bulk copy per token row (spread over the warps) on sbar[0], armed
-    // once with the tile's bytes: a copy completing before the barrier is armed leaves its phase
-    // open, as the arming arrival is still pending ----
+    // with the tile's bytes in the prologue ----
     if (p.xsm) {
-        if (threadIdx.x == 0) ptx::mbar_arrive_expect_tx(&sbar[0], (uint32_t)(NT * ckg * G * 2));
         const int tr = warp + nwarps * lane;   // codes [cg0 G, cg1 G) of token row tr
         if (tr < NT) {
             const int64_t tok = min(tok0 + tr, p.M - 1);
@@ -366,10 +368,14 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     int issued = min(RD, nsub);   // W boxes issued on this warp's ring (warp-uniform count)
     int waited = 0;               // ... and waited for
 
-    if ((p.xsm && !ptx::mbar_wait(&sbar[0], 0, abort_flag, WAIT_NS)) ||
-        (p.sb16 && !ptx::mbar_wait(&sbar[1], 0, abort_flag, WAIT_NS))) {
-        *abort_flag = 1;
-        atomicOr(p.err, DEVERR_TIMEOUT);
+    {
+        int at = 0;
+        if (p.xsm && !ptx::mbar_wait(&sbar[0], 0, abort_flag, WAIT_NS)) at = DEVERR_AT_WARP_X;
+        else if (p.sb16 && !ptx::mbar_wait(&sbar[1], 0, abort_flag, WAIT_NS)) at = DEVERR_AT_WARP_SB;
+        if (at) {
+            atomicOr(p.err, DEVERR_TIMEOUT | (*abort_flag ? 0 : at));
+            *abort_flag = 1;
+        }
     }
     if (!p.sb16) cp_async_wait<0>();
     __syncthreads();
@@ -436,8 +442,8 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
             if (ok) {
                 waited = j + 1;
             } else if (lane == 0) {
+                atomicOr(p.err, DEVERR_TIMEOUT | (*abort_flag ? 0 : DEVERR_AT_WARP_W));
                 *abort_flag = 1;
-                atomicOr(p.err, DEVERR_TIMEOUT);
             }
         }
         uint32_t wv[4][WS];

@@ -335,7 +335,9 @@ const char* aq_last_error_message(void);
  * Reads and clears the device-side error word of the current device after
  * synchronizing `stream`.  Returns AQ_OK if no kernel recorded an error,
  * AQ_ERR_TIMEOUT if a bounded wait expired, AQ_ERR_INDEX if a row gather met an
- * id outside its table, AQ_ERR_CUDA if the read failed.
+ * id outside its table, AQ_ERR_CUDA if the read failed.  For AQ_ERR_TIMEOUT,
+ * aq_last_error_message() names the kernel and the wait that gave up first (a
+ * copy, the tensor core, or another role of the kernel).
  */
 aq_status aq_device_error(void* stream);
 

@@ -221,6 +221,7 @@ def test_bounded_wait_reports_timeout():
     with pytest.raises(aq.AQError) as ei:
         aq.aq_device_error()
     assert ei.value.name == "AQ_ERR_TIMEOUT"
+    assert "bounded-wait self-check" in str(ei.value)   # the wait that expired is named
     aq.aq_device_error()
     M, N, K, group, bits = 40, 300, 512, 64, 4
     w = inputs.normal((N, K), 0.02, seed=81)
