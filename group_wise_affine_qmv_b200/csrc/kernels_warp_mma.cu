@@ -62,9 +62,11 @@ Shape shape_for(const MmaProblem& p, int sms) {
     while (wr < wm::MAX_WARPS && ((nrt + 2 * wr - 1) / (2 * wr)) * units >= sms &&
            (int64_t)(2 * wr) * wm::ROWS * kg * 4 <= SB_MAX_BYTES)
         wr *= 2;
-    // one row block per CTA and still few CTAs: a cluster of cs CTAs splits K of each row block
+    // one row block per CTA and still few CTAs: a cluster of cs CTAs splits K of each row block.
+    // Not for short K (16 groups or fewer): there the split's two cluster barriers cost more than
+    // the second K piece per warp it saves (chained decode launches at K 1024: 7.19 against 7.45 us)
     int cs = 1;
-    if (wr == 1)
+    if (wr == 1 && kg > 16)
         while (cs < wm::MAX_CLUSTER && nrt * units * cs * 2 <= sms && kg >= 4 * cs) cs *= 2;
     const int64_t kgc = (kg + cs - 1) / cs;
     int64_t wk = wm::MAX_WARPS / wr;
