@@ -456,6 +456,21 @@ def barrier(dist, device):
     torch.cuda.synchronize(device)
 
 
+def device_error_on_any_rank(dist, stream, device):
+    """Read and clear this rank's device error word; every rank learns whether any rank had one
+    (so that all take the same next step).  Returns this rank's message, "another rank", or None."""
+    from group_wise_affine_qmv_b200 import aq
+    msg = None
+    try:
+        with torch.cuda.stream(stream):
+            aq.aq_device_error()
+    except aq.AQError as ex:
+        msg = str(ex)
+    if max_over_ranks(dist, 1.0 if msg else 0.0, device) > 0.0:
+        return msg or "another rank"
+    return None
+
+
 def graph_of(fn, stream):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
@@ -539,14 +554,12 @@ def ours(args):
                     graph.replay()
                 ev1.record(stream)
             ev1.synchronize()
-        try:
-            with torch.cuda.stream(stream):
-                aq.aq_device_error()
+        err = device_error_on_any_rank(dist, stream, device)
+        if err is None:
             break
-        except aq.AQError as ex:
-            if attempt == 1:
-                raise
-            remeasured = str(ex)
+        if attempt == 1:
+            raise RuntimeError("timed loop measured twice, a kernel reported an error both times: " + err)
+        remeasured = err
     barrier(dist, device)
     ms = ev0.elapsed_time(ev1)
     ms_max = max_over_ranks(dist, ms, device)
@@ -594,32 +607,34 @@ def ours(args):
     copy_stream = torch.cuda.Stream(device)
     done = {bits: torch.cuda.Event() for bits in BITS_LIST}
     copied = {bits: torch.cuda.Event() for bits in BITS_LIST}
-    torch.cuda.synchronize(device)
-    barrier(dist, device)
-    with torch.cuda.stream(stream):
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for step in range(e2e_steps):
-            A["h0"].copy_(h_host, non_blocking=True)
-            for bits in BITS_LIST:
-                if step > 0:
-                    stream.wait_event(copied[bits])
-                parts[bits].replay()
-                done[bits].record(stream)
-                copy_stream.wait_event(done[bits])
-                with torch.cuda.stream(copy_stream):
-                    logits_host[bits].copy_(A[bits]["logits"], non_blocking=True)
-                copied[bits].record(copy_stream)
-        for bits in BITS_LIST:
-            stream.wait_event(copied[bits])
-        f1.record(stream)
-    f1.synchronize()
     e2e_error = None
-    try:
+    for attempt in range(2):   # measured once more if a kernel reported an expired wait
+        torch.cuda.synchronize(device)
+        barrier(dist, device)
         with torch.cuda.stream(stream):
-            aq.aq_device_error()
-    except aq.AQError as ex:
-        e2e_error = str(ex)
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            for step in range(e2e_steps):
+                A["h0"].copy_(h_host, non_blocking=True)
+                for bits in BITS_LIST:
+                    if step > 0:
+                        stream.wait_event(copied[bits])
+                    parts[bits].replay()
+                    done[bits].record(stream)
+                    copy_stream.wait_event(done[bits])
+                    with torch.cuda.stream(copy_stream):
+                        logits_host[bits].copy_(A[bits]["logits"], non_blocking=True)
+                    copied[bits].record(copy_stream)
+            for bits in BITS_LIST:
+                stream.wait_event(copied[bits])
+            f1.record(stream)
+        f1.synchronize()
+        err = device_error_on_any_rank(dist, stream, device)
+        if err is None:
+            break
+        if attempt == 1:
+            raise RuntimeError("end-to-end loop measured twice, a kernel reported an error both times: " + err)
+        e2e_error = err
     del parts
     barrier(dist, device)
     e2e_ms = max_over_ranks(dist, f0.elapsed_time(f1), device)
@@ -661,7 +676,7 @@ def ours(args):
     if remeasured is not None:
         result["device_error_remeasured"] = remeasured
     if e2e_error is not None:
-        result["e2e"]["device_error"] = e2e_error
+        result["e2e"]["device_error_remeasured"] = e2e_error
     if not args.no_prefill:
         result["detail"]["prefill"] = prefill_and_moe(device, stream)
         result["detail"]["probe_and_ragged_qmv"] = probe_and_ragged(device, stream)
