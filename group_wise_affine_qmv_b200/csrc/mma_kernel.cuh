@@ -443,37 +443,18 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
     // after the wait below, and no y is written before it; W, scales and biases are constant
     // operands of the call, so their staging may start before it.
     ptx::pdl_launch_dependents();
-    // the barriers' initialisation is complete and visible to the copy engine before any copy
-    // that completes on them is issued (the same order every other copy of the kernel keeps)
-    __syncthreads();
-    int w_pre = 0;   // W stages of the first tile already issued by the W producer (warp-uniform)
     if (!p.offsets && warp == 0) {
-        // The first S W stages of the CTA's first tile go straight onto the ring, the rest of its
-        // stages and the next tile's, and
-        // the scales and biases of both, to L2, while the previous kernel in the stream may still
-        // run.  (Grouped tiles depend on the device offsets: nothing before the wait.)
-        const int rk = cs > 1 ? (int)(blockIdx.x % cs) : 0;
+        // The scales and biases of the CTA's first two tiles go to L2 while the previous kernel in
+        // the stream may still run (a prefetch changes no value that any load sees).  The W stages
+        // themselves are copied only after the wait: with W stages (or TMA prefetches of them)
+        // issued before it, a W copy sometimes never completed on some GPUs (the expanders' bounded
+        // wait expired), at a few hundred to a few thousand decode steps apart.
         const int t0 = cs > 1 ? (int)(blockIdx.x / cs) : (int)blockIdx.x;
         const int nt_all = p.n_wtiles * p.n_ttiles * p.nbatch;
-        int pw0 = 0, pw1 = NWS;
-        if (cs > 1) split_range(NWS, GPS, cs, rk, &pw0, &pw1);
-        if (t0 < nt_all) w_pre = min(S, pw1 - pw0);
         for (int k = 0; k < (cs > 1 ? 1 : 2); ++k) {
             const int t = t0 + k * (int)gridDim.x;
             if (t >= nt_all) break;
             const int64_t n0 = (int64_t)(t % p.n_wtiles) * 128;
-            if (lane == 0) {
-                for (int w = pw0; w < pw1; ++w) {
-                    if (k == 0 && w - pw0 < w_pre) {
-                        const int st = w - pw0;
-                        ptx::mbar_arrive_expect_tx(&s.wfull[st], 128u * ROWB);
-                        ptx::tma_load_2d(s.ws + (size_t)st * 128 * ROWB, &p.tw, &s.wfull[st], w * (ROWB / 4),
-                                         (int32_t)n0);
-                    } else {
-                        ptx::tma_prefetch_2d(&p.tw, w * (ROWB / 4), (int32_t)n0);
-                    }
-                }
-            }
             const int64_t nr = min64(128, p.N - n0);
             ptx::prefetch_l2_range(p.scales + n0 * p.kg, (size_t)nr * p.kg * 2, lane, 32);
             ptx::prefetch_l2_range(p.biases + n0 * p.kg, (size_t)nr * p.kg * 2, lane, 32);
@@ -534,7 +515,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 const int st = wg % S;
                 ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.wfree[st], ((wg / S) & 1) ^ 1, s.abort, WAIT_ROLE_NS));
                 if (!ok) break;
-                if (leader && wg >= (uint32_t)w_pre) {   // the first w_pre were issued before the wait
+                if (leader) {
                     // columns past K (a partial last stage) read as zero fill
                     ptx::mbar_arrive_expect_tx(&s.wfull[st], 128u * ROWB);
                     ptx::tma_load_2d(s.ws + (size_t)st * 128 * ROWB, &p.tw, &s.wfull[st], w * (ROWB / 4),
@@ -545,11 +526,9 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         }
         if (leader && !ok) {
             raise_abort(p, s.abort, DEVERR_AT_TC_WFREE);
-            // drain: the copies of every issued stage (those issued before the wait included) must
-            // land before the CTA exits
+            // drain: the copies of every issued stage must land before the CTA exits
             volatile int never = 0;
-            const uint32_t issued = wg > (uint32_t)w_pre ? wg : (uint32_t)w_pre;
-            for (uint32_t j = issued >= (uint32_t)S ? issued - S : 0; j < issued; ++j)
+            for (uint32_t j = wg >= (uint32_t)S ? wg - S : 0; j < wg; ++j)
                 ptx::mbar_wait(&s.wfull[j % S], (j / S) & 1, &never, 200000000ull);
         }
         __syncwarp();
