@@ -416,10 +416,13 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
     // 0 and 1 are X for tokens 2c and 2c + 1 of n tile t (the products are exact, the sums fp32)
     float xsum[NTL][4];
     const uint32_t ONES = BF ? 0x3F803F80u : 0x3C003C00u;   // (1, 1) in the activation dtype
-    // RMS-normalised inputs: sum of squares of this lane's x values (token 8 t + r), two chains
-    float sq[NTL][2];
+    // RMS-normalised inputs: the Gram matrix of the n tile's x rows on the tensor cores, A being the
+    // same x fragments as B (rows 8..15 of A repeat rows 0..7), so that its diagonal element
+    // (token 8 t + n, n) holds the sum of squares of token 8 t + n over the warp's K slice: lane
+    // (r = n, c = n / 2), element n % 2 (the products are exact, the sums fp32)
+    float sq[NTL][4];
 #pragma unroll
-    for (int t = 0; t < NTL; ++t) sq[t][0] = sq[t][1] = 0.0f;
+    for (int t = 0; t < NTL; ++t) sq[t][0] = sq[t][1] = sq[t][2] = sq[t][3] = 0.0f;
     int slot = 0;          // ring slot of sub-block j, and the parity of its fill
     uint32_t par = 0;
 
@@ -483,15 +486,7 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
                     mma16816<BF>(d[m][t], a[2 * m][s][0], a[2 * m + 1][s][0], a[2 * m][s][1], a[2 * m + 1][s][1],
                                  xw[2 * s], xw[2 * s + 1]);
                 mma16816<BF>(xsum[t], ONES, ONES, ONES, ONES, xw[2 * s], xw[2 * s + 1]);
-            }
-            if (p.rms) {
-#pragma unroll
-                for (int v = 0; v < XV; ++v) {
-                    float f[8];
-                    unpack8(xv[v], f, XT{});
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) sq[t][e & 1] = fmaf(f[e], f[e], sq[t][e & 1]);
-                }
+                if (p.rms) mma16816<BF>(sq[t], xw[2 * s], xw[2 * s], xw[2 * s + 1], xw[2 * s + 1], xw[2 * s], xw[2 * s + 1]);
             }
         }
 
@@ -503,6 +498,8 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
                 bv[mh] = half_bits_to_float(s_b[sb_row[mh] + g], XT{});
                 if (OFF != 0.0f) bv[mh] = fmaf(-OFF, sv[mh], bv[mh]);
             }
+            // on fp32 pairs (the two tokens of a lane's accumulator row): the same two roundings per
+            // element as one fmaf for b X and one for s D
 #pragma unroll
             for (int t = 0; t < NTL; ++t) {
                 const float2 X = make_float2(xsum[t][0], xsum[t][1]);
@@ -511,8 +508,11 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const float s = sv[2 * m + h], b = bv[2 * m + h];
-                        acc[m][t][2 * h] = fmaf(s, d[m][t][2 * h], fmaf(b, X.x, acc[m][t][2 * h]));
-                        acc[m][t][2 * h + 1] = fmaf(s, d[m][t][2 * h + 1], fmaf(b, X.y, acc[m][t][2 * h + 1]));
+                        float2 v = make_float2(acc[m][t][2 * h], acc[m][t][2 * h + 1]);
+                        v = ptx::ffma2(make_float2(b, b), X, v);
+                        v = ptx::ffma2(make_float2(s, s), make_float2(d[m][t][2 * h], d[m][t][2 * h + 1]), v);
+                        acc[m][t][2 * h] = v.x;
+                        acc[m][t][2 * h + 1] = v.y;
                     }
             }
         }
@@ -557,14 +557,9 @@ __global__ void __launch_bounds__(MAX_WARPS * 32, 2) qmm_warp_kernel(const __gri
         for (int j = waited; j < issued; ++j) ptx::mbar_wait(&wfull[j % RD], (uint32_t)((j / RD) & 1), &never, 200000000ull);
     }
     __syncwarp();
-    if (p.rms) {   // the warp's sum of squares per token (its K slice), over the 4 lanes of a row
+    if (p.rms && rw == 0 && c == (r >> 1)) {   // the warp's sum of squares per token (its K slice)
 #pragma unroll
-        for (int t = 0; t < NTL; ++t) {
-            float v = sq[t][0] + sq[t][1];
-            v += __shfl_xor_sync(0xffffffffu, v, 1);
-            v += __shfl_xor_sync(0xffffffffu, v, 2);
-            if (rw == 0 && c == 0) xsq[kw * NT + 8 * t + r] = v;
-        }
+        for (int t = 0; t < NTL; ++t) xsq[kw * NT + 8 * t + r] = (r & 1) ? sq[t][1] : sq[t][0];
     }
     {
         float* red = reinterpret_cast<float*>(ring);
@@ -696,7 +691,7 @@ cudaError_t launch_t(const WParams& p, dim3 grid, int warps, size_t smem, cudaSt
     attr[1].val.clusterDim.y = 1;
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = p.cs > 1 ? 2 : 1;   // a plain launch without a split (measured a little faster)
     return cudaLaunchKernelEx(&cfg, qmm_warp_kernel<BITS, XT, G, NTL>, p);
 }
 
