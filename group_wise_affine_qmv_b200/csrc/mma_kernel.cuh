@@ -229,14 +229,6 @@ __device__ __forceinline__ uint32_t sub1024(uint32_t v) {
     return *reinterpret_cast<const uint32_t*>(&r);
 }
 
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-    float2 r;
-    asm("add.rn.f32x2 %0, %1, %2;"
-        : "=l"(*reinterpret_cast<unsigned long long*>(&r))
-        : "l"(*reinterpret_cast<const unsigned long long*>(&a)), "l"(*reinterpret_cast<const unsigned long long*>(&b)));
-    return r;
-}
-
 template <int BITS, typename XT>
 __device__ __forceinline__ void expand32(const uint32_t* w, uint32_t* out) {
     constexpr bool BF = std::is_same<XT, bf16_t>::value;
@@ -272,7 +264,7 @@ __device__ __forceinline__ void expand32(const uint32_t* w, uint32_t* out) {
             for (int j = 0; j < 2; ++j) {
                 const float m0 = __uint_as_float(__byte_perm(w[i], 0x4B000000u, (2 * j) | (4 << 4) | (5 << 8) | (7 << 12)));
                 const float m1 = __uint_as_float(__byte_perm(w[i], 0x4B000000u, (2 * j + 1) | (4 << 4) | (5 << 8) | (7 << 12)));
-                const float2 qf = fadd2(make_float2(m0, m1), make_float2(-8388608.0f, -8388608.0f));
+                const float2 qf = ptx::fadd2(make_float2(m0, m1), make_float2(-8388608.0f, -8388608.0f));
                 const __nv_bfloat162 r = __floats2bfloat162_rn(qf.x, qf.y);
                 out[2 * i + j] = *reinterpret_cast<const uint32_t*>(&r);
             }

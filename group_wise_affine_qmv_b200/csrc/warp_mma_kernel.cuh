@@ -141,7 +141,8 @@ __device__ __forceinline__ void expand_row(const uint32_t* wv, uint32_t (*a)[2])
                 if constexpr (BF) {
                     const float m0 = __uint_as_float(__byte_perm(w, 0x4B000000u, (2 * j) | (4 << 4) | (5 << 8) | (7 << 12)));
                     const float m1 = __uint_as_float(__byte_perm(w, 0x4B000000u, (2 * j + 1) | (4 << 4) | (5 << 8) | (7 << 12)));
-                    const __nv_bfloat162 q = __floats2bfloat162_rn(m0 - 8388608.0f, m1 - 8388608.0f);
+                    const float2 qf = ptx::fadd2(make_float2(m0, m1), make_float2(-8388608.0f, -8388608.0f));
+                    const __nv_bfloat162 q = __floats2bfloat162_rn(qf.x, qf.y);
                     a[s][j] = *reinterpret_cast<const uint32_t*>(&q);
                 } else {
                     a[s][j] = f16_minus_1024(__byte_perm(w, MAGIC, (2 * j) | (5 << 4) | ((2 * j + 1) << 8) | (7 << 12)));
