@@ -17,6 +17,11 @@ __device__ __forceinline__ float half_bits_to_float(uint16_t h, bf16_t) {
 __device__ __forceinline__ float half_bits_to_float(uint16_t h, f16_t) {
     return __half2float(__ushort_as_half(h));
 }
+// fp32 -> the bits of the 16-bit type, round to nearest even (as the stores of y)
+__device__ __forceinline__ uint16_t float_to_half_bits(float v, bf16_t) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+__device__ __forceinline__ uint16_t float_to_half_bits(float v, f16_t) { return __half_as_ushort(__float2half_rn(v)); }
 
 template <typename T> __device__ __forceinline__ float to_float(const T* p);
 template <> __device__ __forceinline__ float to_float<bf16_t>(const bf16_t* p) {

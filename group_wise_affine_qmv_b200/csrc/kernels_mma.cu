@@ -82,18 +82,18 @@ Geom geometry(int bits, int group) {
 
 // Shared memory of one CTA whose K range spans at most `ms` W stages: x (that range when
 // resident, else `xst` x stages of SUB boxes), the sum-of-x table of the range, the partial
-// tile of a split, and the fixed part.
-size_t fixed_bytes(int64_t K, int64_t kg, int ms, int split, int xres, int xst, const Geom& g) {
+// tile of a split, the staged y tile (`ystg` bytes, 0 without), and the fixed part.
+size_t fixed_bytes(int64_t K, int64_t kg, int ms, int split, int xres, int xst, const Geom& g, size_t ystg) {
     const int64_t boxes = std::min<int64_t>((int64_t)ms * g.sub, K / KB);
     const int64_t groups = std::min<int64_t>((int64_t)ms * (g.wsc / (K / kg)), kg);
     return (xres ? (size_t)boxes * NT * 128 : (size_t)xst * g.sub * NT * 128) + (size_t)groups * NT * 4 +
-           (split > 1 ? (size_t)RED_BYTES : 0) + smem_fixed_bytes();
+           (split > 1 ? (size_t)RED_BYTES : 0) + ystg + smem_fixed_bytes();
 }
-size_t smem_for(int stages, int64_t K, int64_t kg, int ms, int split, int xres, int xst, const Geom& g) {
-    return (size_t)stages * 128 * g.rowb + fixed_bytes(K, kg, ms, split, xres, xst, g);
+size_t smem_for(int stages, int64_t K, int64_t kg, int ms, int split, int xres, int xst, const Geom& g, size_t ystg) {
+    return (size_t)stages * 128 * g.rowb + fixed_bytes(K, kg, ms, split, xres, xst, g, ystg);
 }
-int pick_stages(int64_t K, int64_t kg, int ms, int split, int xres, int xst, const Geom& g) {
-    const size_t fixed = fixed_bytes(K, kg, ms, split, xres, xst, g);
+int pick_stages(int64_t K, int64_t kg, int ms, int split, int xres, int xst, const Geom& g, size_t ystg = 0) {
+    const size_t fixed = fixed_bytes(K, kg, ms, split, xres, xst, g, ystg);
     if (fixed >= SMEM_LIMIT) return 0;
     int st = (int)((SMEM_LIMIT - fixed) / ((size_t)128 * g.rowb));
     if (st > MAX_STAGES) st = MAX_STAGES;
@@ -104,19 +104,19 @@ int pick_stages(int64_t K, int64_t kg, int ms, int split, int xres, int xst, con
 struct XPlan {
     int xres, xst, stages;
 };
-XPlan pick_x(const MmaProblem& p, int64_t kg, int ms, int split, const Geom& g) {
+XPlan pick_x(const MmaProblem& p, int64_t kg, int ms, int split, const Geom& g, size_t ystg) {
     XPlan r{0, 2, 0};
-    if (!p.offsets && p.M <= NT && p.nb[0] * p.nb[1] == 1 && pick_stages(p.K, kg, ms, split, 1, 0, g) >= 6) {
+    if (!p.offsets && p.M <= NT && p.nb[0] * p.nb[1] == 1 && pick_stages(p.K, kg, ms, split, 1, 0, g, ystg) >= 6) {
         r.xres = 1;
         r.xst = 0;
     } else {
         for (int xst = MAX_XST; xst > 2; --xst)
-            if (pick_stages(p.K, kg, ms, split, 0, xst, g) >= 4) {
+            if (pick_stages(p.K, kg, ms, split, 0, xst, g, ystg) >= 4) {
                 r.xst = xst;
                 break;
             }
     }
-    r.stages = pick_stages(p.K, kg, ms, split, r.xres, r.xst, g);
+    r.stages = pick_stages(p.K, kg, ms, split, r.xres, r.xst, g, ystg);
     return r;
 }
 
@@ -198,6 +198,31 @@ CUresult encode_w(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap* m, cons
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(pb.wq), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(rowb), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+// y viewed as {N, rows, nb1, nb0} bf16/f16 bits, box {128 rows of W, NT tokens}: the store of one
+// tile (TMA writes nothing outside the tensor, so a tile's rows past N and tokens past M are dropped)
+CUresult encode_y(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap* m, const MmaProblem& pb) {
+    const int64_t rows_total = pb.M;
+    cuuint64_t dims[4] = {(cuuint64_t)pb.N, (cuuint64_t)rows_total, (cuuint64_t)pb.nb[1], (cuuint64_t)pb.nb[0]};
+    const int64_t rowb = rows_total > 1 ? pb.y_row * 2 : (pb.N * 2 + 15) / 16 * 16;
+    const int64_t s1 = pb.nb[1] > 1 ? pb.yb[1] * 2 : rowb * rows_total;
+    const int64_t s2 = pb.nb[0] > 1 ? pb.yb[0] * 2 : s1 * (int64_t)pb.nb[1];
+    cuuint64_t strides[3] = {(cuuint64_t)rowb, (cuuint64_t)((s1 + 15) / 16 * 16), (cuuint64_t)((s2 + 15) / 16 * 16)};
+    cuuint32_t box[4] = {128, (cuuint32_t)NT, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, pb.y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+// Whether the tiles of y can go out as TMA stores: plain (not grouped, no split of K) calls whose y
+// has x's 16-bit type and 16-byte aligned rows and batch strides.
+bool y_tma_ok(const MmaProblem& pb, int split) {
+    if (pb.offsets || split > 1 || pb.ydt != pb.xdt) return false;
+    if (((uintptr_t)pb.y & 15) || (pb.M > 1 && pb.y_row % 8 != 0)) return false;
+    for (int i = 0; i < 2; ++i)
+        if (pb.nb[i] > 1 && pb.yb[i] % 8 != 0) return false;
+    return true;
 }
 
 void fill_common(Params& prm, const MmaProblem& pb) {
@@ -305,7 +330,16 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     const int64_t rows_all = pb.M * pb.nb[0] * pb.nb[1];
     const int split = pb.offsets ? 1 : pick_split(((pb.N + 127) / 128) * ((rows_all + NT - 1) / NT), nws, gps, sms);
     const int ms = split > 1 ? split_max_stages(nws, gps, split) : nws;
-    const XPlan xp = pick_x(pb, kg, ms, split, geo);
+    // the staged y tile takes shared memory from the W ring: only where that keeps x resident (if it
+    // was) and the ring at least 4 stages deep (or as deep as without it)
+    const XPlan xp0 = pick_x(pb, kg, ms, split, geo, 0);
+    bool ytma = y_tma_ok(pb, split);
+    XPlan xp = xp0;
+    if (ytma) {
+        const XPlan xp1 = pick_x(pb, kg, ms, split, geo, YSTG_BYTES);
+        ytma = xp1.xres == xp0.xres && (xp1.stages == xp0.stages || xp1.stages >= 4);
+        if (ytma) xp = xp1;
+    }
     const int stages = xp.stages;
     if (stages < MIN_STAGES) return cudaErrorInvalidValue;
     if (encode_x(encode, &prm.tx, pb, NT) != CUDA_SUCCESS) return cudaErrorInvalidValue;
@@ -317,6 +351,8 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     prm.stages = stages;
     prm.xres = xp.xres;
     prm.xst = xp.xst;
+    prm.ytma = ytma ? 1 : 0;
+    if (ytma && encode_y(encode, &prm.ty, pb) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     // [A block 0 | A block 1 | 2 x (WSC / group) accumulators of NT columns], a power of two >= 32
     uint32_t cols = (uint32_t)(geo.wsc + 2 * (geo.wsc / pb.group) * NT), pw = 32;
     while (pw < cols) pw <<= 1;
@@ -331,7 +367,7 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     if (pb.offsets) grid = sms;
     else if (split > 1) grid = (int)tiles * split;   // one tile per cluster
     else grid = (int)(tiles < sms ? tiles : sms);
-    const size_t smem = smem_for(stages, pb.K, kg, ms, split, xp.xres, xp.xst, geo);
+    const size_t smem = smem_for(stages, pb.K, kg, ms, split, xp.xres, xp.xst, geo, ytma ? YSTG_BYTES : 0);
     const bool bf = pb.xdt == DT::BF16;
     switch (bits) {
         case 2: return launch<2>(bf, pb.group, prm, grid, smem, stream);

@@ -51,6 +51,7 @@ __host__ __device__ constexpr uint32_t stage_swz(int rowb) {
 struct Params {
     CUtensorMap tx;  // x: 4D {K, rows, nb1, nb0} u16, box {64, NT, 1, 1}, 128-byte swizzle
     CUtensorMap tw;  // W: 2D {K*bits/32, rows} u32, box {rowb/4, 128}, swizzle by row bytes
+    CUtensorMap ty;  // y (ytma): 4D {N, M, nb1, nb0} u16, box {128, NT, 1, 1}, no swizzle
     const void* x;
     void* y;
     const uint16_t* scales;
@@ -71,6 +72,7 @@ struct Params {
     const int64_t* offsets;  // grouped mode when non-null
     int n_experts;
     int ksplit;                  // CTAs per cluster splitting each tile's K (1: no split)
+    int ytma;                    // 1: each tile's y goes out as one TMA store of a shared-memory tile
     int* err;                    // device error word (set on a timed-out wait)
 };
 
@@ -92,11 +94,12 @@ __host__ __device__ inline int split_max_stages(int nws, int gps, int cs) {
     return m < nws ? m : nws;
 }
 constexpr int RED_BYTES = FOLD_THREADS * (NT / 2) * 4;  // one CTA's partial y tile (fp32)
+constexpr int YSTG_BYTES = NT * 128 * 2;                 // a tile of y (16-bit) staged for its TMA store
 
 // shared memory besides the x buffer, the W ring and the sum-of-x table
 __host__ __device__ constexpr size_t smem_fixed_bytes() {
     return 2 * 2 * 128 * SCP * 2                                  // scale/bias chunk slots
-           + (2 * MAX_STAGES + 2 * MAX_XST + 2 * 4 + 4) * 8 + 8  // mbarriers, TMEM base, abort flag
+           + (2 * MAX_STAGES + 2 * MAX_XST + 2 * 4 + 5) * 8 + 8  // mbarriers, TMEM base, abort flag
            + (MAX_EXPERTS + 1) * 4                               // grouped tile prefix sums
            + 2 * 1024;                                           // alignment
 }

@@ -30,7 +30,10 @@
 //                i - 2 are complete; then wfree (shared-memory stage) and afull.
 //   warps 10..17 folds: thread <-> W row, two warps per lane quarter take 16 tokens each.
 //                Per stage, y += s*D' + (b - OFF*s)*X per group (tcgen05.ld of D), then dfree;
-//                per tile, the store of y.
+//                per tile, the store of y: with 16-byte aligned rows of y (ytma) the fold
+//                threads write the tile into shared memory and one of them stores it with one
+//                bulk tensor copy (element-wise 2-byte stores of scattered rows of y held the
+//                folds ~1.3 us per tile and with them the next tile's MMAs), else element stores.
 // Tensor memory: [A block 0 | A block 1 | D: 2 x GPS group accumulators of 32 columns].
 //
 // Rows of the last W tile that fall past N read TMA zero fill and the clamped last row's
@@ -88,11 +91,13 @@ struct Smem {
     uint64_t* xres_full; // resident x landed
     uint64_t* mdone;     // teardown: all MMAs retired
     uint64_t* red_full;  // split K: every rank's part of this CTA's rows has arrived (fold warps)
+    uint64_t* ybar;      // ytma: the staged y tile is written (fold threads)
     uint32_t* tmem_base;
     int* abort;
     int* prefix;         // grouped: tile prefix sums [n_experts + 1]
     float* xtab;         // [groups of this CTA's K range][NT] sums of x per group and token
     float* red;          // split K: partial sums of this CTA's rows [ranks][128 / ranks][NT] from every rank
+    uint16_t* ystg;      // ytma: [NT tokens][128 rows] of y, the source of the tile's TMA store
     uint8_t* xs;         // resident: [K/64][NT][128 B]; streamed: [xst][SUB][NT][128 B]
     uint8_t* ws;         // [stages][128 rows][ROWB]
     uint16_t* sb;        // [2 slots][2 arrays][128][SCP]
@@ -113,6 +118,8 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const Params& p, int ms) {
     q += (size_t)min(ms * GPS, p.kg) * NT * 4;
     s.red = reinterpret_cast<float*>(q);
     if (p.ksplit > 1) q += RED_BYTES;
+    s.ystg = reinterpret_cast<uint16_t*>(q);
+    if (p.ytma) q += YSTG_BYTES;
     s.sb = reinterpret_cast<uint16_t*>(q);
     q += 2 * 2 * 128 * SCP * 2;
     s.wfull = reinterpret_cast<uint64_t*>(q);
@@ -127,7 +134,8 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const Params& p, int ms) {
     s.xres_full = s.xbar + 1;
     s.mdone = s.xres_full + 1;
     s.red_full = s.mdone + 1;
-    s.tmem_base = reinterpret_cast<uint32_t*>(s.red_full + 1);
+    s.ybar = s.red_full + 1;
+    s.tmem_base = reinterpret_cast<uint32_t*>(s.ybar + 1);
     s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
     s.prefix = s.abort + 1;
     return s;
@@ -414,6 +422,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
             ptx::mbar_init(&s.sbar[i], FOLD_THREADS);
         }
         ptx::mbar_init(s.xbar, FOLD_THREADS);
+        ptx::mbar_init(s.ybar, FOLD_THREADS);
         ptx::mbar_init(s.xres_full, 1);
         ptx::mbar_init(s.mdone, 1);
         if (cs > 1) {
@@ -687,13 +696,13 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
         // ======================= folds =======================
         // Thread <-> W row; warps q and q + 4 take 16 tokens each.  Per stage:
         // y += s*D'_g + (b - OFF*s)*X_g for each of its groups, then release the stage's
-        // accumulators.  Per tile: store y.
+        // accumulators.  Per tile: store y (staged tile and one TMA store, or element stores).
         const int q = warp & 3;
         const int th = (warp - 2 - EXP_WARPS) >> 2;
         const int row = 32 * q + lane;
         const int tid = threadIdx.x - 32 * (2 + EXP_WARPS);   // 0..255
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        uint32_t wg = 0, xph = 0;
+        uint32_t wg = 0, xph = 0, ytile = 0;
         int unit = 0;
         bool ok = true;
         int at = DEVERR_AT_TC_FOLD;   // which wait gave up
@@ -737,8 +746,11 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
             for (int i = 0; i < H / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
             for (int w = w0; w < w1; ++w, ++wg) {
                 if ((w - w0) % CS_W == 0) {
-                    // this stage opens a scale/bias chunk: its copies were issued a chunk earlier
+                    // this stage opens a scale/bias chunk: its copies were issued a chunk earlier.
+                    // (ytma: every tile opens with a chunk, and the store of the previous tile's y has
+                    // read the staging tile before any fold thread passes this barrier)
                     ptx::cp_async_wait_all();
+                    if (p.ytma && tid == 0) ptx::bulk_wait_read_all();
                     ptx::mbar_arrive(&s.sbar[unit & 1]);
                     ok = __all_sync(0xffffffffu,
                                     ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_ROLE_NS));
@@ -826,6 +838,28 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
                 }
                 break;   // one tile per cluster
             }
+            if (p.ytma) {
+                // ---- the tile's y: every fold thread writes its row of its half of the tokens into
+                //      the staging tile, then one thread stores the tile with TMA (rows past N and
+                //      tokens past M fall outside the tensor map and are not written) ----
+                uint16_t* stg = s.ystg + row;
+#pragma unroll
+                for (int i = 0; i < H / 2; ++i) {
+                    const int tok = th * H + 2 * i;
+                    stg[tok * 128] = float_to_half_bits(acc[i].x, XT{});
+                    stg[(tok + 1) * 128] = float_to_half_bits(acc[i].y, XT{});
+                }
+                ptx::fence_proxy_async();
+                ptx::mbar_arrive(s.ybar);
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.ybar, ytile & 1, s.abort, WAIT_ROLE_NS));
+                ++ytile;
+                if (!ok) break;
+                if (tid == 0) {
+                    ptx::tma_store_4d(&p.ty, s.ystg, (int32_t)ti.n0, (int32_t)ti.xrow0, ti.b1, ti.b0);
+                    ptx::bulk_commit_group();
+                }
+                continue;
+            }
             // ---- this thread's row of y for its half of the tokens ----
             if (row < ti.nvalid) {
                 const int64_t n = ti.n0 + row;
@@ -840,6 +874,7 @@ __global__ void __launch_bounds__(THREADS, 1) qmm_tc_kernel(const __grid_constan
             }
         }
         ptx::cp_async_wait_all();
+        if (p.ytma && tid == 0) ptx::bulk_wait_all();   // every tile's store is complete before the CTA exits
         if (!ok) raise_abort(p, s.abort, at);
     }
 
