@@ -200,25 +200,27 @@ CUresult encode_w(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap* m, cons
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
-// y viewed as {N, rows, nb1, nb0} bf16/f16 bits, box {128 rows of W, NT tokens}: the store of one
-// tile (TMA writes nothing outside the tensor, so a tile's rows past N and tokens past M are dropped)
-CUresult encode_y(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap* m, const MmaProblem& pb) {
+// y viewed as {N, rows, nb1, nb0} bf16/f16 bits, box {128 rows of W, `box_rows` tokens}: the store of
+// one tile (TMA writes nothing outside the tensor, so a tile's rows past N and tokens past M are dropped)
+CUresult encode_y(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap* m, const MmaProblem& pb, int box_rows) {
     const int64_t rows_total = pb.M;
     cuuint64_t dims[4] = {(cuuint64_t)pb.N, (cuuint64_t)rows_total, (cuuint64_t)pb.nb[1], (cuuint64_t)pb.nb[0]};
     const int64_t rowb = rows_total > 1 ? pb.y_row * 2 : (pb.N * 2 + 15) / 16 * 16;
     const int64_t s1 = pb.nb[1] > 1 ? pb.yb[1] * 2 : rowb * rows_total;
     const int64_t s2 = pb.nb[0] > 1 ? pb.yb[0] * 2 : s1 * (int64_t)pb.nb[1];
     cuuint64_t strides[3] = {(cuuint64_t)rowb, (cuuint64_t)((s1 + 15) / 16 * 16), (cuuint64_t)((s2 + 15) / 16 * 16)};
-    cuuint32_t box[4] = {128, (cuuint32_t)NT, 1, 1};
+    cuuint32_t box[4] = {128, (cuuint32_t)box_rows, 1, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, pb.y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
 // Whether the tiles of y can go out as TMA stores: plain (not grouped, no split of K) calls whose y
-// has x's 16-bit type and 16-byte aligned rows and batch strides.
+// has x's 16-bit type, 16-byte aligned rows and batch strides, and N a multiple of 8 (a tile store
+// writes whole 16-byte pieces of a row: on this B200 a piece that straddles N was written in full,
+// past the end of the row)
 bool y_tma_ok(const MmaProblem& pb, int split) {
-    if (pb.offsets || split > 1 || pb.ydt != pb.xdt) return false;
+    if (pb.offsets || split > 1 || pb.ydt != pb.xdt || pb.N % 8 != 0) return false;
     if (((uintptr_t)pb.y & 15) || (pb.M > 1 && pb.y_row % 8 != 0)) return false;
     for (int i = 0; i < 2; ++i)
         if (pb.nb[i] > 1 && pb.yb[i] % 8 != 0) return false;
@@ -273,10 +275,23 @@ cudaError_t launch_prefill_problem(const MmaProblem& pb, cudaStream_t stream) {
     const int rowb = pb.group * pb.bits / 8;
     const size_t xstage = (size_t)sub * NTP * 128, wstage = (size_t)128 * rowb;
     const int xst = sub == 1 ? 4 : 3;
-    const size_t fixed = (size_t)xst * xstage + p_fixed_bytes();
+    size_t fixed = (size_t)xst * xstage + p_fixed_bytes();
     if (fixed + 4 * wstage > SMEM_LIMIT) return cudaErrorInvalidValue;
     int stages = (int)((SMEM_LIMIT - fixed) / wstage);
     if (stages > P_MAX_STAGES) stages = P_MAX_STAGES;
+    // the staged y tile (32 KB) takes shared memory from the W ring where that leaves it at least
+    // 8 stages deep (or as deep as without it)
+    bool ytma = y_tma_ok(pb, 1);
+    if (ytma) {
+        const size_t f1 = fixed + P_YSTG_BYTES;
+        int s1 = f1 + 4 * wstage <= SMEM_LIMIT ? (int)((SMEM_LIMIT - f1) / wstage) : 0;
+        if (s1 > P_MAX_STAGES) s1 = P_MAX_STAGES;
+        ytma = s1 >= 4 && (s1 == stages || s1 >= 8);
+        if (ytma) {
+            fixed = f1;
+            stages = s1;
+        }
+    }
     if (encode_x(encode, &prm.tx, pb, NTP) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     if (encode_w(encode, &prm.tw, pb, rowb) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     fill_common(prm, pb);
@@ -284,6 +299,8 @@ cudaError_t launch_prefill_problem(const MmaProblem& pb, cudaStream_t stream) {
     prm.n_wstages = (int)(pb.K / pb.group);
     prm.stages = stages;
     prm.xst = xst;
+    prm.ytma = ytma ? 1 : 0;
+    if (ytma && encode_y(encode, &prm.ty, pb, NTP) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     prm.tmem_cols = 512;   // [A block 0 | A block 1 | 2 accumulators of 128 columns]
     prm.idesc = ptx::idesc_f16(NTP, pb.xdt == DT::BF16 ? 1 : 0);
     cudaError_t e = device_pointers(prm);
@@ -352,7 +369,7 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     prm.xres = xp.xres;
     prm.xst = xp.xst;
     prm.ytma = ytma ? 1 : 0;
-    if (ytma && encode_y(encode, &prm.ty, pb) != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    if (ytma && encode_y(encode, &prm.ty, pb, NT) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     // [A block 0 | A block 1 | 2 x (WSC / group) accumulators of NT columns], a power of two >= 32
     uint32_t cols = (uint32_t)(geo.wsc + 2 * (geo.wsc / pb.group) * NT), pw = 32;
     while (pw < cols) pw <<= 1;

@@ -30,7 +30,8 @@
 //                i - 2 are complete; then wfree (shared-memory stage) and afull.
 //   warps 10..17 folds: thread <-> W row, two warps per lane quarter take 16 tokens each.
 //                Per stage, y += s*D' + (b - OFF*s)*X per group (tcgen05.ld of D), then dfree;
-//                per tile, the store of y: with 16-byte aligned rows of y (ytma) the fold
+//                per tile, the store of y: with 16-byte aligned rows of y and N a multiple of
+//                8 (ytma) the fold
 //                threads write the tile into shared memory and one of them stores it with one
 //                bulk tensor copy (element-wise 2-byte stores of scattered rows of y held the
 //                folds ~1.3 us per tile and with them the next tile's MMAs), else element stores.

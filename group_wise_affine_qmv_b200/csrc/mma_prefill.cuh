@@ -18,7 +18,9 @@
 //   warps 6..13  folds: thread <-> W row, warps q and q + 4 take 64 tokens each.  Per stage,
 //                X_g of the 128 tokens is summed from the x block in shared memory (fp32, k
 //                order) by all fold threads, then y += s*D' + (b - OFF*s)*X_g; the x slot and
-//                the accumulator are released.  Per tile, the store of y.
+//                the accumulator are released.  Per tile, the store of y: staged in shared
+//                memory and stored with one bulk tensor copy (N a multiple of 8, 16-byte aligned
+//                rows of y), else element stores.
 // Tiles are walked W-tile-fastest, so the CTAs in flight share one token tile (x from L2) and
 // the whole packed W stays in L2 across token tiles.
 #pragma once
@@ -40,9 +42,11 @@ struct PSmem {
     uint64_t* sbar;      // [2] scale/bias chunk slots (fold threads)
     uint64_t* xgbar;     // [2] sums of x of a stage written (fold threads)
     uint64_t* mdone;
+    uint64_t* ybar;      // ytma: the staged y tile is written (fold threads)
     uint32_t* tmem_base;
     int* abort;
     float* xg;           // [2][NTP] sums of x of a stage
+    uint16_t* ystg;      // ytma: [NTP tokens][128 rows] of y, the source of the tile's TMA store
     uint8_t* xs;         // [xst][SUB][NTP][128 B]
     uint8_t* ws;         // [stages][128][ROWB]
     uint16_t* sb;        // [2 slots][2 arrays][128][SCP]
@@ -61,6 +65,8 @@ __device__ __forceinline__ PSmem p_carve(uint8_t* base, const Params& p) {
     q += 2 * 2 * 128 * SCP * 2;
     s.xg = reinterpret_cast<float*>(q);
     q += 2 * NTP * 4;
+    s.ystg = reinterpret_cast<uint16_t*>(q);
+    if (p.ytma) q += P_YSTG_BYTES;
     s.wfull = reinterpret_cast<uint64_t*>(q);
     s.wfree = s.wfull + P_MAX_STAGES;
     s.xfull = s.wfree + P_MAX_STAGES;
@@ -71,7 +77,8 @@ __device__ __forceinline__ PSmem p_carve(uint8_t* base, const Params& p) {
     s.sbar = s.dfree + 2;
     s.xgbar = s.sbar + 2;
     s.mdone = s.xgbar + 2;
-    s.tmem_base = reinterpret_cast<uint32_t*>(s.mdone + 1);
+    s.ybar = s.mdone + 1;
+    s.tmem_base = reinterpret_cast<uint32_t*>(s.ybar + 1);
     s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
     return s;
 }
@@ -147,6 +154,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
             ptx::mbar_init(&s.xgbar[i], P_FOLD_THREADS);
         }
         ptx::mbar_init(s.mdone, 1);
+        ptx::mbar_init(s.ybar, P_FOLD_THREADS);
         *s.abort = 0;
         ptx::fence_mbar_init();
     }
@@ -311,7 +319,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
         const int row = 32 * q + lane;
         const int tid = threadIdx.x - 32 * (2 + P_EXP);   // 0..255
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        uint32_t wg = 0;
+        uint32_t wg = 0, ytile = 0;
         int unit = 0;
         bool ok = true;
         if ((int)blockIdx.x < ntiles) p_issue_sb(p, p_tile(p, blockIdx.x), 0, s.sb, tid);
@@ -325,8 +333,11 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
             for (int i = 0; i < H / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
             for (int w = 0; w < NWS; ++w, ++wg) {
                 if (w % SCW == 0) {
-                    // this stage opens a scale/bias chunk: its copies were issued a chunk earlier
+                    // this stage opens a scale/bias chunk: its copies were issued a chunk earlier.
+                    // (ytma: every tile opens with a chunk, and the store of the previous tile's y has
+                    // read the staging tile before any fold thread passes this barrier)
                     ptx::cp_async_wait_all();
+                    if (p.ytma && tid == 0) ptx::bulk_wait_read_all();
                     ptx::mbar_arrive(&s.sbar[unit & 1]);
                     ok = __all_sync(0xffffffffu,
                                     ptx::mbar_wait(&s.sbar[unit & 1], (unit >> 1) & 1, s.abort, WAIT_NS));
@@ -397,6 +408,28 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
                 if (lane == 0) ptx::mbar_arrive(&s.dfree[slot]);
             }
             if (!ok) break;
+            if (p.ytma) {
+                // ---- the tile's y: every fold thread writes its row of its 64 tokens into the
+                //      staging tile, then one thread stores the tile with TMA (rows past N and
+                //      tokens past M fall outside the tensor map and are not written) ----
+                uint16_t* stg = s.ystg + row;
+#pragma unroll
+                for (int i = 0; i < H / 2; ++i) {
+                    const int tok = th * H + 2 * i;
+                    stg[tok * 128] = float_to_half_bits(acc[i].x, XT{});
+                    stg[(tok + 1) * 128] = float_to_half_bits(acc[i].y, XT{});
+                }
+                ptx::fence_proxy_async();
+                ptx::mbar_arrive(s.ybar);
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(s.ybar, ytile & 1, s.abort, WAIT_NS));
+                ++ytile;
+                if (!ok) break;
+                if (tid == 0) {
+                    ptx::tma_store_4d(&p.ty, s.ystg, (int32_t)ti.n0, (int32_t)ti.xrow0, ti.b1, ti.b0);
+                    ptx::bulk_commit_group();
+                }
+                continue;
+            }
             // ---- this thread's row of y for its 64 tokens ----
             if (row < ti.nvalid) {
                 const int64_t off = ti.xrow0 * p.y_row + ti.n0 + row + (int64_t)ti.b0 * p.yb[0] + (int64_t)ti.b1 * p.yb[1];
@@ -409,6 +442,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
             }
         }
         ptx::cp_async_wait_all();
+        if (p.ytma && tid == 0) ptx::bulk_wait_all();   // every tile's store is complete before the CTA exits
         if (!ok) raise_abort(p, s.abort, DEVERR_AT_PF_FOLD);
     }
 

@@ -70,6 +70,42 @@ def test_prefill_batched_views():
     assert np.all(row_errors(y, oracle_linear_view(x, Q.dequant())) <= 4e-3)
 
 
+@pytest.mark.parametrize("xdtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("group", [64, 128])
+@pytest.mark.parametrize("M,N", [(200, 1000), (128, 128), (70, 300), (70, 1)])
+def test_prefill_y_tile_store_stays_inside_y(xdtype, group, M, N):
+    """With N a multiple of 8 and 16-byte aligned rows of y each 128 x 128 tile leaves as one bulk
+    tensor store of a shared-memory tile (N 300 and 1: element stores): guard columns and rows around
+    a strided y keep their value, ragged tiles write nothing outside y, batch elements of a padded
+    batched y stay apart, and the values are bitwise those of the element-wise stores taken when y's
+    row stride is not a multiple of 8."""
+    K, bits = 1024, 4
+    sd = dtype_name(torch.empty(0, dtype=xdtype))
+    w = inputs.normal((N, K), 0.02, seed=M + N + group)
+    Q, (wq, sc, bi) = _q(w, group, bits, sd)
+    x = inputs.normal((M, K), 1.0, xdtype, seed=M * 5 + N)
+    xd = x.to(DEV)
+    pitch = (N + 15) // 8 * 8 + 8                  # row stride a multiple of 8 elements: tile stores
+    buf = torch.full((M + 2, pitch + 8), 3072.0, dtype=xdtype, device=DEV)
+    y = buf[1:M + 1, 8:8 + N]
+    assert aq.aq_plan_linear(xd, wq, sc, bi, group, bits, y)["kernel"] == "tc_prefill"
+    aq.aq_qmm_t(xd, wq, sc, bi, group, bits, out=y)
+    b = buf.float().cpu()
+    assert torch.all(b[0] == 3072.0) and torch.all(b[-1] == 3072.0)
+    assert torch.all(b[:, :8] == 3072.0) and torch.all(b[:, 8 + N:] == 3072.0)
+    assert np.all(row_errors(y, oracle_linear_view(x, Q.dequant())) <= 4e-3)
+    odd = torch.full((M, N + 1), 3072.0, dtype=xdtype, device=DEV)[:, :N]   # stride N + 1: element stores
+    aq.aq_qmm_t(xd, wq, sc, bi, group, bits, out=odd)
+    assert torch.equal(odd, y)
+    xb = inputs.normal((2, M, K), 1.0, xdtype, seed=M + 9).to(DEV)
+    ybuf = torch.full((2, M + 3, pitch), 3072.0, dtype=xdtype, device=DEV)
+    yb = ybuf[:, :M, :N]
+    aq.aq_qmm_t(xb, wq, sc, bi, group, bits, out=yb)
+    assert torch.all(ybuf[:, M:].float() == 3072.0) and torch.all(ybuf[:, :, N:].float() == 3072.0)
+    for i in range(2):
+        assert torch.equal(yb[i], aq.aq_qmm_t(xb[i].contiguous(), wq, sc, bi, group, bits))
+
+
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("shape", ["up", "down"])
 def test_prefill_full_size_every_batch_element(bits, shape):
