@@ -167,7 +167,10 @@ aq_status aq_dequantize_rows(const aq_view* wq, const aq_view* scales, const aq_
  * tensor-core kernels are launched as programmatic dependents of the previous
  * kernel in the stream: their set-up and (warp-level kernel) the staging of
  * the weights overlap it, x is read only after it completed (see "Weights are
- * constant operands" above).
+ * constant operands" above).  Where y has x's dtype, N is a multiple of 8 and
+ * y's rows and batch strides are 16-byte aligned, the tcgen05 kernels write
+ * each tile of y as one bulk tensor copy from shared memory (nothing outside
+ * y's [.., M, N] is written); elsewhere they store y element by element.
  * Data pointers must be 16-byte aligned.
  */
 aq_status aq_qmm_t(const aq_view* x, const aq_view* wq, const aq_view* scales,
