@@ -312,18 +312,24 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# the sources the warp-level kernel is compiled from (its translation units and every csrc header
+# they include): its committed DRAM counters stay valid while these are unchanged
+WARP_KERNEL_SOURCES = ("aq_internal.h", "device_common.cuh", "kernels_warp_mma.cu", "kernels_warp_mma_b2.cu",
+                       "kernels_warp_mma_b4.cu", "kernels_warp_mma_b8.cu", "sm100_ptx.cuh", "warp_mma.cuh",
+                       "warp_mma_kernel.cuh")
+
+
 def committed_traffic(kernel_tag: str):
     """Per-launch DRAM bytes of `kernel_tag` from the committed ncu summary, if the
-    kernel source has not changed since the capture (source hash recorded there)."""
+    kernel's sources have not changed since the capture (their hash is recorded there)."""
     import hashlib
     summ = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(summ):
         return None
     src_hash = hashlib.sha256()
-    for name in sorted(os.listdir(os.path.join(ROOT, "group_wise_affine_qmv_b200", "csrc"))):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(ROOT, "group_wise_affine_qmv_b200", "csrc", name), "rb") as f:
-                src_hash.update(f.read())
+    for name in WARP_KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "group_wise_affine_qmv_b200", "csrc", name), "rb") as f:
+            src_hash.update(f.read())
     cur = src_hash.hexdigest()[:16]
     for line in open(summ):
         parts = line.split()

@@ -117,7 +117,7 @@ constexpr int P_YSTG_BYTES = NTP * 128 * 2;               // a tile of y (16-bit
 constexpr int P_MAX_XST = 4;
 // scale/bias slots, the two sums-of-x rows, mbarriers, TMEM base, abort flag, alignment
 __host__ __device__ constexpr size_t p_fixed_bytes() {
-    return 2 * 2 * 128 * SCP * 2 + 2 * NTP * 4 + (2 * P_MAX_STAGES + 2 * P_MAX_XST + 2 * 5 + 2) * 8 + 8 + 2 * 1024;
+    return 2 * 2 * 128 * SCP * 2 + 2 * NTP * 4 + (2 * P_MAX_STAGES + 2 * P_MAX_XST + 2 * 6 + 2) * 8 + 8 + 2 * 1024;
 }
 }  // namespace pf
 

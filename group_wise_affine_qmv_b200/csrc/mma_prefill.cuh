@@ -40,7 +40,7 @@ struct PSmem {
     uint64_t* sdone;     // [2] (commit)
     uint64_t* dfree;     // [2] (fold warps)
     uint64_t* sbar;      // [2] scale/bias chunk slots (fold threads)
-    uint64_t* xgbar;     // [2] sums of x of a stage written (fold threads)
+    uint64_t* xgbar;     // [2 token halves][2] sums of x of a stage written (the half's fold threads)
     uint64_t* mdone;
     uint64_t* ybar;      // ytma: the staged y tile is written (fold threads)
     uint32_t* tmem_base;
@@ -76,7 +76,7 @@ __device__ __forceinline__ PSmem p_carve(uint8_t* base, const Params& p) {
     s.dfree = s.sdone + 2;
     s.sbar = s.dfree + 2;
     s.xgbar = s.sbar + 2;
-    s.mdone = s.xgbar + 2;
+    s.mdone = s.xgbar + 4;
     s.ybar = s.mdone + 1;
     s.tmem_base = reinterpret_cast<uint32_t*>(s.ybar + 1);
     s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
@@ -151,7 +151,8 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
             ptx::mbar_init(&s.sdone[i], 1);
             ptx::mbar_init(&s.dfree[i], P_FOLD);
             ptx::mbar_init(&s.sbar[i], P_FOLD_THREADS);
-            ptx::mbar_init(&s.xgbar[i], P_FOLD_THREADS);
+            ptx::mbar_init(&s.xgbar[i], P_FOLD_THREADS / 2);
+            ptx::mbar_init(&s.xgbar[2 + i], P_FOLD_THREADS / 2);
         }
         ptx::mbar_init(s.mdone, 1);
         ptx::mbar_init(s.ybar, P_FOLD_THREADS);
@@ -376,8 +377,9 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
                     const float other = __shfl_xor_sync(0xffffffffu, sum, 1);
                     if (half == 0) s.xg[slot * NTP + tok] = sum + other;
                 }
-                ptx::mbar_arrive(&s.xgbar[slot]);
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.xgbar[slot], (wg >> 1) & 1, s.abort, WAIT_NS));
+                // the sums of a token half are written and read by that half's four fold warps only
+                ptx::mbar_arrive(&s.xgbar[2 * th + slot]);
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s.xgbar[2 * th + slot], (wg >> 1) & 1, s.abort, WAIT_NS));
                 if (!ok) break;
                 if (lane == 0) ptx::mbar_arrive(&s.xfree[xs]);   // x block read by this warp
                 // ---- y += s * D' + (b - OFF*s) * X_g ----
