@@ -47,7 +47,7 @@ class AqPlan(ctypes.Structure):
                 ("x_batch_stride", ctypes.c_int64 * 2), ("y_batch_stride", ctypes.c_int64 * 2),
                 ("w_batch_stride", ctypes.c_int64 * 2), ("s_batch_stride", ctypes.c_int64 * 2),
                 ("b_batch_stride", ctypes.c_int64 * 2), ("x_row_stride", ctypes.c_int64),
-                ("y_row_stride", ctypes.c_int64), ("total_rows", ctypes.c_int64)]
+                ("y_row_stride", ctypes.c_int64), ("total_rows", ctypes.c_int64), ("y_tiles", ctypes.c_int32)]
 
 
 EXPORTED = ("aq_quantize", "aq_dequantize", "aq_dequantize_rows", "aq_qmv", "aq_qmm_t", "aq_qmm_t_grouped", "aq_qmv_gathered", "aq_qmm_t_multi",
@@ -292,7 +292,7 @@ def aq_plan_linear(x, wq, scales, biases, group: int, bits: int, y, force_qmv: b
                 K=p.K, nbatch_dims=p.nbatch_dims, batch_shape=tuple(p.batch_shape),
                 x_batch_stride=tuple(p.x_batch_stride), y_batch_stride=tuple(p.y_batch_stride),
                 w_batch_stride=tuple(p.w_batch_stride), x_row_stride=p.x_row_stride, y_row_stride=p.y_row_stride,
-                total_rows=p.total_rows, note=note)
+                total_rows=p.total_rows, y_tiles=bool(p.y_tiles), note=note)
 
 
 def aq_device_error(device=None):

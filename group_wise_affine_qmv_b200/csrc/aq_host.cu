@@ -314,6 +314,7 @@ aq_status resolve_linear(const aq_view* x, const aq_view* wq, const aq_view* sc,
     }
     P.regime = R->mma_ok ? AQ_REGIME_MMA : AQ_REGIME_QMV;
     P.kernel = R->mma_ok ? (int32_t)aq::mma_kernel_for(R->mp) : AQ_KERNEL_GEMV;
+    P.y_tiles = R->mma_ok && aq::mma_y_tiles(R->mp) ? 1 : 0;
     return AQ_OK;
 }
 

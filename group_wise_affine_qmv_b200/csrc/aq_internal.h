@@ -107,6 +107,8 @@ cudaError_t launch_mma(const MmaProblem& p, cudaStream_t s);
 // Which tensor-core kernel launch_mma runs for a supported problem.
 enum class MmaKernel : int { WARP = AQ_KERNEL_WARP_MMA, SMALL_M = AQ_KERNEL_TC_SMALL_M, PREFILL = AQ_KERNEL_TC_PREFILL };
 MmaKernel mma_kernel_for(const MmaProblem& p);
+// whether the tcgen05 kernel chosen for p writes each tile of y with one bulk tensor store
+bool mma_y_tiles(const MmaProblem& p);
 
 // Warp-level (mma.sync) kernel for up to 32 rows per launch batch: whether it takes the problem
 // (given that mma_supported accepted it) and its launch.

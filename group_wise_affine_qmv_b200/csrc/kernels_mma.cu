@@ -265,33 +265,55 @@ bool prefill_eligible(const MmaProblem& pb) {
     return !pb.offsets && pb.M >= 64 && (pb.group == 64 || pb.group == 128);
 }
 
+// Shared memory plan of the prefill kernel for a problem: x ring depth, W ring depth and whether
+// the tiles of y are staged for bulk tensor stores
+struct PrefillPlan {
+    bool ok;
+    int xst, stages;
+    size_t fixed, wstage;
+    bool ytma;
+};
+PrefillPlan plan_prefill(const MmaProblem& pb) {
+    using namespace pf;
+    PrefillPlan r{};
+    const int sub = pb.group / KB;
+    const int rowb = pb.group * pb.bits / 8;
+    const size_t xstage = (size_t)sub * NTP * 128;
+    r.wstage = (size_t)128 * rowb;
+    r.xst = sub == 1 ? 4 : 3;
+    r.fixed = (size_t)r.xst * xstage + p_fixed_bytes();
+    if (r.fixed + 4 * r.wstage > SMEM_LIMIT) return r;
+    r.ok = true;
+    r.stages = (int)((SMEM_LIMIT - r.fixed) / r.wstage);
+    if (r.stages > P_MAX_STAGES) r.stages = P_MAX_STAGES;
+    // the staged y tile (32 KB) takes shared memory from the W ring where that leaves it at least
+    // 8 stages deep (or as deep as without it)
+    r.ytma = y_tma_ok(pb, 1);
+    if (r.ytma) {
+        const size_t f1 = r.fixed + P_YSTG_BYTES;
+        int s1 = f1 + 4 * r.wstage <= SMEM_LIMIT ? (int)((SMEM_LIMIT - f1) / r.wstage) : 0;
+        if (s1 > P_MAX_STAGES) s1 = P_MAX_STAGES;
+        r.ytma = s1 >= 4 && (s1 == r.stages || s1 >= 8);
+        if (r.ytma) {
+            r.fixed = f1;
+            r.stages = s1;
+        }
+    }
+    return r;
+}
+
 cudaError_t launch_prefill_problem(const MmaProblem& pb, cudaStream_t stream) {
     auto encode = get_encode();
     if (!encode) return cudaErrorNotSupported;
     using namespace pf;
     Params prm;
     memset(&prm, 0, sizeof prm);
-    const int sub = pb.group / KB;
     const int rowb = pb.group * pb.bits / 8;
-    const size_t xstage = (size_t)sub * NTP * 128, wstage = (size_t)128 * rowb;
-    const int xst = sub == 1 ? 4 : 3;
-    size_t fixed = (size_t)xst * xstage + p_fixed_bytes();
-    if (fixed + 4 * wstage > SMEM_LIMIT) return cudaErrorInvalidValue;
-    int stages = (int)((SMEM_LIMIT - fixed) / wstage);
-    if (stages > P_MAX_STAGES) stages = P_MAX_STAGES;
-    // the staged y tile (32 KB) takes shared memory from the W ring where that leaves it at least
-    // 8 stages deep (or as deep as without it)
-    bool ytma = y_tma_ok(pb, 1);
-    if (ytma) {
-        const size_t f1 = fixed + P_YSTG_BYTES;
-        int s1 = f1 + 4 * wstage <= SMEM_LIMIT ? (int)((SMEM_LIMIT - f1) / wstage) : 0;
-        if (s1 > P_MAX_STAGES) s1 = P_MAX_STAGES;
-        ytma = s1 >= 4 && (s1 == stages || s1 >= 8);
-        if (ytma) {
-            fixed = f1;
-            stages = s1;
-        }
-    }
+    const PrefillPlan pl = plan_prefill(pb);
+    if (!pl.ok) return cudaErrorInvalidValue;
+    const int xst = pl.xst, stages = pl.stages;
+    const bool ytma = pl.ytma;
+    const size_t fixed = pl.fixed, wstage = pl.wstage;
     if (encode_x(encode, &prm.tx, pb, NTP) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     if (encode_w(encode, &prm.tw, pb, rowb) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     fill_common(prm, pb);
@@ -327,6 +349,52 @@ MmaKernel mma_kernel_for(const MmaProblem& pb) {
     return MmaKernel::SMALL_M;
 }
 
+namespace {
+
+// Plan of the small-M kernel for a problem: split of K over a cluster, x residency and ring
+// depths, and whether the tiles of y are staged for bulk tensor stores
+struct SmallMPlan {
+    int split, ms;
+    XPlan xp;
+    bool ytma;
+};
+SmallMPlan plan_small_m(const MmaProblem& pb) {
+    SmallMPlan r{};
+    const int64_t kg = pb.K / pb.group;
+    const Geom geo = geometry(pb.bits, pb.group);
+    const int nws = (int)((pb.K + geo.wsc - 1) / geo.wsc);
+    const int gps = geo.wsc / pb.group;
+    // The split depends on the total rows, not on how they are grouped into launch batches, so
+    // that a strided view and its contiguous copy take the same split (and give the same bits).
+    const int64_t rows_all = pb.M * pb.nb[0] * pb.nb[1];
+    r.split = pb.offsets ? 1 : pick_split(((pb.N + 127) / 128) * ((rows_all + NT - 1) / NT), nws, gps, num_sms());
+    r.ms = r.split > 1 ? split_max_stages(nws, gps, r.split) : nws;
+    // the staged y tile takes shared memory from the W ring: only where that keeps x resident (if it
+    // was) and the ring at least 4 stages deep (or as deep as without it)
+    const XPlan xp0 = pick_x(pb, kg, r.ms, r.split, geo, 0);
+    r.ytma = y_tma_ok(pb, r.split);
+    r.xp = xp0;
+    if (r.ytma) {
+        const XPlan xp1 = pick_x(pb, kg, r.ms, r.split, geo, YSTG_BYTES);
+        r.ytma = xp1.xres == xp0.xres && (xp1.stages == xp0.stages || xp1.stages >= 4);
+        if (r.ytma) r.xp = xp1;
+    }
+    return r;
+}
+
+}  // namespace
+
+bool mma_y_tiles(const MmaProblem& pb) {
+    switch (mma_kernel_for(pb)) {
+        case MmaKernel::PREFILL: {
+            const PrefillPlan pl = plan_prefill(pb);
+            return pl.ok && pl.ytma;
+        }
+        case MmaKernel::SMALL_M: return plan_small_m(pb).ytma;
+        default: return false;
+    }
+}
+
 cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     const MmaKernel kind = mma_kernel_for(pb);
     if (kind == MmaKernel::PREFILL) return launch_prefill_problem(pb, stream);
@@ -342,21 +410,10 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     const int gps = geo.wsc / pb.group;
     const int sms = num_sms();
     const int64_t tiles = pb.offsets ? 0 : ((pb.N + 127) / 128) * ((pb.M + NT - 1) / NT) * pb.nb[0] * pb.nb[1];
-    // The split depends on the total rows, not on how they are grouped into launch batches, so
-    // that a strided view and its contiguous copy take the same split (and give the same bits).
-    const int64_t rows_all = pb.M * pb.nb[0] * pb.nb[1];
-    const int split = pb.offsets ? 1 : pick_split(((pb.N + 127) / 128) * ((rows_all + NT - 1) / NT), nws, gps, sms);
-    const int ms = split > 1 ? split_max_stages(nws, gps, split) : nws;
-    // the staged y tile takes shared memory from the W ring: only where that keeps x resident (if it
-    // was) and the ring at least 4 stages deep (or as deep as without it)
-    const XPlan xp0 = pick_x(pb, kg, ms, split, geo, 0);
-    bool ytma = y_tma_ok(pb, split);
-    XPlan xp = xp0;
-    if (ytma) {
-        const XPlan xp1 = pick_x(pb, kg, ms, split, geo, YSTG_BYTES);
-        ytma = xp1.xres == xp0.xres && (xp1.stages == xp0.stages || xp1.stages >= 4);
-        if (ytma) xp = xp1;
-    }
+    const SmallMPlan pl = plan_small_m(pb);
+    const int split = pl.split, ms = pl.ms;
+    const XPlan xp = pl.xp;
+    const bool ytma = pl.ytma;
     const int stages = xp.stages;
     if (stages < MIN_STAGES) return cudaErrorInvalidValue;
     if (encode_x(encode, &prm.tx, pb, NT) != CUDA_SUCCESS) return cudaErrorInvalidValue;

@@ -318,6 +318,8 @@ typedef struct aq_plan {
     int64_t x_row_stride;      /* elements between folded rows                         */
     int64_t y_row_stride;
     int64_t total_rows;        /* product of batch_shape * M                           */
+    int32_t y_tiles;           /* 1: a tcgen05 kernel writes each tile of y with one   */
+                               /*    bulk tensor store from shared memory              */
 } aq_plan;
 
 /*

@@ -132,6 +132,53 @@ def test_mma_y_tile_store_stays_inside_y(xdtype, M, N):
         assert torch.equal(yb[i], aq.aq_qmm_t(xb[i].contiguous(), wq, sc, bi, group, bits))
 
 
+def _plan(x, wq, sc, bi, group, bits, y=None):
+    if y is None:
+        y = torch.empty(tuple(x.shape[:-1]) + (wq.shape[-2],), dtype=x.dtype)
+    return aq.aq_plan_linear(x, wq, sc, bi, group, bits, y)
+
+
+def _empty_weights(N, K, bits, group, dtype=torch.bfloat16):
+    """Uninitialised weight views: the plan reads shapes, strides and pointers only."""
+    return (torch.empty(N, K * bits // 32, dtype=torch.int32), torch.empty(N, K // group, dtype=dtype),
+            torch.empty(N, K // group, dtype=dtype))
+
+
+def test_plan_reports_tile_stores_of_y():
+    """Where the tcgen05 kernels write each tile of y with one bulk tensor store: y in x's 16-bit
+    dtype, N a multiple of 8, 16-byte aligned rows and batch strides, no split of K over a cluster,
+    and (prefill) room in shared memory; elsewhere element stores.  The warp-level kernel and the
+    GEMV never do.  (A host-side plan on CPU tensors; the tensor-core kernels are planned only
+    where the driver offers cuTensorMapEncodeTiled, hence a GPU test.)"""
+    K = 1024
+    lm = _empty_weights(151936, K, 4, 64)
+    x32 = torch.zeros(32, 1, K, dtype=torch.bfloat16)
+    p = _plan(x32, *lm, 64, 4)
+    assert p["kernel"] == "tc_small_m" and p["y_tiles"], p
+    p = _plan(x32, *lm, 64, 4, y=torch.empty(32, 1, 151936, dtype=torch.float32))
+    assert p["kernel"] == "tc_small_m" and not p["y_tiles"]        # fp32 y
+    odd = _empty_weights(151932 + 1, K, 4, 64)
+    assert not _plan(x32, *odd, 64, 4)["y_tiles"]                      # N not a multiple of 8
+    ypad = torch.empty(32, 151936 + 4, dtype=torch.bfloat16)[:, :151936].unsqueeze(1)
+    assert not _plan(x32, *lm, 64, 4, y=ypad)["y_tiles"]               # row stride not a multiple of 8
+    small = _empty_weights(304, K, 4, 64)
+    p = _plan(torch.zeros(40, K, dtype=torch.bfloat16), *small, 64, 4)
+    assert p["kernel"] == "tc_small_m" and not p["y_tiles"]          # few tiles: K split over a cluster
+    up = _empty_weights(4096, K, 4, 64)
+    xp = torch.zeros(2, 128, K, dtype=torch.bfloat16)
+    p = _plan(xp, *up, 64, 4)
+    assert p["kernel"] == "tc_prefill" and p["y_tiles"], p
+    p = _plan(xp.half(), *_empty_weights(4096, K, 8, 64, torch.float16), 64, 8)
+    assert p["kernel"] == "tc_prefill" and p["y_tiles"], p
+    # groups of 128: the 32 KB staging tile would leave the W ring too shallow
+    p = _plan(xp, *_empty_weights(4096, K, 4, 128), 128, 4)
+    assert p["kernel"] == "tc_prefill" and not p["y_tiles"], p
+    assert not _plan(xp, *_empty_weights(4100, K, 4, 64), 64, 4)["y_tiles"]
+    assert _plan(torch.zeros(8, K, dtype=torch.bfloat16), *up, 64, 4)["kernel"] == "warp_mma"
+    assert not _plan(torch.zeros(8, K, dtype=torch.bfloat16), *up, 64, 4)["y_tiles"]
+    assert not _plan(torch.zeros(2, K, dtype=torch.bfloat16), *up, 64, 4)["y_tiles"]   # GEMV
+
+
 @pytest.mark.parametrize("bits", [4, 8])
 def test_mma_matches_gemv_numerics(bits):
     """The two regimes agree with each other to the same bar (different kernels)."""

@@ -75,7 +75,8 @@ def test_prefill_batched_views():
 @pytest.mark.parametrize("M,N", [(200, 1000), (128, 128), (70, 300), (70, 1)])
 def test_prefill_y_tile_store_stays_inside_y(xdtype, group, M, N):
     """With N a multiple of 8 and 16-byte aligned rows of y each 128 x 128 tile leaves as one bulk
-    tensor store of a shared-memory tile (N 300 and 1: element stores): guard columns and rows around
+    tensor store of a shared-memory tile (groups of 64; N 300 and 1, and groups of 128, whose W
+    ring would get too shallow, take element stores): guard columns and rows around
     a strided y keep their value, ragged tiles write nothing outside y, batch elements of a padded
     batched y stay apart, and the values are bitwise those of the element-wise stores taken when y's
     row stride is not a multiple of 8."""
