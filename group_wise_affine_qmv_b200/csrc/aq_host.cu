@@ -91,9 +91,10 @@ bool overlaps(const aq_view* a, const aq_view* b) {
 bool self_overlapping(const aq_view* v) {
     int idx[4];
     int n = 0;
-    for (int i = 0; i < v->rank; ++i)
+    for (int i = 0; i < v->rank && i < 4; ++i)   // (ranks above 4 are rejected before)
         if (v->shape[i] > 1) idx[n++] = i;
-    std::sort(idx, idx + n, [&](int a, int b) { return v->stride[a] < v->stride[b]; });
+    for (int j = 1; j < n; ++j)                   // by stride, ascending (at most 4 entries)
+        for (int k = j; k > 0 && v->stride[idx[k]] < v->stride[idx[k - 1]]; --k) std::swap(idx[k], idx[k - 1]);
     int64_t reach = 0;
     for (int j = 0; j < n; ++j) {
         const int i = idx[j];

@@ -407,7 +407,6 @@ cudaError_t launch_mma(const MmaProblem& pb, cudaStream_t stream) {
     const int64_t kg = pb.K / pb.group;
     const Geom geo = geometry(bits, pb.group);
     const int nws = (int)((pb.K + geo.wsc - 1) / geo.wsc);
-    const int gps = geo.wsc / pb.group;
     const int sms = num_sms();
     const int64_t tiles = pb.offsets ? 0 : ((pb.N + 127) / 128) * ((pb.M + NT - 1) / NT) * pb.nb[0] * pb.nb[1];
     const SmallMPlan pl = plan_small_m(pb);
