@@ -64,3 +64,22 @@ def test_reference_arm_line_on_rank0():
     assert line["unit"] == "GB/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_committed_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
+    """The roofline's DRAM traffic is reported only while the warp-level kernel's sources hash to
+    the value recorded with the capture: the committed tree matches, and any edit of one of those
+    sources (a copy of the tree here) makes the number disappear."""
+    import shutil
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.committed_traffic("qmm_warp_kernel_decode_chain") is not None
+    assert bench.committed_traffic("no_such_kernel") is None
+    root = tmp_path / "repo"
+    shutil.copytree(os.path.join(ROOT, "profiles"), root / "profiles")
+    shutil.copytree(os.path.join(ROOT, "group_wise_affine_qmv_b200", "csrc"), root / "group_wise_affine_qmv_b200" / "csrc")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.committed_traffic("qmm_warp_kernel_decode_chain") is not None
+    src = root / "group_wise_affine_qmv_b200" / "csrc" / "warp_mma_kernel.cuh"
+    src.write_text(src.read_text() + "\n// edited\n")
+    assert bench.committed_traffic("qmm_warp_kernel_decode_chain") is None
