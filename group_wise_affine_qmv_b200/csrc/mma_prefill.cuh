@@ -413,7 +413,8 @@ __global__ void __launch_bounds__(P_THREADS, 1) qmm_prefill_kernel(const __grid_
             if (p.ytma) {
                 // ---- the tile's y: every fold thread writes its row of its 64 tokens into the
                 //      staging tile, then one thread stores the tile with TMA (rows past N and
-                //      tokens past M fall outside the tensor map and are not written) ----
+                //      tokens past M fall outside the tensor map and are not written; N is a multiple
+                //      of 8, so a row's end is a 16-byte boundary of the store) ----
                 uint16_t* stg = s.ystg + row;
 #pragma unroll
                 for (int i = 0; i < H / 2; ++i) {
